@@ -1,0 +1,177 @@
+"""CPU oracle for dynamic block-sparse attention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s cpu_baseline /
+reference arm import this package.  The product library (``video_dit_dynamic_b200``)
+never imports it and shares no code with it.
+
+This module only marshals numpy arrays into ``liboracle.so``, compiled with gcc from
+``sbsa_oracle.c``, which holds all of the oracle's arithmetic (fp64, two-pass softmax).
+The method it follows is described in that file's header: block means of Q and K
+(page "知识卡片：600倍加速，720p视频实时生成！单卡也能带的动14B模型", 方法/产品要点,
+bullet 动态稀疏量化注意力), keep-top blocks with the diagonal forced, and dense
+softmax attention inside the kept blocks (page "单卡 RTX 5090 跑 Wan2.2-A14B：720p
+视频生成只要 3.8 秒", 四步拆解 item 3).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sbsa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+F32, BF16, F64 = 0, 1, 2
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so with gcc (-O2, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+                               "-fno-fast-math", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        lib.oracle_pool.argtypes = [I, I, I, I, I, I, P, I, P]
+        lib.oracle_pool.restype = None
+        lib.oracle_score_row.argtypes = [I, I, P, P, I, P, P]
+        lib.oracle_score_row.restype = None
+        lib.oracle_select.argtypes = [I, I, I, I, I, P, P, P, P]
+        lib.oracle_select.restype = I
+        lib.oracle_attention.argtypes = [I, I, I, I, I, I, P, P, P, I, P, P,
+                                         ctypes.c_double, ctypes.c_long, P, P]
+        lib.oracle_attention.restype = I
+        lib.oracle_set_threads.argtypes = [I]
+        lib.oracle_threads_used.restype = I
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _as_input(x) -> tuple[np.ndarray, int]:
+    """Return a C-contiguous numpy view and its dtype code.
+
+    bf16 data is passed as its raw uint16 bit patterns (numpy has no bf16)."""
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float32:
+        return x, F32
+    if x.dtype == np.uint16:
+        return x, BF16
+    if x.dtype == np.float64:
+        return x, F64
+    raise TypeError(f"oracle input dtype {x.dtype} not supported (float32, float64, bf16-as-uint16)")
+
+
+def set_threads(n: int) -> None:
+    _load().oracle_set_threads(int(n))
+
+
+def threads_used() -> int:
+    return int(_load().oracle_threads_used())
+
+
+def num_blocks(Lp: int, blk: int) -> int:
+    return Lp // blk
+
+
+def pool(x, L: int, blk: int) -> np.ndarray:
+    """Block means over valid tokens.  x: [B,H,Lp,d] -> [B,H,nb,d] float64."""
+    xa, dt = _as_input(x)
+    B, H, Lp, d = xa.shape
+    nb = Lp // blk
+    out = np.empty((B, H, nb, d), dtype=np.float64)
+    _load().oracle_pool(B, H, L, Lp, d, blk, _ptr(xa), dt, _ptr(out))
+    return out
+
+
+def score_row(qmean_bh: np.ndarray, kmean_bh: np.ndarray, i: int):
+    """Scores s_j = <qmean_i, kmean_j> and a_j = sum |products| for one query block."""
+    qm = np.ascontiguousarray(qmean_bh, dtype=np.float64)
+    km = np.ascontiguousarray(kmean_bh, dtype=np.float64)
+    nb, d = km.shape
+    s = np.empty(nb, dtype=np.float64)
+    a = np.empty(nb, dtype=np.float64)
+    _load().oracle_score_row(nb, d, _ptr(qm), _ptr(km), int(i), _ptr(s), _ptr(a))
+    return s, a
+
+
+def select(qmean: np.ndarray, kmean: np.ndarray, k: int, want_kth: bool = False):
+    """Diagonal + top-(k-1) per query block, ascending.  Returns col_idx [B,H,nb,k]
+    (int32) and, if asked, the per-row score of the last kept non-diagonal block."""
+    qm = np.ascontiguousarray(qmean, dtype=np.float64)
+    km = np.ascontiguousarray(kmean, dtype=np.float64)
+    B, H, nb, d = qm.shape
+    col = np.empty((B, H, nb, k), dtype=np.int32)
+    kth = np.empty((B, H, nb), dtype=np.float64) if want_kth else None
+    rc = _load().oracle_select(B, H, nb, d, int(k), _ptr(qm), _ptr(km), _ptr(col),
+                               _ptr(kth) if want_kth else None)
+    if rc != 0:
+        raise ValueError(f"oracle_select failed (rc={rc}, k={k}, nb={nb})")
+    return (col, kth) if want_kth else col
+
+
+def uniform_row_ptr(B: int, H: int, nb: int, k: int) -> np.ndarray:
+    return (np.arange(B * H * nb + 1, dtype=np.int64) * k).astype(np.int32)
+
+
+def attention(q, k, v, L: int, blk: int, row_ptr: np.ndarray, col_idx: np.ndarray,
+              scale: float = 0.0, units=None) -> np.ndarray:
+    """Softmax attention over the kept blocks, fp64.
+
+    units: None for every (b,h,query block), else a list of unit ids bh*nb + i.
+    Returns [B,H,Lp,d] (units=None) or [len(units), blk, d]."""
+    qa, dt = _as_input(q)
+    ka, dt2 = _as_input(k)
+    va, dt3 = _as_input(v)
+    if not (dt == dt2 == dt3):
+        raise TypeError("q, k, v must share a dtype")
+    B, H, Lp, d = qa.shape
+    nb = Lp // blk
+    rp = np.ascontiguousarray(row_ptr, dtype=np.int32).reshape(-1)
+    ci = np.ascontiguousarray(col_idx, dtype=np.int32).reshape(-1)
+    if units is None:
+        out = np.empty((B, H, Lp, d), dtype=np.float64)
+        n_units, up = B * H * nb, None
+    else:
+        ua = np.ascontiguousarray(units, dtype=np.int64)
+        out = np.empty((len(ua), blk, d), dtype=np.float64)
+        n_units, up = len(ua), _ptr(ua)
+    rc = _load().oracle_attention(B, H, L, Lp, d, blk, _ptr(qa), _ptr(ka), _ptr(va), dt,
+                                  _ptr(rp), _ptr(ci), float(scale), n_units, up, _ptr(out))
+    if rc != 0:
+        raise MemoryError("oracle_attention failed")
+    return out
+
+
+def keep_blocks(nb: int, keep_fraction: float) -> int:
+    """k = round-half-up(keep * nb), clamped to [1, nb] (the reading of 'keep about
+    10-20% of the blocks' as a per-query-block count)."""
+    k = int(np.floor(keep_fraction * nb + 0.5))
+    return max(1, min(nb, k))
+
+
+def forward(q, k, v, L: int, blk: int, k_keep: int, scale: float = 0.0):
+    """pool -> select -> attend.  Returns (out [B,H,Lp,d], col_idx, qmean, kmean)."""
+    qm = pool(q, L, blk)
+    km = pool(k, L, blk)
+    col = select(qm, km, k_keep)
+    B, H, nb, _ = qm.shape
+    rp = uniform_row_ptr(B, H, nb, k_keep)
+    out = attention(q, k, v, L, blk, rp, col, scale)
+    return out, col, qm, km

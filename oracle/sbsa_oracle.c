@@ -1,0 +1,234 @@
+/*
+ * CPU oracle for dynamic block-sparse self-attention -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Only tests/, __graft_entry__.smoke() and bench.py's cpu_baseline / reference arm
+ * may load or run this file.  The product path (the sm_100a library under
+ * video_dit_dynamic_b200/) shares no code with it and never calls it.
+ *
+ * What it computes is the plain definition of the method, step by step, in fp64:
+ *
+ *   [Card]  = page "知识卡片：600倍加速，720p视频实时生成！单卡也能带的动14B模型",
+ *             section 方法/产品要点, bullet 动态稀疏量化注意力
+ *   [Guide] = page "单卡 RTX 5090 跑 Wan2.2-A14B：720p 视频生成只要 3.8 秒",
+ *             section 四步拆解, item 3 动态稀疏注意力
+ *
+ *   1. pool    ([Card], [Guide]): block-level MEANS of Query and of Key are the
+ *              cheap importance estimate.  Mean over the valid tokens of a block.
+ *   2. select  ([Card], [Guide]): keep only ~10-20% of the key blocks for each query
+ *              block.  Reading taken here: score(i,j) = <qmean_i, kmean_j>, the
+ *              diagonal block j == i is always kept and counts toward k, the other
+ *              k-1 are the largest scores, ties broken by the lower block index.
+ *              The kept list is written in ascending block order.
+ *   3. attend  ([Guide]): the kept blocks are computed densely.  Softmax attention
+ *              of each query row over exactly the valid keys of its kept blocks,
+ *              non-causal, scale 1/sqrt(d) unless given.  Two-pass softmax (max,
+ *              then exp-sums), not the online form.
+ *
+ * Inputs are read as fp32, bf16 (raw 16-bit patterns, converted exactly) or fp64.
+ * Tensors are row-major [B][H][Lp][d]; means are [B][H][nb][d]; col_idx is
+ * [B][H][nb][k].  Padded tokens t >= L are ignored as keys and their query rows
+ * produce 0.
+ *
+ * Parity pins live in tests/test_oracle_pins.py.  Every function below is pinned there.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_F64 = 2 };
+
+static int g_threads = 0; /* 0: OpenMP default */
+
+void oracle_set_threads(int n) { g_threads = n; }
+
+int oracle_threads_used(void) {
+#ifdef _OPENMP
+    return g_threads > 0 ? g_threads : omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+static double elem(const void *x, int dtype, size_t i) {
+    if (dtype == ORC_F32) return (double)((const float *)x)[i];
+    if (dtype == ORC_BF16) {
+        uint32_t bits = (uint32_t)((const uint16_t *)x)[i] << 16;
+        float f;
+        memcpy(&f, &bits, sizeof f);
+        return (double)f;
+    }
+    return ((const double *)x)[i];
+}
+
+/* Step 1: block means over valid tokens.  out[(bh*nb + i)*d + c]. */
+void oracle_pool(int B, int H, int L, int Lp, int d, int blk,
+                 const void *x, int dtype, double *out) {
+    int nb = Lp / blk;
+    long rows = (long)B * H * nb;
+#pragma omp parallel for schedule(static) num_threads(oracle_threads_used())
+    for (long r = 0; r < rows; ++r) {
+        long bh = r / nb;
+        int i = (int)(r % nb);
+        int t0 = i * blk;
+        int t1 = t0 + blk < L ? t0 + blk : L;
+        for (int c = 0; c < d; ++c) {
+            double s = 0.0;
+            for (int t = t0; t < t1; ++t)
+                s += elem(x, dtype, ((size_t)bh * Lp + t) * d + c);
+            out[r * d + c] = t1 > t0 ? s / (double)(t1 - t0) : 0.0;
+        }
+    }
+}
+
+/* Step 2, part a: one row of the block-score matrix, s_j = sum_c qm[i,c]*km[j,c],
+ * and a_j = sum_c |qm[i,c]*km[j,c]| (the magnitude that bounds its rounding error). */
+void oracle_score_row(int nb, int d, const double *qmean_bh, const double *kmean_bh,
+                      int i, double *score, double *absum) {
+    for (int j = 0; j < nb; ++j) {
+        double s = 0.0, a = 0.0;
+        for (int c = 0; c < d; ++c) {
+            double p = qmean_bh[(size_t)i * d + c] * kmean_bh[(size_t)j * d + c];
+            s += p;
+            a += fabs(p);
+        }
+        score[j] = s;
+        if (absum) absum[j] = a;
+    }
+}
+
+typedef struct { double s; int j; } cand_t;
+
+/* Descending score; equal scores: lower block index first. */
+static int by_score_desc(const void *pa, const void *pb) {
+    const cand_t *a = (const cand_t *)pa, *b = (const cand_t *)pb;
+    if (a->s > b->s) return -1;
+    if (a->s < b->s) return 1;
+    return (a->j > b->j) - (a->j < b->j);
+}
+
+static int by_int_asc(const void *pa, const void *pb) {
+    int a = *(const int *)pa, b = *(const int *)pb;
+    return (a > b) - (a < b);
+}
+
+/* Step 2, part b: diagonal plus the top k-1 of the rest, written ascending.
+ * kth_score (nullable) receives, per row, the score of the last kept non-diagonal
+ * block (or -inf when k == 1). */
+int oracle_select(int B, int H, int nb, int d, int k,
+                  const double *qmean, const double *kmean,
+                  int32_t *col_idx, double *kth_score) {
+    if (k < 1 || k > nb) return 1;
+    long rows = (long)B * H * nb;
+    int fail = 0;
+#pragma omp parallel num_threads(oracle_threads_used())
+    {
+        double *score = (double *)malloc(sizeof(double) * (size_t)nb);
+        cand_t *cand = (cand_t *)malloc(sizeof(cand_t) * (size_t)nb);
+        int *keep = (int *)malloc(sizeof(int) * (size_t)k);
+        if (!score || !cand || !keep) {
+#pragma omp atomic write
+            fail = 1;
+        } else {
+#pragma omp for schedule(static)
+            for (long r = 0; r < rows; ++r) {
+                long bh = r / nb;
+                int i = (int)(r % nb);
+                oracle_score_row(nb, d, qmean + (size_t)bh * nb * d,
+                                 kmean + (size_t)bh * nb * d, i, score, NULL);
+                int n = 0;
+                for (int j = 0; j < nb; ++j)
+                    if (j != i) { cand[n].s = score[j]; cand[n].j = j; ++n; }
+                qsort(cand, (size_t)n, sizeof(cand_t), by_score_desc);
+                keep[0] = i;
+                for (int q = 0; q < k - 1; ++q) keep[q + 1] = cand[q].j;
+                qsort(keep, (size_t)k, sizeof(int), by_int_asc);
+                for (int q = 0; q < k; ++q) col_idx[r * k + q] = keep[q];
+                if (kth_score) kth_score[r] = k > 1 ? cand[k - 2].s : -INFINITY;
+            }
+        }
+        free(score);
+        free(cand);
+        free(keep);
+    }
+    return fail ? 2 : 0;
+}
+
+/* Step 3: attention of one (b,h,query block) unit over its kept blocks.
+ * out: [blk][d]; rows t >= L are 0.  Two passes: the max, then the exp sums. */
+static void attend_unit(int L, int Lp, int d, int blk, long bh, int i,
+                        const void *q, const void *kx, const void *v, int dtype,
+                        const int32_t *cols, int ncols, double scale,
+                        double *logit, double *out) {
+    int nkeys = ncols * blk;
+    for (int r = 0; r < blk; ++r) {
+        int t = i * blk + r;
+        double *o = out + (size_t)r * d;
+        for (int c = 0; c < d; ++c) o[c] = 0.0;
+        if (t >= L) continue;
+        size_t qrow = ((size_t)bh * Lp + t) * d;
+        double m = -INFINITY;
+        for (int n = 0; n < nkeys; ++n) {
+            int u = cols[n / blk] * blk + n % blk;
+            logit[n] = -INFINITY;
+            if (u >= L) continue;
+            size_t krow = ((size_t)bh * Lp + u) * d;
+            double s = 0.0;
+            for (int c = 0; c < d; ++c)
+                s += elem(q, dtype, qrow + c) * elem(kx, dtype, krow + c);
+            logit[n] = s * scale;
+            if (logit[n] > m) m = logit[n];
+        }
+        if (m == -INFINITY) continue; /* no valid key kept: output stays 0 */
+        double den = 0.0;
+        for (int n = 0; n < nkeys; ++n) {
+            if (logit[n] == -INFINITY) continue;
+            int u = cols[n / blk] * blk + n % blk;
+            size_t vrow = ((size_t)bh * Lp + u) * d;
+            double p = exp(logit[n] - m);
+            den += p;
+            for (int c = 0; c < d; ++c) o[c] += p * elem(v, dtype, vrow + c);
+        }
+        for (int c = 0; c < d; ++c) o[c] /= den;
+    }
+}
+
+/* Step 3 over a list of units (unit = bh*nb + i), or all units when units == NULL.
+ * CSR: row_ptr[unit]..row_ptr[unit+1] index col_idx.  out: [n_units][blk][d]. */
+int oracle_attention(int B, int H, int L, int Lp, int d, int blk,
+                     const void *q, const void *k, const void *v, int dtype,
+                     const int32_t *row_ptr, const int32_t *col_idx, double scale,
+                     long n_units, const int64_t *units, double *out) {
+    int nb = Lp / blk;
+    if (scale == 0.0) scale = 1.0 / sqrt((double)d);
+    if (!units) n_units = (long)B * H * nb;
+    int maxcols = 0;
+    for (long u = 0; u < (long)B * H * nb; ++u) {
+        int n = row_ptr[u + 1] - row_ptr[u];
+        if (n > maxcols) maxcols = n;
+    }
+    int fail = 0;
+#pragma omp parallel num_threads(oracle_threads_used())
+    {
+        double *logit = (double *)malloc(sizeof(double) * (size_t)(maxcols > 0 ? maxcols : 1) * blk);
+        if (!logit) {
+#pragma omp atomic write
+            fail = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long n = 0; n < n_units; ++n) {
+                long unit = units ? (long)units[n] : n;
+                long bh = unit / nb;
+                int i = (int)(unit % nb);
+                int a = row_ptr[unit], b = row_ptr[unit + 1];
+                attend_unit(L, Lp, d, blk, bh, i, q, k, v, dtype, col_idx + a, b - a,
+                            scale, logit, out + (size_t)n * blk * d);
+            }
+        }
+        free(logit);
+    }
+    return fail ? 2 : 0;
+}

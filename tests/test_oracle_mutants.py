@@ -1,0 +1,100 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case below plants one mistake in a copy of oracle/sbsa_oracle.c (a text edit,
+compiled with gcc into a temporary library, on the CPU), swaps it in for the real
+oracle, and runs every pin in test_oracle_pins.py.  At least one pin must fail for
+each mutant; the real oracle passes them all.
+"""
+import ctypes
+import inspect
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "sbsa_oracle.c")
+
+MUTANTS = {
+    # pool divides by the block size instead of the number of valid tokens
+    "pool_divides_by_block": ("s / (double)(t1 - t0)", "s / (double)blk"),
+    # pool also averages the padded tokens
+    "pool_counts_padding": ("int t1 = t0 + blk < L ? t0 + blk : L;", "int t1 = t0 + blk;"),
+    # score uses a transposed operand (key block i against query block j)
+    "score_transposed": ("qmean_bh[(size_t)i * d + c] * kmean_bh[(size_t)j * d + c]",
+                         "qmean_bh[(size_t)j * d + c] * kmean_bh[(size_t)i * d + c]"),
+    # ties broken toward the higher block index
+    "ties_to_higher_index": ("return (a->j > b->j) - (a->j < b->j);",
+                             "return (a->j < b->j) - (a->j > b->j);"),
+    # the diagonal competes like any other block instead of being forced
+    "diagonal_not_forced": ("if (j != i) { cand[n].s", "if (1) { cand[n].s"),
+    # attention forgets to mask padded keys
+    "padded_keys_kept": ("if (u >= L) continue;\n            size_t krow", "size_t krow"),
+    # softmax without the max subtraction
+    "no_max_subtraction": ("double p = exp(logit[n] - m);", "double p = exp(logit[n]);"),
+    # off-by-one in the gather of the kept block's tokens
+    "gather_off_by_one": ("int u = cols[n / blk] * blk + n % blk;\n            logit[n]",
+                          "int u = cols[n / blk] * blk + (n + 1) % blk;\n            logit[n]"),
+    # the scale is dropped
+    "scale_dropped": ("logit[n] = s * scale;", "logit[n] = s;"),
+}
+
+
+def _build_mutant(tmp_path, name, old, new):
+    text = open(SRC).read()
+    assert text.count(old) == 1, f"mutation anchor for {name} not unique/present"
+    path = tmp_path / f"{name}.c"
+    path.write_text(text.replace(old, new))
+    so = tmp_path / f"{name}.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+                           str(path), "-o", str(so), "-lm"])
+    return str(so)
+
+
+def _pin_functions():
+    out = []
+    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+        if not name.startswith("test_"):
+            continue
+        marks = getattr(fn, "pytestmark", [])
+        params = [m for m in marks if m.name == "parametrize"]
+        if params:
+            argname, values = params[0].args[0], params[0].args[1]
+            for val in values:
+                out.append((f"{name}[{val}]", fn, {argname: val}))
+        else:
+            out.append((name, fn, {}))
+    return out
+
+
+def _run_pins_with(lib_path):
+    saved = oracle._lib
+    oracle._lib = None
+    real_build = oracle.build
+    oracle.build = lambda force=False: lib_path
+    failed = []
+    try:
+        for name, fn, kw in _pin_functions():
+            try:
+                fn(**kw)
+            except Exception:  # AssertionError, or ValueError from a broken selection
+                failed.append(name)
+    finally:
+        oracle.build = real_build
+        oracle._lib = saved
+    return failed
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(tmp_path, name):
+    old, new = MUTANTS[name]
+    so = _build_mutant(tmp_path, name, old, new)
+    failed = _run_pins_with(so)
+    assert failed, f"mutant {name} passed every pin"
+
+
+def test_real_oracle_passes_all_pins():
+    assert _run_pins_with(oracle.build()) == []
+    assert ctypes  # keep import

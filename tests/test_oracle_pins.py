@@ -1,0 +1,310 @@
+"""Pins for the CPU oracle: each check comes from something other than the oracle.
+
+Sources of truth used here:
+  * the hand-computed 4-block example in tests/golden/four_block_example.json;
+  * closed forms (constant inputs, uniform softmax when Q = 0, block-indicator V);
+  * special cases that reduce to a library routine (keep every block -> dense softmax
+    attention, computed by torch's fp64 scaled_dot_product_attention);
+  * the defining property of a top-k (every kept score >= every dropped one, ties to
+    the lower index) and invariances (permuting keys inside a block).
+
+Each is chosen so that a plausible mistake in the oracle -- dividing by the block size
+instead of the valid-token count, counting padded keys, dropping the max subtraction,
+a transposed operand, an off-by-one in the block gather, a wrong tie order -- fails at
+least one test.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from video_dit_dynamic_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "four_block_example.json")
+
+
+def _golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def _arr(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+def _as4(x):  # [L, d] -> [1, 1, L, d]
+    return _arr(x)[None, None]
+
+
+def _sdpa(q, k, v, scale, key_mask=None):
+    """Dense softmax attention in fp64 via torch's library routine."""
+    tq, tk, tv = (torch.from_numpy(np.asarray(a, dtype=np.float64)) for a in (q, k, v))
+    mask = None if key_mask is None else torch.from_numpy(key_mask)
+    return torch.nn.functional.scaled_dot_product_attention(
+        tq, tk, tv, attn_mask=mask, scale=scale).numpy()
+
+
+# ---------------------------------------------------------------- pool
+
+def test_pool_hand_example():
+    g = _golden()
+    qm = oracle.pool(_as4(g["Q"]), g["L"], g["blk"])
+    km = oracle.pool(_as4(g["K"]), g["L"], g["blk"])
+    np.testing.assert_array_equal(qm[0, 0], _arr(g["qmean"]))
+    np.testing.assert_array_equal(km[0, 0], _arr(g["kmean"]))
+
+
+def test_pool_partial_last_block_ignores_padding():
+    g = _golden()
+    p = g["partial_block"]
+    Q = _arr(g["Q"]).copy()
+    K = _arr(g["K"]).copy()
+    Q[7] = p["Q_row7_junk"]
+    K[7] = p["K_row7_junk"]
+    qm = oracle.pool(Q[None, None], p["L"], g["blk"])
+    km = oracle.pool(K[None, None], p["L"], g["blk"])
+    np.testing.assert_array_equal(qm[0, 0], _arr(p["qmean"]))
+    np.testing.assert_array_equal(km[0, 0], _arr(p["kmean"]))
+
+
+def test_pool_block_constant_input():
+    B, H, nb, blk, d = 2, 3, 5, 4, 8
+    rng = np.random.default_rng(7)
+    c = rng.normal(size=(B, H, nb, d))
+    x = np.repeat(c, blk, axis=2)  # every token of block i equals c[..., i, :]
+    L = nb * blk - 3               # partial last block: still the constant
+    np.testing.assert_allclose(oracle.pool(x, L, blk), c, rtol=0, atol=1e-15)
+
+
+def test_pool_reads_bf16_bits_exactly():
+    # bf16 patterns for 1.0, -2.0, 0.5, 3.0 (sign | exponent | 7-bit mantissa)
+    bits = np.array([0x3F80, 0xC000, 0x3F00, 0x4040], dtype=np.uint16).reshape(1, 1, 4, 1)
+    qm = oracle.pool(bits, 4, 2)
+    np.testing.assert_array_equal(qm.reshape(-1), [(1.0 - 2.0) / 2, (0.5 + 3.0) / 2])
+
+
+# ---------------------------------------------------------------- select
+
+def test_select_hand_example_with_ties():
+    g = _golden()
+    qm, km = _arr(g["qmean"])[None, None], _arr(g["kmean"])[None, None]
+    for i in range(4):
+        s, _ = oracle.score_row(qm[0, 0], km[0, 0], i)
+        np.testing.assert_array_equal(s, _arr(g["scores"][i]))
+    np.testing.assert_array_equal(oracle.select(qm, km, 2)[0, 0], g["col_idx_k2"])
+    np.testing.assert_array_equal(oracle.select(qm, km, 3)[0, 0], g["col_idx_k3"])
+
+
+def test_select_k_all_and_k_one():
+    rng = np.random.default_rng(1)
+    qm = rng.normal(size=(1, 2, 9, 4))
+    km = rng.normal(size=(1, 2, 9, 4))
+    np.testing.assert_array_equal(oracle.select(qm, km, 9), np.broadcast_to(np.arange(9), (1, 2, 9, 9)))
+    np.testing.assert_array_equal(oracle.select(qm, km, 1)[..., 0], np.broadcast_to(np.arange(9), (1, 2, 9)))
+
+
+def test_select_is_a_topk_with_diagonal():
+    """Defining property: ascending, contains i, and every kept off-diagonal score is
+    >= every dropped score (strictly greater, or equal with a lower index)."""
+    rng = np.random.default_rng(2)
+    B, H, nb, d, k = 1, 2, 16, 8, 5
+    qm = rng.normal(size=(B, H, nb, d))
+    km = rng.normal(size=(B, H, nb, d))
+    col, kth = oracle.select(qm, km, k, want_kth=True)
+    for h in range(H):
+        S = qm[0, h] @ km[0, h].T  # independent score computation (numpy matmul)
+        for i in range(nb):
+            row = col[0, h, i]
+            assert list(row) == sorted(set(row)) and i in row and len(row) == k
+            kept = [j for j in row if j != i]
+            dropped = [j for j in range(nb) if j not in row]
+            for a in kept:
+                for b in dropped:
+                    assert S[i, a] > S[i, b] or (S[i, a] == S[i, b] and a < b)
+            assert math.isclose(kth[0, h, i], min(S[i, a] for a in kept), rel_tol=1e-12)
+
+
+def test_select_exact_ties_prefer_lower_index():
+    # key blocks 2, 5 and 7 are identical copies: exact ties between them
+    rng = np.random.default_rng(3)
+    nb, d = 8, 4
+    qm = rng.normal(size=(1, 1, nb, d))
+    km = rng.normal(size=(1, 1, nb, d)) * 0.01
+    km[0, 0, 5] = km[0, 0, 7] = km[0, 0, 2] = qm[0, 0, 0] * 3.0  # the top score for row 0
+    col = oracle.select(qm, km, 3)  # row 0: diag + two of {2, 5, 7}
+    np.testing.assert_array_equal(col[0, 0, 0], [0, 2, 5])
+    col = oracle.select(qm, km, 2)
+    np.testing.assert_array_equal(col[0, 0, 0], [0, 2])
+
+
+def test_select_rejects_bad_k():
+    qm = np.zeros((1, 1, 4, 2))
+    with pytest.raises(ValueError):
+        oracle.select(qm, qm, 0)
+    with pytest.raises(ValueError):
+        oracle.select(qm, qm, 5)
+
+
+def test_keep_blocks_rounding():
+    assert [oracle.keep_blocks(256, f) for f in (1.0, 0.5, 0.3, 0.2, 0.1)] == [256, 128, 77, 51, 26]
+    assert oracle.keep_blocks(960, 0.1) == 96
+    assert oracle.keep_blocks(591, 0.15) == 89
+    assert oracle.keep_blocks(16, 0.25) == 4
+    assert oracle.keep_blocks(10, 0.0) == 1
+
+
+# ---------------------------------------------------------------- attention
+
+def test_attention_hand_example_exact_rationals():
+    g = _golden()
+    q, k, v = _as4(g["Q"]), _as4(g["K"]), _as4(g["V"])
+    out, col, qm, km = oracle.forward(q, k, v, g["L"], g["blk"], 2, scale=math.log(2.0))
+    np.testing.assert_array_equal(col[0, 0], g["col_idx_k2"])
+    want0 = [float(Fraction(s)) for s in g["out_k2_col0"]]
+    want1 = [float(Fraction(s)) for s in g["out_k2_col1"]]
+    np.testing.assert_allclose(out[0, 0, :, 0], want0, rtol=1e-13, atol=0)
+    np.testing.assert_allclose(out[0, 0, :, 1], want1, rtol=1e-13, atol=0)
+
+
+@pytest.mark.parametrize("L", [96, 90])
+def test_attention_keep_all_equals_dense_sdpa(L):
+    """k = nb: the sparse path must be dense softmax attention over the valid keys."""
+    B, H, blk, d = 1, 2, 16, 8
+    Lp = -(-L // blk) * blk
+    nb = Lp // blk
+    q, k, v = (t.double().numpy() for t in inputs.random_qkv(B, H, Lp, d, L=L, seed=4, dtype=torch.float64))
+    k[:, :, L:] = 5.0  # junk in padded keys must not matter
+    v[:, :, L:] = 7.0
+    out, col, _, _ = oracle.forward(q, k, v, L, blk, nb)
+    mask = np.zeros((Lp, Lp), dtype=bool)
+    mask[:, :L] = True
+    ref = _sdpa(q, k, v, 1.0 / math.sqrt(d), mask)
+    np.testing.assert_allclose(out[:, :, :L], ref[:, :, :L], rtol=1e-12, atol=1e-12)
+    assert np.all(out[:, :, L:] == 0.0)
+
+
+def test_attention_k1_is_dense_within_diagonal_block():
+    B, H, Lp, blk, d = 1, 1, 64, 16, 8
+    q, k, v = (t.numpy() for t in inputs.random_qkv(B, H, Lp, d, seed=5, dtype=torch.float64))
+    out, col, _, _ = oracle.forward(q, k, v, Lp, blk, 1)
+    for i in range(Lp // blk):
+        s = slice(i * blk, (i + 1) * blk)
+        ref = _sdpa(q[:, :, s], k[:, :, s], v[:, :, s], 1.0 / math.sqrt(d))
+        np.testing.assert_allclose(out[:, :, s], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_block_indicator_v_pins_the_mask():
+    """V[t, c] = 1 if block(t) == c: O[q, c] is the softmax mass on block c, so it is
+    0 on dropped blocks, > 0 on kept ones, and sums to 1."""
+    B, H, Lp, blk, d, k = 1, 2, 128, 8, 16, 4
+    nb = Lp // blk
+    q, kk, _ = (t.numpy() for t in inputs.random_qkv(B, H, Lp, d, seed=6, dtype=torch.float64))
+    v = np.zeros((B, H, Lp, d))
+    for t in range(Lp):
+        v[:, :, t, t // blk] = 1.0
+    out, col, _, _ = oracle.forward(q, kk, v, Lp, blk, k)
+    for h in range(H):
+        for t in range(Lp):
+            kept = set(col[0, h, t // blk])
+            row = out[0, h, t]
+            for c in range(nb):
+                if c in kept:
+                    assert row[c] > 0.0
+                else:
+                    assert row[c] == 0.0
+            assert abs(row.sum() - 1.0) < 1e-13
+
+
+def test_attention_uniform_when_q_zero():
+    """Q = 0: every logit equals, so O is the plain mean of V over the kept valid keys."""
+    g = _golden()
+    B, H, Lp, blk, d, L, k = 1, 1, 48, 8, 4, 45, 2
+    _, kk, v = (t.numpy() for t in inputs.random_qkv(B, H, Lp, d, L=L, seed=8, dtype=torch.float64))
+    q = np.zeros_like(kk)
+    qm = np.zeros((1, 1, Lp // blk, d))
+    km = oracle.pool(kk, L, blk)
+    col = oracle.select(qm, km, k)  # all scores 0: diagonal + lowest other index
+    rp = oracle.uniform_row_ptr(1, 1, Lp // blk, k)
+    out = oracle.attention(q, kk, v, L, blk, rp, col)
+    for t in range(L):
+        keys = [u for j in col[0, 0, t // blk] for u in range(j * blk, (j + 1) * blk) if u < L]
+        np.testing.assert_allclose(out[0, 0, t], v[0, 0, keys].mean(axis=0), rtol=1e-13, atol=1e-14)
+    assert g  # golden file present
+
+
+def test_attention_constant_v():
+    B, H, Lp, blk, d = 1, 1, 64, 16, 8
+    q, k, _ = (t.numpy() for t in inputs.random_qkv(B, H, Lp, d, seed=9, dtype=torch.float64))
+    v = np.broadcast_to(np.arange(d, dtype=np.float64), (B, H, Lp, d)).copy()
+    out, _, _, _ = oracle.forward(q, k, v, Lp, blk, 2)
+    np.testing.assert_allclose(out, v, rtol=1e-13, atol=1e-13)
+
+
+def test_attention_invariant_to_key_order_within_block():
+    B, H, Lp, blk, d, k = 1, 1, 64, 16, 8, 2
+    q, kk, v = (t.numpy() for t in inputs.random_qkv(B, H, Lp, d, seed=10, dtype=torch.float64))
+    out1, col1, _, _ = oracle.forward(q, kk, v, Lp, blk, k)
+    perm = np.arange(Lp)
+    rng = np.random.default_rng(11)
+    for i in range(Lp // blk):
+        perm[i * blk:(i + 1) * blk] = rng.permutation(np.arange(i * blk, (i + 1) * blk))
+    out2, col2, _, _ = oracle.forward(q, kk[:, :, perm], v[:, :, perm], Lp, blk, k)
+    np.testing.assert_array_equal(col1, col2)  # block means unchanged by the permutation
+    np.testing.assert_allclose(out1, out2, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_large_logits_need_max_subtraction():
+    """Logits of several hundred overflow exp() unless the max is subtracted first."""
+    B, H, Lp, blk, d = 1, 1, 32, 8, 8
+    q, k, v = (t.numpy() for t in inputs.random_qkv(B, H, Lp, d, seed=12, dtype=torch.float64, q_scale=300.0))
+    nb = Lp // blk
+    out, _, _, _ = oracle.forward(q, k, v, Lp, blk, nb)
+    ref = _sdpa(q, k, v, 1.0 / math.sqrt(d))
+    assert np.all(np.isfinite(out))
+    np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)
+
+
+def test_attention_general_csr_rows():
+    """Rows of different lengths, including an empty row (output 0)."""
+    B, H, Lp, blk, d = 1, 1, 32, 8, 4
+    q, k, v = (t.numpy() for t in inputs.random_qkv(B, H, Lp, d, seed=13, dtype=torch.float64))
+    rows = [[0, 3], [], [1, 2, 3], [3]]
+    rp = np.cumsum([0] + [len(r) for r in rows]).astype(np.int32)
+    ci = np.array([j for r in rows for j in r], dtype=np.int32)
+    out = oracle.attention(q, k, v, Lp, blk, rp, ci)
+    for i, r in enumerate(rows):
+        s = slice(i * blk, (i + 1) * blk)
+        if not r:
+            assert np.all(out[0, 0, s] == 0.0)
+            continue
+        keys = np.concatenate([np.arange(j * blk, (j + 1) * blk) for j in r])
+        ref = _sdpa(q[:, :, s], k[:, :, keys], v[:, :, keys], 1.0 / math.sqrt(d))
+        np.testing.assert_allclose(out[:, :, s], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_unit_sampling_matches_full():
+    B, H, Lp, blk, d, k = 1, 2, 64, 16, 8, 2
+    q, kk, v = (t.numpy() for t in inputs.random_qkv(B, H, Lp, d, L=60, seed=14, dtype=torch.float64))
+    full, col, _, _ = oracle.forward(q, kk, v, 60, blk, k)
+    nb = Lp // blk
+    rp = oracle.uniform_row_ptr(B, H, nb, k)
+    units = [5, 0, 3, 7]
+    part = oracle.attention(q, kk, v, 60, blk, rp, col, units=units)
+    for n, u in enumerate(units):
+        h, i = divmod(u, nb)
+        np.testing.assert_array_equal(part[n], full[0, h, i * blk:(i + 1) * blk])
+
+
+def test_oracle_accepts_fp32_and_bf16_consistently():
+    q, k, v = inputs.random_qkv(1, 1, 64, 8, seed=15, dtype=torch.bfloat16)
+    as_f32 = [t.float().numpy() for t in (q, k, v)]
+    as_bits = [inputs.bf16_bits(t) for t in (q, k, v)]
+    o1, c1, _, _ = oracle.forward(*as_f32, 64, 16, 2)
+    o2, c2, _, _ = oracle.forward(*as_bits, 64, 16, 2)
+    np.testing.assert_array_equal(c1, c2)
+    np.testing.assert_array_equal(o1, o2)
