@@ -1,0 +1,147 @@
+/*
+ * sbsa -- dynamic block-sparse self-attention for NVIDIA B200 (sm_100a).
+ *
+ * The method (the hot path of 14B video-DiT inference at ~120K tokens):
+ *   1. pool   : block-level means of Query and Key estimate attention importance
+ *               (page "知识卡片：600倍加速，720p视频实时生成！单卡也能带的动14B模型",
+ *               section 方法/产品要点, bullet 动态稀疏量化注意力);
+ *   2. select : each query block keeps only ~10-20% of the key blocks, decided at run
+ *               time per input (same bullet, "稀疏率 80%-90%");
+ *   3. attend : the kept blocks are computed densely
+ *               (page "单卡 RTX 5090 跑 Wan2.2-A14B：720p 视频生成只要 3.8 秒",
+ *               section 四步拆解, item 3 动态稀疏注意力).
+ *
+ * Readings this library takes where those pages are silent: the score of a (query
+ * block i, key block j) pair is <qmean_i, kmean_j>; each query block keeps a fixed
+ * count k of key blocks, the diagonal j == i always among them, the rest the k-1
+ * highest scores, ties to the lower block index; attention is non-causal with scale
+ * 1/sqrt(d) by default; padded tokens are masked as keys and produce zero rows.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are row-major, contiguous [B][H][Lp][d] (bf16 for Q/K/V/O), block means
+ *     [B][H][nb][d] fp32, where nb = Lp / block_size.  Device pointers.  bf16 and fp32
+ *     tensors must be 16-byte aligned.
+ *   - The caller owns every buffer.  No call allocates device memory.
+ *   - All calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream).  Argument errors are returned before anything is
+ *     launched.  Errors detected on the device (a bounded wait that ran out, an
+ *     out-of-range block index) are latched in a per-device error word and reported by
+ *     sbsa_check().
+ *   - Calls are safe to issue from several host threads; the last error message is
+ *     thread-local.
+ */
+#ifndef SBSA_H
+#define SBSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SBSA_OK = 0,
+    SBSA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, inconsistent shape, k out of range */
+    SBSA_ERR_UNSUPPORTED = 2, /* head_dim or block_size not in {64,128}, too many blocks */
+    SBSA_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or smaller than sbsa_workspace_bytes() */
+    SBSA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (launch, tensor-map encode) */
+    SBSA_ERR_TIMEOUT = 5,     /* a kernel's bounded wait expired (device-side, via sbsa_check) */
+    SBSA_ERR_BAD_INDEX = 6    /* a CSR block index / row pointer was out of range (device-side) */
+} sbsa_status;
+
+/* Problem shape.  seq_len = L valid tokens; seq_len_padded = Lp must be the smallest
+ * multiple of block_size >= L (every block holds at least one valid token).
+ * head_dim in {64, 128}; block_size in {64, 128}; nb = Lp / block_size <= 2048;
+ * batch * heads * Lp < 2^31. */
+typedef struct {
+    int32_t batch;
+    int32_t heads;
+    int32_t seq_len;
+    int32_t seq_len_padded;
+    int32_t head_dim;
+    int32_t block_size;
+} sbsa_shape;
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t sbsa_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char *sbsa_status_string(sbsa_status status);
+
+/* Detail of the last error returned on the calling host thread ("" if none). */
+const char *sbsa_last_error_message(void);
+
+/* Kept key blocks per query block for a keep fraction: round-half-up(keep * nb),
+ * clamped to [1, nb].  ("keep about 10-20% of the blocks" read as a per-row count.)
+ * Returns 0 if num_blocks < 1 or keep_fraction is not finite. */
+int32_t sbsa_keep_blocks(int32_t num_blocks, double keep_fraction);
+
+/* Bytes of workspace sbsa_forward() needs: q_mean and k_mean (fp32, B*H*nb*d each),
+ * row_ptr (int32, B*H*nb+1) and col_idx (int32, B*H*nb*k), each 256-byte aligned.
+ * Returns 0 for an invalid shape or k. */
+size_t sbsa_workspace_bytes(const sbsa_shape *shape, int32_t k_keep);
+
+/* Step 1 -- block means (page "知识卡片…", 方法/产品要点, 动态稀疏量化注意力: Q/K
+ * block-level means as the importance estimate).
+ *   q, k   : bf16 [B][H][Lp][d] (device).  Padded tokens may hold any value.
+ *   q_mean : fp32 [B][H][nb][d] (device, written) = mean of Q over the valid tokens
+ *            of each block; k_mean likewise for K.
+ * One kernel launch, HBM-bandwidth bound. */
+sbsa_status sbsa_pool_qk(const sbsa_shape *shape, const void *q, const void *k, float *q_mean, float *k_mean,
+                         void *stream);
+
+/* Step 2 -- block selection (same bullet: keep ~10-20% of the blocks, chosen per
+ * input at run time).  For each (b, h, query block i): score_j = <q_mean_i, k_mean_j>
+ * in fp32; keep j = i plus the k_keep-1 highest-scoring other blocks (ties: lower j);
+ * write them in ascending order.
+ *   q_mean, k_mean : fp32 [B][H][nb][d] (device).  Scores must be finite.
+ *   k_keep         : 1 <= k_keep <= nb.
+ *   row_ptr        : int32 [B*H*nb + 1] (device, written) CSR row offsets, r * k_keep.
+ *   col_idx        : int32 [B*H*nb*k_keep] (device, written) key-block indices.
+ * One kernel launch. */
+sbsa_status sbsa_select_blocks(const sbsa_shape *shape, const float *q_mean, const float *k_mean, int32_t k_keep,
+                               int32_t *row_ptr, int32_t *col_idx, void *stream);
+
+/* Step 3 -- dense attention inside the kept blocks (page "单卡 RTX 5090 跑
+ * Wan2.2-A14B…", 四步拆解 item 3: kept blocks computed densely).  For every valid query
+ * row t of query block i:  O[t] = sum over valid keys u of the blocks listed in
+ * col_idx[row_ptr[r] .. row_ptr[r+1]) of softmax_u(scale * Q[t].K[u]) V[u], where
+ * r = (b*H + h)*nb + i.  Non-causal.  Rows t >= L, and rows whose list holds no valid
+ * key, are written as 0.
+ *   q, k, v : bf16 [B][H][Lp][d] (device).
+ *   row_ptr : int32 [B*H*nb + 1], non-decreasing, row_ptr[0] == 0; any list length.
+ *   col_idx : int32 key-block indices in [0, nb).  An index outside that range is
+ *             skipped (contributes nothing) and latches SBSA_ERR_BAD_INDEX.
+ *   scale   : logit scale; 0 means 1/sqrt(head_dim).
+ *   o       : bf16 [B][H][Lp][d] (device, written).
+ * Arithmetic: bf16 tensor-core products (tcgen05) with fp32 accumulation, fp32 online
+ * softmax, probabilities rounded to bf16 before the P.V product, bf16 output. */
+sbsa_status sbsa_attention_fwd(const sbsa_shape *shape, const void *q, const void *k, const void *v,
+                               const int32_t *row_ptr, const int32_t *col_idx, float scale, void *o, void *stream);
+
+/* Steps 1-3 in one call on one stream: pool -> select -> attend, with the means and
+ * the CSR lists carved out of `workspace` (device, 256-byte aligned, at least
+ * sbsa_workspace_bytes(shape, k_keep) bytes).  If col_idx_out is non-NULL the
+ * selected blocks ([B*H*nb*k_keep] int32, device) are written there as well. */
+sbsa_status sbsa_forward(const sbsa_shape *shape, const void *q, const void *k, const void *v, int32_t k_keep,
+                         float scale, void *o, int32_t *col_idx_out, void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/* Synchronizes `stream`, then reads and clears the calling device's error word.
+ * Returns SBSA_OK, SBSA_ERR_TIMEOUT, SBSA_ERR_BAD_INDEX or SBSA_ERR_CUDA (a sticky
+ * CUDA error or a failed synchronize). */
+sbsa_status sbsa_check(void *stream);
+
+/* Validates a CSR block list on the device: row_ptr[0] == 0, non-decreasing,
+ * row_ptr[nrows] == nnz, every index in [0, nb) and strictly ascending within a row,
+ * and (if require_diagonal) each row r contains its own block r % nb.
+ * Synchronous: it synchronizes `stream` and returns SBSA_OK or SBSA_ERR_BAD_INDEX. */
+sbsa_status sbsa_validate_csr(const sbsa_shape *shape, const int32_t *row_ptr, const int32_t *col_idx, int64_t nnz,
+                              int32_t require_diagonal, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SBSA_H */

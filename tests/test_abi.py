@@ -1,0 +1,115 @@
+"""CPU checks of the C ABI: the library builds, loads and exports every symbol the
+header declares; host-side logic (keep count, workspace size, argument validation)
+behaves as documented.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from video_dit_dynamic_b200 import build as sbuild
+from video_dit_dynamic_b200 import sbsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sbsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sbuild.build()
+    return sbsa.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sbsa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declarations_match_binding_list():
+    assert declared_functions() == sorted(sbsa.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in sbsa.STATUS_NAMES.items():
+        assert sbsa.sbsa_status_string(code) == name
+    assert sbsa.sbsa_status_string(99) == "SBSA_ERR_UNKNOWN"
+    assert sbsa.sbsa_version() >= 100
+
+
+def test_keep_blocks_rounding(lib):
+    assert [sbsa.sbsa_keep_blocks(256, f) for f in (1.0, 0.5, 0.3, 0.2, 0.1)] == [256, 128, 77, 51, 26]
+    assert sbsa.sbsa_keep_blocks(960, 0.10) == 96
+    assert sbsa.sbsa_keep_blocks(591, 0.15) == 89
+    assert sbsa.sbsa_keep_blocks(16, 0.25) == 4
+    assert sbsa.sbsa_keep_blocks(10, 0.0) == 1
+    assert sbsa.sbsa_keep_blocks(10, 5.0) == 10
+    assert sbsa.sbsa_keep_blocks(0, 0.5) == 0
+    assert sbsa.sbsa_keep_blocks(10, float("nan")) == 0
+
+
+def test_workspace_bytes(lib):
+    s = sbsa.make_shape(1, 40, 122880, 128, 128)
+    k = 96
+    rows = 40 * 960
+    means = rows * 128 * 4
+    want = means + means + ((rows + 1) * 4 + 255) // 256 * 256 + rows * k * 4
+    assert sbsa.sbsa_workspace_bytes(s, k) == want
+    assert sbsa.sbsa_workspace_bytes(s, 0) == 0
+    assert sbsa.sbsa_workspace_bytes(s, 961) == 0
+    bad = sbsa.make_shape(1, 1, 100, 96, 64)
+    assert sbsa.sbsa_workspace_bytes(bad, 1) == 0
+
+
+def _status(lib, fn, *args):
+    return getattr(lib, fn)(*args)
+
+
+def test_argument_errors_return_before_launch(lib):
+    P = ctypes.c_void_p
+    good = sbsa.make_shape(1, 2, 1000, 64, 64)
+    fake = P(0x10000)  # never dereferenced: validation fails first or the call is not made
+    # null pointers
+    assert lib.sbsa_pool_qk(ctypes.byref(good), None, fake, fake, fake, None) == 1
+    # misaligned pointer
+    assert lib.sbsa_pool_qk(ctypes.byref(good), P(0x10008), fake, fake, fake, None) == 1
+    assert b"aligned" in lib.sbsa_last_error_message()
+    # unsupported head_dim / block size
+    assert lib.sbsa_pool_qk(ctypes.byref(sbsa.make_shape(1, 2, 1000, 96, 64)), fake, fake, fake, fake, None) == 2
+    assert lib.sbsa_pool_qk(ctypes.byref(sbsa.make_shape(1, 2, 1000, 64, 32)), fake, fake, fake, fake, None) == 2
+    # Lp not the rounded-up L
+    s = sbsa.Shape(1, 2, 1000, 1088, 64, 64)
+    assert lib.sbsa_pool_qk(ctypes.byref(s), fake, fake, fake, fake, None) == 1
+    # too many blocks
+    s = sbsa.make_shape(1, 1, 64 * 2049, 64, 64)
+    assert lib.sbsa_pool_qk(ctypes.byref(s), fake, fake, fake, fake, None) == 2
+    # k out of range
+    assert lib.sbsa_select_blocks(ctypes.byref(good), fake, fake, 0, fake, fake, None) == 1
+    assert lib.sbsa_select_blocks(ctypes.byref(good), fake, fake, 17, fake, fake, None) == 1
+    # non-finite scale
+    assert lib.sbsa_attention_fwd(ctypes.byref(good), fake, fake, fake, fake, fake, ctypes.c_float(float("inf")),
+                                  fake, None) == 1
+    # workspace missing, misaligned or too small
+    assert lib.sbsa_forward(ctypes.byref(good), fake, fake, fake, 4, ctypes.c_float(0), fake, None, None, 0,
+                            None) == 3
+    assert lib.sbsa_forward(ctypes.byref(good), fake, fake, fake, 4, ctypes.c_float(0), fake, None, P(0x10010),
+                            1 << 30, None) == 3
+    assert lib.sbsa_forward(ctypes.byref(good), fake, fake, fake, 4, ctypes.c_float(0), fake, None, P(0x10000),
+                            16, None) == 3
+    assert b"smaller" in lib.sbsa_last_error_message()
+    # null shape
+    assert lib.sbsa_pool_qk(None, fake, fake, fake, fake, None) == 1
+
+
+def test_binding_rejects_cpu_tensors(lib):
+    import torch
+    s = sbsa.make_shape(1, 1, 128, 64, 64)
+    x = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    m = torch.zeros(1, 1, 2, 64)
+    with pytest.raises(TypeError):
+        sbsa.sbsa_pool_qk(s, x, x, m, m, stream=0)

@@ -1,0 +1,67 @@
+"""GPU parity at the full workload sizes, in the launch configuration bench.py times
+(one sbsa_forward call: pool -> select -> attend).  The oracle checks the block means
+and the selection of EVERY query block, and the attention output on a sample of
+(head, query block) units that includes first, last (ragged) and interior blocks."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests import parity_utils as pu
+from video_dit_dynamic_b200 import inputs, sbsa
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    pu.require_cuda()
+
+
+def _sample_units(H, nb, n, seed):
+    rng = np.random.default_rng(seed)
+    units = {0, nb - 1, (H - 1) * nb, H * nb - 1}
+    while len(units) < n:
+        units.add(int(rng.integers(0, H * nb)))
+    return sorted(units)
+
+
+@pytest.mark.parametrize("name", ["480p", "720p", "long122880"])
+def test_forward_full_size(name):
+    wl = inputs.WORKLOADS[name]
+    q, k, v = inputs.make_qkv(wl, seed=0, device="cuda")
+    L, blk, nb, H = wl.seq_len, wl.block, wl.num_blocks, wl.heads
+    kk = sbsa.sbsa_keep_blocks(nb, wl.keep)
+    s = pu.shape_of(q, L, blk)
+    o = torch.empty_like(q)
+    col = torch.empty(H * nb * kk, dtype=torch.int32, device="cuda")
+    ws = sbsa.alloc_workspace(s, kk)
+    sbsa.sbsa_forward(s, q, k, v, kk, 0.0, o, col, ws)
+    sbsa.sbsa_check()
+    qb, kb, vb = pu.bits(q), pu.bits(k), pu.bits(v)
+    del q, k, v
+    # means: the workspace holds them (q_mean first, k_mean 256-byte aligned after it)
+    rows = H * nb
+    nmean = rows * wl.head_dim
+    qm_gpu = ws[: nmean * 4].view(torch.float32).view(1, H, nb, wl.head_dim)
+    off = (nmean * 4 + 255) // 256 * 256
+    km_gpu = ws[off: off + nmean * 4].view(torch.float32).view(1, H, nb, wl.head_dim)
+    qm = oracle.pool(qb, L, blk)
+    km = oracle.pool(kb, L, blk)
+    pu.assert_means_close(qm_gpu, qm)
+    pu.assert_means_close(km_gpu, km)
+    ref_col = oracle.select(qm, km, kk)
+    gcol = col.cpu().numpy().reshape(1, H, nb, kk)
+    swaps = pu.assert_selection_ok(gcol, ref_col, qm, km, kk)
+    assert swaps <= rows // 100, f"{swaps} rows differ by tie swaps"
+    units = _sample_units(H, nb, 24, seed=nb)
+    rp = oracle.uniform_row_ptr(1, H, nb, kk)
+    ref = oracle.attention(qb, kb, vb, L, blk, rp, ref_col, units=units)
+    got = o.view(H * nb, blk, wl.head_dim)[torch.tensor(units, device="cuda")]
+    # compare under the oracle's mask where the GPU chose the same blocks
+    same = [n for n, u in enumerate(units) if np.array_equal(gcol.reshape(-1, kk)[u], ref_col.reshape(-1, kk)[u])]
+    assert len(same) >= len(units) - 2
+    pu.assert_attention_close(got[same], ref[same], f"{name} sampled units")
+    # padded query rows are zero
+    if L % blk:
+        assert torch.all(o[:, :, L:] == 0)

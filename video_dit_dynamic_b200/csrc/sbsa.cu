@@ -1,0 +1,389 @@
+// C ABI of the sbsa library (declared in include/sbsa.h): argument checking, tensor-map
+// encoding, workspace carving and kernel launches.  All compute is in the kernels of
+// pool.cuh, select.cuh and attn.cuh; nothing here touches tensor data on the host.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/sbsa.h"
+#include "attn.cuh"
+#include "common.cuh"
+#include "pool.cuh"
+#include "ptx.cuh"
+#include "select.cuh"
+
+namespace sbsa {
+namespace {
+
+thread_local char t_errmsg[512] = "";
+
+sbsa_status fail(sbsa_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_errmsg, sizeof t_errmsg, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+sbsa_status ok() {
+    t_errmsg[0] = '\0';
+    return SBSA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxBlocks = 2048;
+
+sbsa_status check_shape(const sbsa_shape* s) {
+    if (!s) return fail(SBSA_ERR_INVALID_ARG, "shape is NULL");
+    if (s->batch < 1 || s->heads < 1 || s->seq_len < 1)
+        return fail(SBSA_ERR_INVALID_ARG, "batch, heads and seq_len must be >= 1");
+    if (s->head_dim != 64 && s->head_dim != 128)
+        return fail(SBSA_ERR_UNSUPPORTED, "head_dim %d not in {64, 128}", s->head_dim);
+    if (s->block_size != 64 && s->block_size != 128)
+        return fail(SBSA_ERR_UNSUPPORTED, "block_size %d not in {64, 128}", s->block_size);
+    const long long want = (static_cast<long long>(s->seq_len) + s->block_size - 1) / s->block_size * s->block_size;
+    if (s->seq_len_padded != want)
+        return fail(SBSA_ERR_INVALID_ARG, "seq_len_padded %d must be seq_len %d rounded up to block_size %d (= %lld)",
+                    s->seq_len_padded, s->seq_len, s->block_size, want);
+    const long long nb = s->seq_len_padded / s->block_size;
+    if (nb > kMaxBlocks) return fail(SBSA_ERR_UNSUPPORTED, "%lld blocks exceed the limit %d", nb, kMaxBlocks);
+    const long long rows = static_cast<long long>(s->batch) * s->heads * s->seq_len_padded;
+    if (rows >= (1ll << 31)) return fail(SBSA_ERR_UNSUPPORTED, "batch*heads*seq_len_padded must be < 2^31");
+    return SBSA_OK;
+}
+
+int num_blocks(const sbsa_shape* s) { return s->seq_len_padded / s->block_size; }
+long long num_rows(const sbsa_shape* s) { return static_cast<long long>(s->batch) * s->heads * num_blocks(s); }
+
+sbsa_status check_k(const sbsa_shape* s, int32_t k) {
+    const int nb = num_blocks(s);
+    if (k < 1 || k > nb) return fail(SBSA_ERR_INVALID_ARG, "k_keep %d not in [1, %d]", k, nb);
+    if (num_rows(s) * k >= (1ll << 31)) return fail(SBSA_ERR_UNSUPPORTED, "B*H*nb*k_keep must be < 2^31");
+    return SBSA_OK;
+}
+
+sbsa_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(SBSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2D view [rows][d] of a bf16 tensor, box {64, box_rows}, 128-byte swizzle.
+sbsa_status make_map(CUtensorMap* m, const void* base, long long rows, int d, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(SBSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SBSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return SBSA_OK;
+}
+
+std::atomic<unsigned int> g_epoch{1};
+
+// ---------------------------------------------------------------- launchers
+sbsa_status launch_pool(const sbsa_shape* s, const void* q, const void* k, float* qm, float* km, cudaStream_t st) {
+    const long long units = num_rows(s);
+    const dim3 grid(static_cast<unsigned>(2 * units));
+    const int L = s->seq_len, Lp = s->seq_len_padded, nb = num_blocks(s);
+    const uint4* q4 = static_cast<const uint4*>(q);
+    const uint4* k4 = static_cast<const uint4*>(k);
+    if (s->head_dim == 128) {
+        if (s->block_size == 128) pool_kernel<128, 128><<<grid, 256, 0, st>>>(q4, k4, qm, km, L, Lp, nb, units);
+        else pool_kernel<128, 64><<<grid, 256, 0, st>>>(q4, k4, qm, km, L, Lp, nb, units);
+    } else {
+        if (s->block_size == 128) pool_kernel<64, 128><<<grid, 256, 0, st>>>(q4, k4, qm, km, L, Lp, nb, units);
+        else pool_kernel<64, 64><<<grid, 256, 0, st>>>(q4, k4, qm, km, L, Lp, nb, units);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SBSA_OK : cuda_fail(e, "pool launch");
+}
+
+template <int D, int KPL>
+sbsa_status launch_select_t(const sbsa_shape* s, const float* qm, const float* km, int k, int32_t* rp, int32_t* ci,
+                            cudaStream_t st) {
+    constexpr int QT = 16;
+    const int nb = num_blocks(s);
+    const size_t smem = static_cast<size_t>(QT) * D * 4 + static_cast<size_t>(QT) * 32 * KPL * 4;
+    auto kern = select_kernel<D, QT, KPL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_fail(e, "select smem attribute");
+    const dim3 grid((nb + QT - 1) / QT, static_cast<unsigned>(s->batch * s->heads));
+    kern<<<grid, 256, smem, st>>>(qm, km, nb, k, rp, ci, num_rows(s));
+    e = cudaGetLastError();
+    return e == cudaSuccess ? SBSA_OK : cuda_fail(e, "select launch");
+}
+
+template <int D>
+sbsa_status launch_select_d(const sbsa_shape* s, const float* qm, const float* km, int k, int32_t* rp, int32_t* ci,
+                            cudaStream_t st) {
+    const int nb = num_blocks(s);
+    if (nb <= 64) return launch_select_t<D, 2>(s, qm, km, k, rp, ci, st);
+    if (nb <= 256) return launch_select_t<D, 8>(s, qm, km, k, rp, ci, st);
+    if (nb <= 512) return launch_select_t<D, 16>(s, qm, km, k, rp, ci, st);
+    if (nb <= 1024) return launch_select_t<D, 32>(s, qm, km, k, rp, ci, st);
+    return launch_select_t<D, 64>(s, qm, km, k, rp, ci, st);
+}
+
+sbsa_status launch_select(const sbsa_shape* s, const float* qm, const float* km, int k, int32_t* rp, int32_t* ci,
+                          cudaStream_t st) {
+    return s->head_dim == 128 ? launch_select_d<128>(s, qm, km, k, rp, ci, st)
+                              : launch_select_d<64>(s, qm, km, k, rp, ci, st);
+}
+
+template <int D, int BLK>
+sbsa_status launch_attn_t(const sbsa_shape* s, const void* q, const void* k, const void* v, const int32_t* rp,
+                          const int32_t* ci, float scale, void* o, cudaStream_t st) {
+    using C = AttnCfg<D, BLK>;
+    const long long rows = static_cast<long long>(s->batch) * s->heads * s->seq_len_padded;
+    CUtensorMap mq, mk, mv;
+    sbsa_status r;
+    if ((r = make_map(&mq, q, rows, D, 128)) != SBSA_OK) return r;
+    if ((r = make_map(&mk, k, rows, D, BLK)) != SBSA_OK) return r;
+    if ((r = make_map(&mv, v, rows, D, BLK)) != SBSA_OK) return r;
+    AttnParams p;
+    p.row_ptr = rp;
+    p.col_idx = ci;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.L = s->seq_len;
+    p.Lp = s->seq_len_padded;
+    p.nb = num_blocks(s);
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.epoch = g_epoch.fetch_add(1);
+    auto kern = attn_kernel<D, BLK>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "attention smem attribute");
+    kern<<<static_cast<unsigned>(num_rows(s)), 192, C::kSmemBytes, st>>>(mq, mk, mv, p);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? SBSA_OK : cuda_fail(e, "attention launch");
+}
+
+sbsa_status launch_attn(const sbsa_shape* s, const void* q, const void* k, const void* v, const int32_t* rp,
+                        const int32_t* ci, float scale, void* o, cudaStream_t st) {
+    if (s->head_dim == 128)
+        return s->block_size == 128 ? launch_attn_t<128, 128>(s, q, k, v, rp, ci, scale, o, st)
+                                    : launch_attn_t<128, 64>(s, q, k, v, rp, ci, scale, o, st);
+    return s->block_size == 128 ? launch_attn_t<64, 128>(s, q, k, v, rp, ci, scale, o, st)
+                                : launch_attn_t<64, 64>(s, q, k, v, rp, ci, scale, o, st);
+}
+
+float resolve_scale(const sbsa_shape* s, float scale) {
+    return scale == 0.f ? 1.0f / std::sqrt(static_cast<float>(s->head_dim)) : scale;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+    size_t q_mean, k_mean, row_ptr, col_idx, total;
+};
+
+WsLayout ws_layout(const sbsa_shape* s, int k) {
+    WsLayout w;
+    const size_t means = static_cast<size_t>(num_rows(s)) * s->head_dim * sizeof(float);
+    w.q_mean = 0;
+    w.k_mean = align256(means);
+    w.row_ptr = w.k_mean + align256(means);
+    w.col_idx = w.row_ptr + align256((static_cast<size_t>(num_rows(s)) + 1) * sizeof(int32_t));
+    w.total = w.col_idx + align256(static_cast<size_t>(num_rows(s)) * k * sizeof(int32_t));
+    return w;
+}
+
+// ---------------------------------------------------------------- CSR validation
+__global__ void validate_csr_kernel(const int32_t* row_ptr, const int32_t* col_idx, long long nrows, long long nnz,
+                                    int nb, int require_diag, unsigned int* bad) {
+    const long long r = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+    if (r > nrows) return;
+    if (r == nrows) {
+        if (row_ptr[nrows] != nnz || row_ptr[0] != 0) atomicOr(bad, 1u);
+        return;
+    }
+    const long long a = row_ptr[r], b = row_ptr[r + 1];
+    if (a < 0 || b < a || b > nnz) { atomicOr(bad, 1u); return; }
+    const int diag = static_cast<int>(r % nb);
+    bool has_diag = false;
+    int prev = -1;
+    for (long long e = a; e < b; ++e) {
+        const int j = col_idx[e];
+        if (j < 0 || j >= nb || j <= prev) { atomicOr(bad, 1u); return; }
+        has_diag |= (j == diag);
+        prev = j;
+    }
+    if (require_diag && !has_diag) atomicOr(bad, 1u);
+}
+
+}  // namespace
+}  // namespace sbsa
+
+using namespace sbsa;
+
+extern "C" {
+
+int32_t sbsa_version(void) { return 100; }
+
+const char* sbsa_status_string(sbsa_status st) {
+    switch (st) {
+        case SBSA_OK: return "SBSA_OK";
+        case SBSA_ERR_INVALID_ARG: return "SBSA_ERR_INVALID_ARG";
+        case SBSA_ERR_UNSUPPORTED: return "SBSA_ERR_UNSUPPORTED";
+        case SBSA_ERR_WORKSPACE: return "SBSA_ERR_WORKSPACE";
+        case SBSA_ERR_CUDA: return "SBSA_ERR_CUDA";
+        case SBSA_ERR_TIMEOUT: return "SBSA_ERR_TIMEOUT";
+        case SBSA_ERR_BAD_INDEX: return "SBSA_ERR_BAD_INDEX";
+    }
+    return "SBSA_ERR_UNKNOWN";
+}
+
+const char* sbsa_last_error_message(void) { return t_errmsg; }
+
+int32_t sbsa_keep_blocks(int32_t num_blocks, double keep_fraction) {
+    if (num_blocks < 1 || !std::isfinite(keep_fraction)) return 0;
+    double k = std::floor(keep_fraction * num_blocks + 0.5);
+    if (k < 1) k = 1;
+    if (k > num_blocks) k = num_blocks;
+    return static_cast<int32_t>(k);
+}
+
+size_t sbsa_workspace_bytes(const sbsa_shape* shape, int32_t k_keep) {
+    if (check_shape(shape) != SBSA_OK || check_k(shape, k_keep) != SBSA_OK) return 0;
+    return ws_layout(shape, k_keep).total;
+}
+
+sbsa_status sbsa_pool_qk(const sbsa_shape* shape, const void* q, const void* k, float* q_mean, float* k_mean,
+                         void* stream) {
+    sbsa_status r = check_shape(shape);
+    if (r != SBSA_OK) return r;
+    if (!q || !k || !q_mean || !k_mean) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(q_mean) || !aligned16(k_mean))
+        return fail(SBSA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    if ((r = launch_pool(shape, q, k, q_mean, k_mean, static_cast<cudaStream_t>(stream))) != SBSA_OK) return r;
+    return ok();
+}
+
+sbsa_status sbsa_select_blocks(const sbsa_shape* shape, const float* q_mean, const float* k_mean, int32_t k_keep,
+                               int32_t* row_ptr, int32_t* col_idx, void* stream) {
+    sbsa_status r = check_shape(shape);
+    if (r != SBSA_OK) return r;
+    if ((r = check_k(shape, k_keep)) != SBSA_OK) return r;
+    if (!q_mean || !k_mean || !row_ptr || !col_idx) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q_mean) || !aligned16(k_mean)) return fail(SBSA_ERR_INVALID_ARG, "means must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(row_ptr) | reinterpret_cast<uintptr_t>(col_idx)) & 3u)
+        return fail(SBSA_ERR_INVALID_ARG, "row_ptr/col_idx must be 4-byte aligned");
+    if ((r = launch_select(shape, q_mean, k_mean, k_keep, row_ptr, col_idx, static_cast<cudaStream_t>(stream))) !=
+        SBSA_OK)
+        return r;
+    return ok();
+}
+
+sbsa_status sbsa_attention_fwd(const sbsa_shape* shape, const void* q, const void* k, const void* v,
+                               const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o, void* stream) {
+    sbsa_status r = check_shape(shape);
+    if (r != SBSA_OK) return r;
+    if (!q || !k || !v || !o || !row_ptr || !col_idx) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return fail(SBSA_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(row_ptr) | reinterpret_cast<uintptr_t>(col_idx)) & 3u)
+        return fail(SBSA_ERR_INVALID_ARG, "row_ptr/col_idx must be 4-byte aligned");
+    if (!std::isfinite(scale)) return fail(SBSA_ERR_INVALID_ARG, "scale must be finite");
+    if ((r = launch_attn(shape, q, k, v, row_ptr, col_idx, resolve_scale(shape, scale), o,
+                         static_cast<cudaStream_t>(stream))) != SBSA_OK)
+        return r;
+    return ok();
+}
+
+sbsa_status sbsa_forward(const sbsa_shape* shape, const void* q, const void* k, const void* v, int32_t k_keep,
+                         float scale, void* o, int32_t* col_idx_out, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+    sbsa_status r = check_shape(shape);
+    if (r != SBSA_OK) return r;
+    if ((r = check_k(shape, k_keep)) != SBSA_OK) return r;
+    if (!q || !k || !v || !o) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return fail(SBSA_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
+    if (col_idx_out && (reinterpret_cast<uintptr_t>(col_idx_out) & 3u))
+        return fail(SBSA_ERR_INVALID_ARG, "col_idx_out must be 4-byte aligned");
+    if (!std::isfinite(scale)) return fail(SBSA_ERR_INVALID_ARG, "scale must be finite");
+    const WsLayout w = ws_layout(shape, k_keep);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return fail(SBSA_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+    if (workspace_bytes < w.total)
+        return fail(SBSA_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes,
+                    w.total);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* qm = reinterpret_cast<float*>(ws + w.q_mean);
+    float* km = reinterpret_cast<float*>(ws + w.k_mean);
+    int32_t* rp = reinterpret_cast<int32_t*>(ws + w.row_ptr);
+    int32_t* ci = col_idx_out ? col_idx_out : reinterpret_cast<int32_t*>(ws + w.col_idx);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((r = launch_pool(shape, q, k, qm, km, st)) != SBSA_OK) return r;
+    if ((r = launch_select(shape, qm, km, k_keep, rp, ci, st)) != SBSA_OK) return r;
+    if ((r = launch_attn(shape, q, k, v, rp, ci, resolve_scale(shape, scale), o, st)) != SBSA_OK) return r;
+    return ok();
+}
+
+sbsa_status sbsa_check(void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    unsigned int bits = 0, zero = 0;
+    if ((e = cudaMemcpyFromSymbol(&bits, g_error_bits, sizeof bits)) != cudaSuccess)
+        return cuda_fail(e, "read error word");
+    if ((e = cudaMemcpyToSymbol(g_error_bits, &zero, sizeof zero)) != cudaSuccess)
+        return cuda_fail(e, "clear error word");
+    if (bits & kErrTimeout) return fail(SBSA_ERR_TIMEOUT, "a kernel wait ran out of time");
+    if (bits & kErrBadIndex) return fail(SBSA_ERR_BAD_INDEX, "a block index or row pointer was out of range");
+    return ok();
+}
+
+sbsa_status sbsa_validate_csr(const sbsa_shape* shape, const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz,
+                              int32_t require_diagonal, void* stream) {
+    sbsa_status r = check_shape(shape);
+    if (r != SBSA_OK) return r;
+    if (!row_ptr || (!col_idx && nnz > 0) || nnz < 0) return fail(SBSA_ERR_INVALID_ARG, "null pointer or nnz < 0");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned int* bad = nullptr;  // module-scope device flag (no allocation)
+    cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&bad), g_csr_bad);
+    if (e != cudaSuccess) return cuda_fail(e, "csr flag address");
+    if ((e = cudaMemsetAsync(bad, 0, sizeof(unsigned int), st)) != cudaSuccess) return cuda_fail(e, "csr flag clear");
+    const long long nrows = num_rows(shape);
+    const long long threads = nrows + 1;
+    validate_csr_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(
+        row_ptr, col_idx, nrows, nnz, num_blocks(shape), require_diagonal, bad);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "csr validate launch");
+    unsigned int h = 0;
+    if ((e = cudaMemcpyAsync(&h, bad, sizeof h, cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+        return cuda_fail(e, "csr flag read");
+    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    if (h) return fail(SBSA_ERR_BAD_INDEX, "CSR block list is malformed");
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,133 @@
+// Step 2: block scores and per-query-block top-k with the diagonal forced.
+//
+// The method keeps only ~10-20% of the key blocks per query block, chosen at run time
+// from the block means (page "知识卡片：600倍加速，720p视频实时生成！单卡也能带的动14B模型",
+// 方法/产品要点, bullet 动态稀疏量化注意力).  Score of (i, j) = <qmean_i, kmean_j> in
+// fp32.  Kept: j = i, plus the k-1 highest-scoring j != i, ties to the lower j; written
+// in ascending j order into a CSR list with a uniform row length k.
+//
+// One CTA per (b*h, tile of QT query blocks), 256 threads.
+//   scores : each thread takes one key block j at a time, holds kmean_j in registers
+//            and forms its dot product with the QT query means broadcast from shared
+//            memory; the fp32 scores go to shared memory as order-preserving uint32 keys.
+//   top-k  : one warp per query row.  Lane l holds keys j = l + 32 r.  The (k-1)-th
+//            largest key T is found by a 32-step bisection on the key bits (warp-wide
+//            counts); then keys > T are kept, and keys == T in ascending j until k-1
+//            are kept; the output position of each kept j is a ballot prefix count,
+//            which yields the ascending order directly.
+#pragma once
+#include "common.cuh"
+
+namespace sbsa {
+
+// fp32 -> uint32 with the same order (larger float -> larger key).
+__device__ __forceinline__ uint32_t order_key(float s) {
+    const uint32_t u = __float_as_uint(s);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+template <int D, int QT, int KPL>
+__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ q_mean,
+                                                     const float* __restrict__ k_mean, int nb, int k_keep,
+                                                     int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx,
+                                                     long long n_rows) {
+    extern __shared__ __align__(16) uint8_t sel_smem[];
+    float* qs = reinterpret_cast<float*>(sel_smem);                    // [QT][D]
+    uint32_t* keys = reinterpret_cast<uint32_t*>(qs + QT * D);         // [QT][32*KPL]
+    constexpr int NBP = 32 * KPL;
+
+    const long long bh = blockIdx.y;
+    const int i0 = blockIdx.x * QT;
+    const int nq = min(QT, nb - i0);
+    const float* qm = q_mean + (bh * nb + i0) * D;
+    const float* km = k_mean + bh * nb * D;
+
+    for (int e = threadIdx.x; e < QT * D; e += blockDim.x) qs[e] = e < nq * D ? qm[e] : 0.f;
+    __syncthreads();
+
+    // ---- scores
+    for (int j = threadIdx.x; j < nb; j += blockDim.x) {
+        float kr[D];
+        const float4* kj = reinterpret_cast<const float4*>(km + static_cast<long long>(j) * D);
+#pragma unroll
+        for (int c4 = 0; c4 < D / 4; ++c4) {
+            const float4 t = __ldg(kj + c4);
+            kr[4 * c4] = t.x; kr[4 * c4 + 1] = t.y; kr[4 * c4 + 2] = t.z; kr[4 * c4 + 3] = t.w;
+        }
+#pragma unroll 1
+        for (int r = 0; r < QT; ++r) {
+            const float4* qr = reinterpret_cast<const float4*>(qs + r * D);
+            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+            for (int c4 = 0; c4 < D / 4; ++c4) {
+                const float4 t = qr[c4];
+                s0 = fmaf(t.x, kr[4 * c4], s0);
+                s1 = fmaf(t.y, kr[4 * c4 + 1], s1);
+                s2 = fmaf(t.z, kr[4 * c4 + 2], s2);
+                s3 = fmaf(t.w, kr[4 * c4 + 3], s3);
+            }
+            keys[r * NBP + j] = order_key((s0 + s1) + (s2 + s3));
+        }
+    }
+    __syncthreads();
+
+    // ---- top-k per row, one warp per row
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t lt = lanemask_lt();
+    const int kk = k_keep - 1;  // off-diagonal blocks to keep
+    for (int r = warp; r < nq; r += blockDim.x / 32) {
+        const int i = i0 + r;
+        uint32_t key[KPL];
+#pragma unroll
+        for (int s = 0; s < KPL; ++s) {
+            const int j = s * 32 + lane;
+            key[s] = (j < nb) ? keys[r * NBP + j] : 0u;
+        }
+        // candidates: j < nb and j != i.  T = kk-th largest candidate key (kk >= 1).
+        uint32_t T = 0u;
+        if (kk > 0) {
+#pragma unroll 1
+            for (int bit = 31; bit >= 0; --bit) {
+                const uint32_t cand = T | (1u << bit);
+                int cnt = 0;
+#pragma unroll
+                for (int s = 0; s < KPL; ++s) {
+                    const int j = s * 32 + lane;
+                    cnt += (j < nb && j != i && key[s] >= cand) ? 1 : 0;
+                }
+                cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
+                if (cnt >= kk) T = cand;
+            }
+        }
+        int n_gt = 0;
+        if (kk > 0) {
+#pragma unroll
+            for (int s = 0; s < KPL; ++s) {
+                const int j = s * 32 + lane;
+                n_gt += (j < nb && j != i && key[s] > T) ? 1 : 0;
+            }
+            n_gt = __reduce_add_sync(0xFFFFFFFFu, n_gt);
+        }
+        const int need_eq = kk - n_gt;  // how many keys equal to T to keep (lowest j first)
+        const long long row = bh * nb + i;
+        int32_t* out = col_idx + row * k_keep;
+        int pos = 0, eq_seen = 0;
+#pragma unroll
+        for (int s = 0; s < KPL; ++s) {
+            const int j = s * 32 + lane;
+            const bool cand = j < nb && j != i;
+            const bool is_eq = kk > 0 && cand && key[s] == T;
+            const uint32_t eq_mask = __ballot_sync(0xFFFFFFFFu, is_eq);
+            const int eq_rank = eq_seen + __popc(eq_mask & lt);
+            const bool keep = (j == i) || (kk > 0 && cand && key[s] > T) || (is_eq && eq_rank < need_eq);
+            const uint32_t m = __ballot_sync(0xFFFFFFFFu, keep);
+            if (keep) out[pos + __popc(m & lt)] = j;
+            pos += __popc(m);
+            eq_seen += __popc(eq_mask);
+        }
+        if (lane == 0) row_ptr[row] = static_cast<int32_t>(row * k_keep);
+    }
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) row_ptr[n_rows] = static_cast<int32_t>(n_rows * k_keep);
+}
+
+}  // namespace sbsa

@@ -1,0 +1,232 @@
+"""ctypes binding of libsbsa.so: one Python function per C entry point, same names.
+
+Argument marshalling only (torch tensors -> device pointers, current CUDA stream);
+every step of the computation runs in the library's kernels.  There is no fallback:
+if the library cannot be loaded, or a tensor is not a CUDA tensor of the right dtype
+and layout, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+SBSA_OK = 0
+STATUS_NAMES = {0: "SBSA_OK", 1: "SBSA_ERR_INVALID_ARG", 2: "SBSA_ERR_UNSUPPORTED", 3: "SBSA_ERR_WORKSPACE",
+                4: "SBSA_ERR_CUDA", 5: "SBSA_ERR_TIMEOUT", 6: "SBSA_ERR_BAD_INDEX"}
+
+# Every symbol include/sbsa.h declares.
+EXPORTS = ("sbsa_version", "sbsa_status_string", "sbsa_last_error_message", "sbsa_keep_blocks",
+           "sbsa_workspace_bytes", "sbsa_pool_qk", "sbsa_select_blocks", "sbsa_attention_fwd", "sbsa_forward",
+           "sbsa_check", "sbsa_validate_csr")
+
+
+class SbsaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("heads", ctypes.c_int32), ("seq_len", ctypes.c_int32),
+                ("seq_len_padded", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("block_size", ctypes.c_int32)]
+
+    @property
+    def num_blocks(self) -> int:
+        return self.seq_len_padded // self.block_size
+
+    def __repr__(self):
+        return (f"Shape(B={self.batch}, H={self.heads}, L={self.seq_len}, Lp={self.seq_len_padded}, "
+                f"d={self.head_dim}, block={self.block_size})")
+
+
+def make_shape(batch, heads, seq_len, head_dim, block_size, seq_len_padded=None) -> Shape:
+    if seq_len_padded is None:
+        seq_len_padded = -(-seq_len // block_size) * block_size
+    return Shape(batch, heads, seq_len, seq_len_padded, head_dim, block_size)
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libsbsa.so")
+
+
+def load(path: str | None = None):
+    """Load libsbsa.so (raises OSError if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or library_path()
+    if not os.path.exists(path):
+        raise OSError(f"{path} not found: build it with `python -m video_dit_dynamic_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    SP = ctypes.POINTER(Shape)
+    lib.sbsa_version.restype = I32
+    lib.sbsa_status_string.argtypes = [ctypes.c_int]
+    lib.sbsa_status_string.restype = ctypes.c_char_p
+    lib.sbsa_last_error_message.restype = ctypes.c_char_p
+    lib.sbsa_keep_blocks.argtypes = [I32, ctypes.c_double]
+    lib.sbsa_keep_blocks.restype = I32
+    lib.sbsa_workspace_bytes.argtypes = [SP, I32]
+    lib.sbsa_workspace_bytes.restype = SZ
+    lib.sbsa_pool_qk.argtypes = [SP, P, P, P, P, P]
+    lib.sbsa_select_blocks.argtypes = [SP, P, P, I32, P, P, P]
+    lib.sbsa_attention_fwd.argtypes = [SP, P, P, P, P, P, ctypes.c_float, P, P]
+    lib.sbsa_forward.argtypes = [SP, P, P, P, I32, ctypes.c_float, P, P, P, SZ, P]
+    lib.sbsa_check.argtypes = [P]
+    lib.sbsa_validate_csr.argtypes = [SP, P, P, ctypes.c_int64, I32, P]
+    for name in ("sbsa_pool_qk", "sbsa_select_blocks", "sbsa_attention_fwd", "sbsa_forward", "sbsa_check",
+                 "sbsa_validate_csr"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _raise_on(status: int):
+    if status != SBSA_OK:
+        msg = load().sbsa_last_error_message().decode(errors="replace")
+        raise SbsaError(status, msg)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dev(t: torch.Tensor, dtype, name: str) -> ctypes.c_void_p:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check_numel(t: torch.Tensor, n: int, name: str):
+    if t.numel() < n:
+        raise ValueError(f"{name} has {t.numel()} elements, needs {n}")
+
+
+# ---------------------------------------------------------------- entry points
+
+def sbsa_version() -> int:
+    return int(load().sbsa_version())
+
+
+def sbsa_status_string(status: int) -> str:
+    return load().sbsa_status_string(int(status)).decode()
+
+
+def sbsa_keep_blocks(num_blocks: int, keep_fraction: float) -> int:
+    return int(load().sbsa_keep_blocks(int(num_blocks), float(keep_fraction)))
+
+
+def sbsa_workspace_bytes(shape: Shape, k_keep: int) -> int:
+    return int(load().sbsa_workspace_bytes(ctypes.byref(shape), int(k_keep)))
+
+
+def sbsa_pool_qk(shape: Shape, q, k, q_mean, k_mean, stream=None):
+    n_in = shape.batch * shape.heads * shape.seq_len_padded * shape.head_dim
+    n_out = shape.batch * shape.heads * shape.num_blocks * shape.head_dim
+    for t, nm, n in ((q, "q", n_in), (k, "k", n_in), (q_mean, "q_mean", n_out), (k_mean, "k_mean", n_out)):
+        _check_numel(t, n, nm)
+    _raise_on(load().sbsa_pool_qk(ctypes.byref(shape), _dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"),
+                                  _dev(q_mean, torch.float32, "q_mean"), _dev(k_mean, torch.float32, "k_mean"),
+                                  _stream(stream)))
+
+
+def sbsa_select_blocks(shape: Shape, q_mean, k_mean, k_keep: int, row_ptr, col_idx, stream=None):
+    rows = shape.batch * shape.heads * shape.num_blocks
+    _check_numel(q_mean, rows * shape.head_dim, "q_mean")
+    _check_numel(k_mean, rows * shape.head_dim, "k_mean")
+    _check_numel(row_ptr, rows + 1, "row_ptr")
+    _check_numel(col_idx, rows * int(k_keep), "col_idx")
+    _raise_on(load().sbsa_select_blocks(ctypes.byref(shape), _dev(q_mean, torch.float32, "q_mean"),
+                                        _dev(k_mean, torch.float32, "k_mean"), int(k_keep),
+                                        _dev(row_ptr, torch.int32, "row_ptr"), _dev(col_idx, torch.int32, "col_idx"),
+                                        _stream(stream)))
+
+
+def sbsa_attention_fwd(shape: Shape, q, k, v, row_ptr, col_idx, scale: float, o, stream=None):
+    n_in = shape.batch * shape.heads * shape.seq_len_padded * shape.head_dim
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _check_numel(t, n_in, nm)
+    _check_numel(row_ptr, shape.batch * shape.heads * shape.num_blocks + 1, "row_ptr")
+    _raise_on(load().sbsa_attention_fwd(ctypes.byref(shape), _dev(q, torch.bfloat16, "q"),
+                                        _dev(k, torch.bfloat16, "k"), _dev(v, torch.bfloat16, "v"),
+                                        _dev(row_ptr, torch.int32, "row_ptr"), _dev(col_idx, torch.int32, "col_idx"),
+                                        float(scale), _dev(o, torch.bfloat16, "o"), _stream(stream)))
+
+
+def sbsa_forward(shape: Shape, q, k, v, k_keep: int, scale: float, o, col_idx_out, workspace, stream=None):
+    n_in = shape.batch * shape.heads * shape.seq_len_padded * shape.head_dim
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _check_numel(t, n_in, nm)
+    ci = ctypes.c_void_p(0)
+    if col_idx_out is not None:
+        _check_numel(col_idx_out, shape.batch * shape.heads * shape.num_blocks * int(k_keep), "col_idx_out")
+        ci = _dev(col_idx_out, torch.int32, "col_idx_out")
+    if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda:
+        raise TypeError("workspace must be a CUDA tensor")
+    _raise_on(load().sbsa_forward(ctypes.byref(shape), _dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"),
+                                  _dev(v, torch.bfloat16, "v"), int(k_keep), float(scale),
+                                  _dev(o, torch.bfloat16, "o"), ci, ctypes.c_void_p(workspace.data_ptr()),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def sbsa_check(stream=None):
+    _raise_on(load().sbsa_check(_stream(stream)))
+
+
+def sbsa_validate_csr(shape: Shape, row_ptr, col_idx, nnz: int, require_diagonal: bool = True, stream=None) -> bool:
+    """True if the CSR list is well formed; False on SBSA_ERR_BAD_INDEX; raises otherwise."""
+    st = load().sbsa_validate_csr(ctypes.byref(shape), _dev(row_ptr, torch.int32, "row_ptr"),
+                                  ctypes.c_void_p(col_idx.data_ptr() if col_idx is not None and col_idx.numel() else 0),
+                                  int(nnz), 1 if require_diagonal else 0, _stream(stream))
+    if st == 6:
+        return False
+    _raise_on(st)
+    return True
+
+
+# ---------------------------------------------------------------- conveniences
+
+def alloc_workspace(shape: Shape, k_keep: int, device="cuda") -> torch.Tensor:
+    """A device byte buffer of sbsa_workspace_bytes() (torch allocations are 256-byte aligned)."""
+    n = sbsa_workspace_bytes(shape, k_keep)
+    if n == 0:
+        raise SbsaError(1, "invalid shape or k_keep for workspace")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def forward_from_host(shape: Shape, q_host, k_host, v_host, k_keep: int, scale: float = 0.0, *, o_host=None,
+                      device_buffers=None, stream=None):
+    """End-to-end call from host tensors: copy Q/K/V (pinned host memory) to the device,
+    run sbsa_forward, copy O back.  ``device_buffers`` (q, k, v, o, workspace) may be
+    passed to reuse device memory across calls.  Returns the host output tensor."""
+    s = stream or torch.cuda.current_stream()
+    if device_buffers is None:
+        dq = torch.empty(q_host.shape, dtype=torch.bfloat16, device="cuda")
+        dk, dv, do = torch.empty_like(dq), torch.empty_like(dq), torch.empty_like(dq)
+        ws = alloc_workspace(shape, k_keep)
+    else:
+        dq, dk, dv, do, ws = device_buffers
+    with torch.cuda.stream(s):
+        dq.copy_(q_host, non_blocking=True)
+        dk.copy_(k_host, non_blocking=True)
+        dv.copy_(v_host, non_blocking=True)
+        sbsa_forward(shape, dq, dk, dv, k_keep, scale, do, None, ws, stream=s)
+        if o_host is None:
+            o_host = torch.empty(do.shape, dtype=do.dtype, pin_memory=True)
+        o_host.copy_(do, non_blocking=True)
+    return o_host
