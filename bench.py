@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Benchmark of the dynamic block-sparse attention layer (pool -> select -> attend).
+
+One step = the whole hot path over one layer's synthetic Q/K/V: block means of Q and
+K, per-query-block top-k selection, and attention inside the kept blocks.  The default
+workload is the long-sequence case: batch 1, 40 heads, d = 128, L = 122,880 tokens
+(24 x 64 x 80 latent grid, 960 blocks of 128), keep 10% (96 key blocks per query
+block, diagonal included).
+
+Prints ONE JSON line (rank 0).  `value` is effective TFLOP/s over the selected blocks
+(4 * Lp * k * block * d * heads per layer, all ranks' layers / max-over-ranks time).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+With N > 1 it runs under torch.distributed (one process per GPU): every rank runs its
+own layer (independent problems, weak scaling, no data-path collective).
+`--impl reference` times the CPU oracle (the reference arm) on this host instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from video_dit_dynamic_b200 import inputs  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="long122880",
+                    help="tiny | 480p | 720p | long122880 | sweep<keep%%> e.g. sweep100")
+    ap.add_argument("--impl", default="sbsa", choices=["sbsa", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-units", type=int, default=16, help="attention units in the CPU sample")
+    return ap.parse_args()
+
+
+def workload(name: str) -> inputs.Workload:
+    if name.startswith("sweep"):
+        return inputs.sweep_workload(int(name[5:]) / 100.0)
+    return inputs.WORKLOADS[name]
+
+
+def keep_count(nb: int, keep: float) -> int:
+    # the library's own sbsa_keep_blocks is used on the GPU path; this mirrors it for
+    # the CPU-only reference arm (round-half-up, clamped to [1, nb])
+    return max(1, min(nb, int(math.floor(keep * nb + 0.5))))
+
+
+def layer_flops(wl: inputs.Workload, k: int) -> float:
+    return 4.0 * wl.seq_len_padded * k * wl.block * wl.head_dim * wl.heads * wl.batch
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = os.path.join("/tmp", f"sbsa_clocks_{os.getpid()}.csv")
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.gpu_id = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            self.gpu_id = None
+
+    def start(self):
+        if self.gpu_id is None:
+            return
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 7:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx.append(float(parts[1]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[3:7]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ traffic record
+def recorded_traffic(kernel_src: str, workload_name: str):
+    """DRAM bytes per attention launch from a committed ncu capture, valid only while
+    the kernel source is unchanged (hash match); else None."""
+    path = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        with open(kernel_src, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()[:16]
+        if rec.get("attn_source_sha256_16") != h:
+            return None
+        return rec.get("dram_bytes_per_launch", {}).get(workload_name)
+    except (OSError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+def cpu_oracle_sample(wl: inputs.Workload, k: int, q, kt, v, n_units: int, seed: int = 0):
+    """Time the oracle on a bounded sample of the layer: pool + select of one full head
+    and attention of n_units (head 0, query block) units; extrapolate to the layer."""
+    import numpy as np
+    import oracle
+    oracle.set_threads(os.cpu_count() or 1)
+    cores = oracle.threads_used()
+    h = 0
+    qb = inputs.bf16_bits(q[:, h:h + 1])
+    kb = inputs.bf16_bits(kt[:, h:h + 1])
+    vb = inputs.bf16_bits(v[:, h:h + 1])
+    L, blk, nb = wl.seq_len, wl.block, wl.num_blocks
+    t0 = time.perf_counter()
+    qm = oracle.pool(qb, L, blk)
+    km = oracle.pool(kb, L, blk)
+    col = oracle.select(qm, km, k)
+    t_ps = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    units = sorted(rng.choice(nb, size=min(n_units, nb), replace=False).tolist())
+    rp = oracle.uniform_row_ptr(1, 1, nb, k)
+    t0 = time.perf_counter()
+    oracle.attention(qb, kb, vb, L, blk, rp, col, units=units)
+    t_at = time.perf_counter() - t0
+    heads = wl.heads * wl.batch
+    layer_s = t_ps * heads + t_at / len(units) * (nb * heads)
+    tflops = layer_flops(wl, k) / layer_s / 1e12
+    return {
+        "value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+        "sample": (f"pool+select of 1 of {heads} heads ({t_ps:.2f} s) and attention of {len(units)} of "
+                   f"{nb * heads} (head, query-block) units ({t_at:.2f} s), extrapolated to the layer: "
+                   f"{layer_s:.1f} s/layer"),
+        "layer_seconds_extrapolated": layer_s,
+    }
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, wl):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    nb = wl.num_blocks
+    k = keep_count(nb, wl.keep)
+    q, kt, v = inputs.make_qkv(inputs.Workload(wl.name, 1, 1, wl.grid, wl.head_dim, wl.block, wl.keep),
+                               seed=0, device="cpu")
+    # every step is a bounded sample (one head) of the same layer, extrapolated
+    results = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_oracle_sample(inputs.Workload(wl.name, 1, wl.heads, wl.grid, wl.head_dim, wl.block, wl.keep),
+                              k, q, kt, v, n_units=args.cpu_units, seed=i)
+        if i >= args.warmup:
+            results.append(r)
+    layer_s = statistics.mean(r["layer_seconds_extrapolated"] for r in results)
+    value = layer_flops(wl, k) / layer_s / 1e12
+    cb = dict(results[-1])
+    cb["value"] = value
+    cb.pop("layer_seconds_extrapolated", None)
+    line = {
+        "impl": "reference", "metric": "sparse-attn ms/layer & TFLOP/s (selected blocks) at L=122880, 90% sparse",
+        "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": layer_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl, k, "oracle on host cores; sample per step, extrapolated"),
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl, k, note):
+    return {"workload": f"{wl.name}: B={wl.batch} H={wl.heads} d={wl.head_dim} L={wl.seq_len} "
+                        f"(Lp={wl.seq_len_padded}, grid {'x'.join(map(str, wl.grid))}) block={wl.block} "
+                        f"keep={wl.keep:g} (k={k} of {wl.num_blocks})",
+            "batch": wl.batch, "heads": wl.heads, "head_dim": wl.head_dim, "seq_len": wl.seq_len,
+            "seq_len_padded": wl.seq_len_padded, "block": wl.block, "keep": wl.keep, "k_blocks": k,
+            "num_blocks": wl.num_blocks, "parallelism": "replica per GPU (independent layers)",
+            "l2": "inputs larger than L2 (Q+K+V = %.2f GB)" % (3 * wl.batch * wl.heads * wl.seq_len_padded *
+                                                                wl.head_dim * 2 / 1e9),
+            "note": note}
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gpu(args, wl):
+    from video_dit_dynamic_b200 import sbsa
+
+    ws_n, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    pg = None
+    if ws_n > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    dev = torch.device("cuda", local)
+    sbsa.load()
+    nb = wl.num_blocks
+    k = sbsa.sbsa_keep_blocks(nb, wl.keep)
+    shape = sbsa.make_shape(wl.batch, wl.heads, wl.seq_len, wl.head_dim, wl.block)
+    q, kt, v = inputs.make_qkv(wl, seed=rank, device=dev)
+    rows = wl.batch * wl.heads * nb
+    qm = torch.empty(rows * wl.head_dim, dtype=torch.float32, device=dev)
+    km = torch.empty_like(qm)
+    rp = torch.empty(rows + 1, dtype=torch.int32, device=dev)
+    ci = torch.empty(rows * k, dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+    flops = layer_flops(wl, k)
+    pool_bytes = 2 * q.numel() * 2 + 2 * qm.numel() * 4
+
+    def step(evs=None):
+        # sbsa_forward issues exactly these three launches; they are called one by one
+        # here so that each kernel's time can be read from events on the same stream
+        if evs: evs[0].record(stream)
+        sbsa.sbsa_pool_qk(shape, q, kt, qm, km, stream=stream)
+        if evs: evs[1].record(stream)
+        sbsa.sbsa_select_blocks(shape, qm, km, k, rp, ci, stream=stream)
+        if evs: evs[2].record(stream)
+        sbsa.sbsa_attention_fwd(shape, q, kt, v, rp, ci, 0.0, o, stream=stream)
+        if evs: evs[3].record(stream)
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    sbsa.sbsa_check(stream)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    barrier()
+    clk = clocks.stop()
+    sbsa.sbsa_check(stream)
+    elapsed_ms = t_start.elapsed_time(t_end)
+    pool_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    sel_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    att_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    # the same step through the fused entry point, for cross-checking
+    ws_buf = sbsa.alloc_workspace(shape, k, device=dev)
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    sbsa.sbsa_forward(shape, q, kt, v, k, 0.0, o, None, ws_buf, stream=stream)
+    torch.cuda.synchronize(dev)
+    f0.record(stream)
+    for _ in range(min(args.steps, 5)):
+        sbsa.sbsa_forward(shape, q, kt, v, k, 0.0, o, None, ws_buf, stream=stream)
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    forward_ms = f0.elapsed_time(f1) / min(args.steps, 5)
+    sbsa.sbsa_check(stream)
+
+    # end to end through the public API from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (t.cpu().pin_memory() for t in (q, kt, v))
+        oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        bufs = (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q), torch.empty_like(q), ws_buf)
+        for _ in range(2):
+            sbsa.forward_from_host(shape, qh, kh, vh, k, o_host=oh, device_buffers=bufs, stream=stream)
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 5))
+        e0.record(stream)
+        for _ in range(n_e2e):
+            sbsa.forward_from_host(shape, qh, kh, vh, k, o_host=oh, device_buffers=bufs, stream=stream)
+        e1.record(stream)
+        barrier()
+        sbsa.sbsa_check(stream)
+        e2e_ms = e0.elapsed_time(e1) / n_e2e
+        e2e = {"ms": e2e_ms, "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2}
+
+    def max_over_ranks(x: float) -> float:
+        if pg is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    elapsed_ms = max_over_ranks(elapsed_ms)
+    att_avg = max_over_ranks(statistics.mean(att_ms))
+    pool_avg = max_over_ranks(statistics.mean(pool_ms))
+    sel_avg = max_over_ranks(statistics.mean(sel_ms))
+    forward_ms = max_over_ranks(forward_ms)
+    if e2e is not None:
+        e2e["ms"] = max_over_ranks(e2e["ms"])
+    ms_step = elapsed_ms / args.steps
+    value = flops * ws_n / (ms_step / 1e3) / 1e12
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        att_tflops = flops / (att_avg / 1e3) / 1e12
+        traffic = recorded_traffic(os.path.join(ROOT, "video_dit_dynamic_b200", "csrc", "attn.cuh"), wl.name)
+        pool_gbs = pool_bytes / (pool_avg / 1e3) / 1e9
+        line = {
+            "metric": "sparse-attn ms/layer & TFLOP/s (selected blocks) at L=122880, 90% sparse",
+            "value": value, "unit": "TFLOP/s", "n_gpus": ws_n, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": config_of(wl, k, "step = pool + select + attention of one layer; value = selected-block "
+                                       "FLOP / step time"),
+            "clocks": clk,
+            "gpu_launches": 3 * args.steps,
+            "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": att_tflops / peaks["bf16_tflops"], "traffic": traffic,
+                         "kernel": f"attn_kernel<{wl.head_dim},{wl.block}>",
+                         "peak_source": f"{peak_src} bf16 dense (burst)",
+                         "frac_of_sustained": att_tflops / peaks["bf16_tflops_sustained"],
+                         "algorithmic_flop_per_launch": flops, "avg_launch_ms": att_avg},
+            "kernels": {
+                "pool": {"ms": pool_avg, "GB/s": pool_gbs, "hbm_frac": pool_gbs / peaks["hbm_gbs"],
+                         "algorithmic_bytes": pool_bytes},
+                "select": {"ms": sel_avg, "flop": 2.0 * wl.batch * wl.heads * nb * nb * wl.head_dim},
+                "pool_plus_select_effective_GB/s": pool_bytes / ((pool_avg + sel_avg) / 1e3) / 1e9,
+                "attention": {"ms": att_avg, "TFLOP/s": att_tflops},
+                "sbsa_forward_ms": forward_ms,
+            },
+            "peaks": {"source": peak_src, **peaks},
+        }
+        if e2e is not None:
+            line["e2e"] = {"value": flops * ws_n / (e2e["ms"] / 1e3) / 1e12, "unit": "TFLOP/s",
+                           "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
+                           "d2h_bytes_per_step": e2e["d2h_bytes_per_step"], "ms_per_step": e2e["ms"]}
+        if ws_n == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_oracle_sample(wl, k, q, kt, v, args.cpu_units)
+            line["cpu_baseline"].pop("layer_seconds_extrapolated", None)
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    wl = workload(args.workload)
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_gpu(args, wl)
+
+
+if __name__ == "__main__":
+    main()
