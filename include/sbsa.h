@@ -128,6 +128,27 @@ sbsa_status sbsa_forward(const sbsa_shape *shape, const void *q, const void *k, 
                          float scale, void *o, int32_t *col_idx_out, void *workspace, size_t workspace_bytes,
                          void *stream);
 
+/* sbsa_forward without a workspace, for callers that cannot allocate device memory:
+ * for example a plug-in inside another engine that owns every device allocation, or
+ * a latency-critical loop where cudaMalloc/cudaFree would synchronize the device.
+ * The pages describe no such call; it exists only for these callers.
+ *   Same arguments, results and launches as sbsa_forward, minus the workspace.  The
+ *   block means and the CSR list go to a 16 MiB scratch array that the library
+ *   reserves on every GPU it is loaded on, for the life of the process.  Shapes
+ *   with sbsa_workspace_bytes(shape, k_keep) > 16 MiB (16,777,216 bytes) are rejected
+ *   with SBSA_ERR_WORKSPACE before anything is launched.  Example: the 480p case
+ *   (40 heads, 256 blocks of 128, d = 128, k = 51) needs 12.6 MB.
+ *   The first call on a device looks up the scratch array's device address, with
+ *   that device current; make that first call before any stream capture.
+ *   All calls share the one array, and it keeps the last call's contents.  Calls
+ *   whose work overlaps on the GPU (different streams, or different host threads
+ *   without ordering) race on it and must be serialized by the caller.  Every scratch
+ *   element read within a call is written earlier in the same call, so nothing needs
+ *   clearing.  This call allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ *   library routine. */
+sbsa_status sbsa_forward_noalloc(const sbsa_shape *shape, const void *q, const void *k, const void *v,
+                                 int32_t k_keep, float scale, void *o, int32_t *col_idx_out, void *stream);
+
 /* Synchronizes `stream`, then reads and clears the calling device's error word.
  * Returns SBSA_OK, SBSA_ERR_TIMEOUT, SBSA_ERR_BAD_INDEX or SBSA_ERR_CUDA (a sticky
  * CUDA error or a failed synchronize). */

@@ -241,6 +241,38 @@ __global__ void validate_csr_kernel(const int32_t* row_ptr, const int32_t* col_i
 }
 
 }  // namespace
+
+// ---------------------------------------------------------------- allocation-free forward
+// Scratch for sbsa_forward_noalloc: block means and the CSR block list live in this
+// fixed module-scope array instead of a caller-provided workspace.  Every GPU that
+// loads the library reserves it for the life of the process.  Host code must never
+// hand the symbol itself to a kernel (on the host it is only a stand-in); its device
+// address is looked up once per device with cudaGetSymbolAddress.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 256;
+void* g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device (looked up on first use).
+sbsa_status noalloc_scratch(void** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(SBSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SBSA_OK;
+}
+}  // namespace
 }  // namespace sbsa
 
 using namespace sbsa;
@@ -343,6 +375,39 @@ sbsa_status sbsa_forward(const sbsa_shape* shape, const void* q, const void* k, 
     int32_t* rp = reinterpret_cast<int32_t*>(ws + w.row_ptr);
     int32_t* ci = col_idx_out ? col_idx_out : reinterpret_cast<int32_t*>(ws + w.col_idx);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((r = launch_pool(shape, q, k, qm, km, st)) != SBSA_OK) return r;
+    if ((r = launch_select(shape, qm, km, k_keep, rp, ci, st)) != SBSA_OK) return r;
+    if ((r = launch_attn(shape, q, k, v, rp, ci, resolve_scale(shape, scale), o, st)) != SBSA_OK) return r;
+    return ok();
+}
+
+sbsa_status sbsa_forward_noalloc(const sbsa_shape* shape, const void* q, const void* k, const void* v,
+                                 int32_t k_keep, float scale, void* o, int32_t* col_idx_out, void* stream) {
+    sbsa_status r = check_shape(shape);
+    if (r != SBSA_OK) return r;
+    if ((r = check_k(shape, k_keep)) != SBSA_OK) return r;
+    if (!q || !k || !v || !o) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return fail(SBSA_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
+    if (col_idx_out && (reinterpret_cast<uintptr_t>(col_idx_out) & 3u))
+        return fail(SBSA_ERR_INVALID_ARG, "col_idx_out must be 4-byte aligned");
+    if (!std::isfinite(scale)) return fail(SBSA_ERR_INVALID_ARG, "scale must be finite");
+    const WsLayout w = ws_layout(shape, k_keep);
+    if (w.total > kNoAllocScratchBytes)
+        return fail(SBSA_ERR_WORKSPACE,
+                    "this shape needs %zu bytes of scratch; the built-in scratch holds %zu (use sbsa_forward "
+                    "with a workspace)",
+                    w.total, kNoAllocScratchBytes);
+    void* scratch = nullptr;
+    if ((r = noalloc_scratch(&scratch)) != SBSA_OK) return r;
+    uint8_t* ws = static_cast<uint8_t*>(scratch);
+    float* qm = reinterpret_cast<float*>(ws + w.q_mean);
+    float* km = reinterpret_cast<float*>(ws + w.k_mean);
+    int32_t* rp = reinterpret_cast<int32_t*>(ws + w.row_ptr);
+    int32_t* ci = col_idx_out ? col_idx_out : reinterpret_cast<int32_t*>(ws + w.col_idx);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // every scratch element the later kernels read is written earlier in this call,
+    // so nothing needs clearing between calls
     if ((r = launch_pool(shape, q, k, qm, km, st)) != SBSA_OK) return r;
     if ((r = launch_select(shape, qm, km, k_keep, rp, ci, st)) != SBSA_OK) return r;
     if ((r = launch_attn(shape, q, k, v, rp, ci, resolve_scale(shape, scale), o, st)) != SBSA_OK) return r;

@@ -23,7 +23,7 @@ STATUS_NAMES = {0: "SBSA_OK", 1: "SBSA_ERR_INVALID_ARG", 2: "SBSA_ERR_UNSUPPORTE
 # Every symbol include/sbsa.h declares.
 EXPORTS = ("sbsa_version", "sbsa_status_string", "sbsa_last_error_message", "sbsa_keep_blocks",
            "sbsa_workspace_bytes", "sbsa_pool_qk", "sbsa_select_blocks", "sbsa_attention_fwd", "sbsa_forward",
-           "sbsa_check", "sbsa_validate_csr")
+           "sbsa_check", "sbsa_validate_csr", "sbsa_forward_noalloc")
 
 
 class SbsaError(RuntimeError):
@@ -81,10 +81,11 @@ def load(path: str | None = None):
     lib.sbsa_select_blocks.argtypes = [SP, P, P, I32, P, P, P]
     lib.sbsa_attention_fwd.argtypes = [SP, P, P, P, P, P, ctypes.c_float, P, P]
     lib.sbsa_forward.argtypes = [SP, P, P, P, I32, ctypes.c_float, P, P, P, SZ, P]
+    lib.sbsa_forward_noalloc.argtypes = [SP, P, P, P, I32, ctypes.c_float, P, P, P]
     lib.sbsa_check.argtypes = [P]
     lib.sbsa_validate_csr.argtypes = [SP, P, P, ctypes.c_int64, I32, P]
     for name in ("sbsa_pool_qk", "sbsa_select_blocks", "sbsa_attention_fwd", "sbsa_forward", "sbsa_check",
-                 "sbsa_validate_csr"):
+                 "sbsa_validate_csr", "sbsa_forward_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -182,6 +183,22 @@ def sbsa_forward(shape: Shape, q, k, v, k_keep: int, scale: float, o, col_idx_ou
                                   _dev(v, torch.bfloat16, "v"), int(k_keep), float(scale),
                                   _dev(o, torch.bfloat16, "o"), ci, ctypes.c_void_p(workspace.data_ptr()),
                                   workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def sbsa_forward_noalloc(shape: Shape, q, k, v, k_keep: int, scale: float, o, col_idx_out=None, stream=None):
+    """sbsa_forward for callers that cannot allocate device memory (no workspace: the
+    library's built-in 16 MiB scratch array holds the block means and block lists).
+    Calls that overlap on the GPU share that array and must be serialized."""
+    n_in = shape.batch * shape.heads * shape.seq_len_padded * shape.head_dim
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _check_numel(t, n_in, nm)
+    ci = ctypes.c_void_p(0)
+    if col_idx_out is not None:
+        _check_numel(col_idx_out, shape.batch * shape.heads * shape.num_blocks * int(k_keep), "col_idx_out")
+        ci = _dev(col_idx_out, torch.int32, "col_idx_out")
+    _raise_on(load().sbsa_forward_noalloc(ctypes.byref(shape), _dev(q, torch.bfloat16, "q"),
+                                          _dev(k, torch.bfloat16, "k"), _dev(v, torch.bfloat16, "v"), int(k_keep),
+                                          float(scale), _dev(o, torch.bfloat16, "o"), ci, _stream(stream)))
 
 
 def sbsa_check(stream=None):
