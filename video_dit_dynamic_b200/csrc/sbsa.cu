@@ -174,15 +174,18 @@ sbsa_status launch_attn_t(const sbsa_shape* s, const void* q, const void* k, con
     p.row_ptr = rp;
     p.col_idx = ci;
     p.o = static_cast<__nv_bfloat16*>(o);
+    p.units = num_rows(s);
     p.L = s->seq_len;
     p.Lp = s->seq_len_padded;
     p.nb = num_blocks(s);
-    p.scale_log2 = scale * 1.4426950408889634f;
+    p.scale_log2 = std::fabs(scale) * 1.4426950408889634f;
+    p.neg_scale = scale < 0.f ? 1 : 0;
     p.epoch = g_epoch.fetch_add(1);
     auto kern = attn_kernel<D, BLK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "attention smem attribute");
-    kern<<<static_cast<unsigned>(num_rows(s)), 192, C::kSmemBytes, st>>>(mq, mk, mv, p);
+    const long long ctas = (p.units + 1) / 2;  // two query tiles per CTA
+    kern<<<static_cast<unsigned>(ctas), C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
     e = cudaGetLastError();
     return e == cudaSuccess ? SBSA_OK : cuda_fail(e, "attention launch");
 }
