@@ -143,10 +143,31 @@ sbsa_status launch_select_t(const sbsa_shape* s, const float* qm, const float* k
     return e == cudaSuccess ? SBSA_OK : cuda_fail(e, "select launch");
 }
 
+template <int KPL>
+sbsa_status launch_select_gemm(const sbsa_shape* s, const float* qm, const float* km, int k, int32_t* rp, int32_t* ci,
+                               cudaStream_t st) {
+    const int nb = num_blocks(s);
+    const size_t smem = select_gemm_smem_bytes(KPL);
+    auto kern = select_gemm_kernel<KPL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_fail(e, "select smem attribute");
+    const dim3 grid((nb + kSelQT - 1) / kSelQT, static_cast<unsigned>(s->batch * s->heads));
+    kern<<<grid, 256, smem, st>>>(qm, km, nb, k, rp, ci, num_rows(s));
+    e = cudaGetLastError();
+    return e == cudaSuccess ? SBSA_OK : cuda_fail(e, "select launch");
+}
+
 template <int D>
 sbsa_status launch_select_d(const sbsa_shape* s, const float* qm, const float* km, int k, int32_t* rp, int32_t* ci,
                             cudaStream_t st) {
     const int nb = num_blocks(s);
+    if constexpr (D == 128) {
+        // register-blocked GEMM path (head_dim 128, up to 1024 blocks)
+        if (nb <= 64) return launch_select_gemm<2>(s, qm, km, k, rp, ci, st);
+        if (nb <= 256) return launch_select_gemm<8>(s, qm, km, k, rp, ci, st);
+        if (nb <= 512) return launch_select_gemm<16>(s, qm, km, k, rp, ci, st);
+        if (nb <= 1024) return launch_select_gemm<32>(s, qm, km, k, rp, ci, st);
+    }
     if (nb <= 64) return launch_select_t<D, 2>(s, qm, km, k, rp, ci, st);
     if (nb <= 256) return launch_select_t<D, 8>(s, qm, km, k, rp, ci, st);
     if (nb <= 512) return launch_select_t<D, 16>(s, qm, km, k, rp, ci, st);

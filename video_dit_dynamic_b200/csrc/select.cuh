@@ -26,6 +26,68 @@ __device__ __forceinline__ uint32_t order_key(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Keep, for query block i, the diagonal and the k_keep-1 largest of the other keys
+// (ties: lower j), writing them in ascending j.  One warp; lane l holds keys
+// j = l + 32 s.  The (k-1)-th largest key T is found by bisection on the key bits with
+// warp-wide counts, stopping early once exactly k-1 keys lie at or above the candidate.
+template <int KPL>
+__device__ __forceinline__ void select_row_topk(const uint32_t* __restrict__ keys_row, int nb, int i, int k_keep,
+                                                long long row, int32_t* __restrict__ row_ptr,
+                                                int32_t* __restrict__ col_idx) {
+    const int lane = threadIdx.x % 32;
+    const uint32_t lt = lanemask_lt();
+    const int kk = k_keep - 1;  // off-diagonal blocks to keep
+    uint32_t key[KPL];
+#pragma unroll
+    for (int s = 0; s < KPL; ++s) {
+        const int j = s * 32 + lane;
+        // non-candidates (padding, the diagonal) get key 0 and are excluded by index below
+        key[s] = (j < nb && j != i) ? keys_row[j] : 0u;
+    }
+    uint32_t T = 0u;
+    if (kk > 0) {
+#pragma unroll 1
+        for (int bit = 31; bit >= 0; --bit) {
+            const uint32_t cand = T | (1u << bit);
+            int cnt = 0;
+#pragma unroll
+            for (int s = 0; s < KPL; ++s) {
+                const int j = s * 32 + lane;
+                cnt += (j < nb && j != i && key[s] >= cand) ? 1 : 0;
+            }
+            cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
+            if (cnt >= kk) T = cand;
+            if (cnt == kk) break;  // {key >= cand} is exactly the top k-1
+        }
+    }
+    int n_gt = 0;
+    if (kk > 0) {
+#pragma unroll
+        for (int s = 0; s < KPL; ++s) {
+            const int j = s * 32 + lane;
+            n_gt += (j < nb && j != i && key[s] > T) ? 1 : 0;
+        }
+        n_gt = __reduce_add_sync(0xFFFFFFFFu, n_gt);
+    }
+    const int need_eq = kk - n_gt;  // how many keys equal to T to keep (lowest j first)
+    int32_t* out = col_idx + row * k_keep;
+    int pos = 0, eq_seen = 0;
+#pragma unroll
+    for (int s = 0; s < KPL; ++s) {
+        const int j = s * 32 + lane;
+        const bool cand = j < nb && j != i;
+        const bool is_eq = kk > 0 && cand && key[s] == T;
+        const uint32_t eq_mask = __ballot_sync(0xFFFFFFFFu, is_eq);
+        const int eq_rank = eq_seen + __popc(eq_mask & lt);
+        const bool keep = (j == i) || (kk > 0 && cand && key[s] > T) || (is_eq && eq_rank < need_eq);
+        const uint32_t m = __ballot_sync(0xFFFFFFFFu, keep);
+        if (keep) out[pos + __popc(m & lt)] = j;
+        pos += __popc(m);
+        eq_seen += __popc(eq_mask);
+    }
+    if (lane == 0) row_ptr[row] = static_cast<int32_t>(row * k_keep);
+}
+
 template <int D, int QT, int KPL>
 __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ q_mean,
                                                      const float* __restrict__ k_mean, int nb, int k_keep,
@@ -72,62 +134,113 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ q
     __syncthreads();
 
     // ---- top-k per row, one warp per row
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const uint32_t lt = lanemask_lt();
-    const int kk = k_keep - 1;  // off-diagonal blocks to keep
-    for (int r = warp; r < nq; r += blockDim.x / 32) {
-        const int i = i0 + r;
-        uint32_t key[KPL];
-#pragma unroll
-        for (int s = 0; s < KPL; ++s) {
-            const int j = s * 32 + lane;
-            key[s] = (j < nb) ? keys[r * NBP + j] : 0u;
-        }
-        // candidates: j < nb and j != i.  T = kk-th largest candidate key (kk >= 1).
-        uint32_t T = 0u;
-        if (kk > 0) {
-#pragma unroll 1
-            for (int bit = 31; bit >= 0; --bit) {
-                const uint32_t cand = T | (1u << bit);
-                int cnt = 0;
-#pragma unroll
-                for (int s = 0; s < KPL; ++s) {
-                    const int j = s * 32 + lane;
-                    cnt += (j < nb && j != i && key[s] >= cand) ? 1 : 0;
-                }
-                cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
-                if (cnt >= kk) T = cand;
-            }
-        }
-        int n_gt = 0;
-        if (kk > 0) {
-#pragma unroll
-            for (int s = 0; s < KPL; ++s) {
-                const int j = s * 32 + lane;
-                n_gt += (j < nb && j != i && key[s] > T) ? 1 : 0;
-            }
-            n_gt = __reduce_add_sync(0xFFFFFFFFu, n_gt);
-        }
-        const int need_eq = kk - n_gt;  // how many keys equal to T to keep (lowest j first)
-        const long long row = bh * nb + i;
-        int32_t* out = col_idx + row * k_keep;
-        int pos = 0, eq_seen = 0;
-#pragma unroll
-        for (int s = 0; s < KPL; ++s) {
-            const int j = s * 32 + lane;
-            const bool cand = j < nb && j != i;
-            const bool is_eq = kk > 0 && cand && key[s] == T;
-            const uint32_t eq_mask = __ballot_sync(0xFFFFFFFFu, is_eq);
-            const int eq_rank = eq_seen + __popc(eq_mask & lt);
-            const bool keep = (j == i) || (kk > 0 && cand && key[s] > T) || (is_eq && eq_rank < need_eq);
-            const uint32_t m = __ballot_sync(0xFFFFFFFFu, keep);
-            if (keep) out[pos + __popc(m & lt)] = j;
-            pos += __popc(m);
-            eq_seen += __popc(eq_mask);
-        }
-        if (lane == 0) row_ptr[row] = static_cast<int32_t>(row * k_keep);
-    }
+    const int warp = threadIdx.x / 32;
+    for (int r = warp; r < nq; r += blockDim.x / 32)
+        select_row_topk<KPL>(keys + r * NBP, nb, i0 + r, k_keep, bh * nb + i0 + r, row_ptr, col_idx);
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) row_ptr[n_rows] = static_cast<int32_t>(n_rows * k_keep);
+}
+
+// Scores through a shared-memory, register-blocked fp32 GEMM, for nb <= 1024.
+// CTA = (b*h, 32 query blocks), 256 threads.  Key means stream through shared memory
+// in chunks of 256 key blocks x 32 channels.  Thread (warp w, lane l) owns query rows
+// {l/8 + 4 r : r < 8} and key blocks {256 c + 32 w + l%8 + 8 s : s < 4}; rows and key
+// blocks interleave so that each shared-memory load is conflict-free or broadcast.
+// Products accumulate over channel pairs with packed fp32x2 FMAs, (even, odd) channel
+// partial sums added at the end.  Then one warp per row selects as above.
+constexpr int kSelQT = 32;
+constexpr int kSelQStride = 132;  // floats per query-mean row in shared memory (128 + 4)
+constexpr int kSelKStride = 36;   // floats per key-mean row of a 32-channel chunk (32 + 4)
+constexpr int kSelJChunk = 256;
+constexpr int kSelCChunk = 32;
+
+template <int KPL>
+__global__ void __launch_bounds__(256, 1) select_gemm_kernel(const float* __restrict__ q_mean,
+                                                            const float* __restrict__ k_mean, int nb, int k_keep,
+                                                            int32_t* __restrict__ row_ptr,
+                                                            int32_t* __restrict__ col_idx, long long n_rows) {
+    constexpr int D = 128;
+    constexpr int NBP = 32 * KPL;
+    extern __shared__ __align__(16) uint8_t sel_smem[];
+    float* qs = reinterpret_cast<float*>(sel_smem);                        // [32][132]
+    float* ks = qs + kSelQT * kSelQStride;                                 // [2][256][36]
+    uint32_t* keys = reinterpret_cast<uint32_t*>(ks + 2 * kSelJChunk * kSelKStride);  // [32][NBP]
+
+    const long long bh = blockIdx.y;
+    const int i0 = blockIdx.x * kSelQT;
+    const int nq = min(kSelQT, nb - i0);
+    const float* qm = q_mean + (bh * nb + i0) * D;
+    const float* km = k_mean + bh * nb * D;
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+
+    // query means -> qs (rows past nq are zero)
+    for (int f = tid; f < kSelQT * D / 4; f += 256) {
+        const int r = f / (D / 4), c4 = f % (D / 4);
+        const float4 v = r < nq ? __ldg(reinterpret_cast<const float4*>(qm) + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(qs + r * kSelQStride + c4 * 4) = v;
+    }
+
+    const int li = lane / 8, lj = lane % 8;
+    auto load_chunk = [&](int jc, int cc, float* dst) {
+        // 256 key rows x 32 channels = 2048 float4, 8 per thread, coalesced along channels
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int f = tid + 256 * r;
+            const int row = f / 8, q4 = f % 8;
+            const int j = jc + row;
+            const float4 v = j < nb ? __ldg(reinterpret_cast<const float4*>(km + static_cast<long long>(j) * D + cc * kSelCChunk) + q4)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4*>(dst + row * kSelKStride + q4 * 4) = v;
+        }
+    };
+
+    for (int jc = 0; jc < nb; jc += kSelJChunk) {
+        float2 acc[8][4];
+#pragma unroll
+        for (int a = 0; a < 8; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[a][b] = make_float2(0.f, 0.f);
+        __syncthreads();  // previous chunk's readers are done with ks
+        load_chunk(jc, 0, ks);
+        for (int cc = 0; cc < D / kSelCChunk; ++cc) {
+            float* cur = ks + (cc & 1) * kSelJChunk * kSelKStride;
+            __syncthreads();  // cur is filled; the other buffer is free
+            if (cc + 1 < D / kSelCChunk) load_chunk(jc, cc + 1, ks + ((cc + 1) & 1) * kSelJChunk * kSelKStride);
+#pragma unroll
+            for (int c = 0; c < kSelCChunk; c += 4) {
+                float4 qv[8], kv[4];
+#pragma unroll
+                for (int a = 0; a < 8; ++a)
+                    qv[a] = *reinterpret_cast<const float4*>(qs + (li + 4 * a) * kSelQStride + cc * kSelCChunk + c);
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    kv[b] = *reinterpret_cast<const float4*>(cur + (warp * 32 + lj + 8 * b) * kSelKStride + c);
+#pragma unroll
+                for (int a = 0; a < 8; ++a)
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        acc[a][b] = __ffma2_rn(make_float2(qv[a].x, qv[a].y), make_float2(kv[b].x, kv[b].y), acc[a][b]);
+                        acc[a][b] = __ffma2_rn(make_float2(qv[a].z, qv[a].w), make_float2(kv[b].z, kv[b].w), acc[a][b]);
+                    }
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < 8; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int j = jc + warp * 32 + lj + 8 * b;
+                if (j < NBP) keys[(li + 4 * a) * NBP + j] = order_key(acc[a][b].x + acc[a][b].y);
+            }
+    }
+    __syncthreads();
+
+    for (int r = warp; r < nq; r += 8)
+        select_row_topk<KPL>(keys + r * NBP, nb, i0 + r, k_keep, bh * nb + i0 + r, row_ptr, col_idx);
+    if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) row_ptr[n_rows] = static_cast<int32_t>(n_rows * k_keep);
+}
+
+constexpr size_t select_gemm_smem_bytes(int KPL) {
+    return (static_cast<size_t>(kSelQT) * kSelQStride + 2ull * kSelJChunk * kSelKStride) * 4 +
+           static_cast<size_t>(kSelQT) * 32 * KPL * 4;
 }
 
 }  // namespace sbsa
