@@ -11,8 +11,8 @@
 //            and forms its dot product with the QT query means broadcast from shared
 //            memory; the fp32 scores go to shared memory as order-preserving uint32 keys.
 //   top-k  : one warp per query row.  Lane l holds keys j = l + 32 r.  The (k-1)-th
-//            largest key T is found by a 32-step bisection on the key bits (warp-wide
-//            counts); then keys > T are kept, and keys == T in ascending j until k-1
+//            largest key T is found by bisection on the key bits (warp-wide counts,
+//            early exit); then keys > T are kept, and keys == T in ascending j until k-1
 //            are kept; the output position of each kept j is a ballot prefix count,
 //            which yields the ascending order directly.
 #pragma once
@@ -41,33 +41,31 @@ __device__ __forceinline__ void select_row_topk(const uint32_t* __restrict__ key
 #pragma unroll
     for (int s = 0; s < KPL; ++s) {
         const int j = s * 32 + lane;
-        // non-candidates (padding, the diagonal) get key 0 and are excluded by index below
-        key[s] = (j < nb && j != i) ? keys_row[j] : 0u;
+        // non-candidates (padding, the diagonal) get key 0; every bisection candidate is
+        // >= 1, so they never count (a real score's key is >= 1: only the all-ones NaN
+        // pattern maps to 0, and it is clamped to 1)
+        key[s] = (j < nb && j != i) ? max(keys_row[j], 1u) : 0u;
     }
     uint32_t T = 0u;
     if (kk > 0) {
 #pragma unroll 1
         for (int bit = 31; bit >= 0; --bit) {
             const uint32_t cand = T | (1u << bit);
-            int cnt = 0;
+            // four independent partial counts keep the add chains short
+            int c4[4] = {0, 0, 0, 0};
 #pragma unroll
-            for (int s = 0; s < KPL; ++s) {
-                const int j = s * 32 + lane;
-                cnt += (j < nb && j != i && key[s] >= cand) ? 1 : 0;
-            }
-            cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
+            for (int s = 0; s < KPL; ++s) c4[s & 3] += key[s] >= cand ? 1 : 0;
+            const int cnt = __reduce_add_sync(0xFFFFFFFFu, (c4[0] + c4[1]) + (c4[2] + c4[3]));
             if (cnt >= kk) T = cand;
             if (cnt == kk) break;  // {key >= cand} is exactly the top k-1
         }
     }
     int n_gt = 0;
     if (kk > 0) {
+        int g4[4] = {0, 0, 0, 0};
 #pragma unroll
-        for (int s = 0; s < KPL; ++s) {
-            const int j = s * 32 + lane;
-            n_gt += (j < nb && j != i && key[s] > T) ? 1 : 0;
-        }
-        n_gt = __reduce_add_sync(0xFFFFFFFFu, n_gt);
+        for (int s = 0; s < KPL; ++s) g4[s & 3] += key[s] > T ? 1 : 0;
+        n_gt = __reduce_add_sync(0xFFFFFFFFu, (g4[0] + g4[1]) + (g4[2] + g4[3]));
     }
     const int need_eq = kk - n_gt;  // how many keys equal to T to keep (lowest j first)
     int32_t* out = col_idx + row * k_keep;
@@ -75,7 +73,7 @@ __device__ __forceinline__ void select_row_topk(const uint32_t* __restrict__ key
 #pragma unroll
     for (int s = 0; s < KPL; ++s) {
         const int j = s * 32 + lane;
-        const bool cand = j < nb && j != i;
+        const bool cand = key[s] != 0u;  // j < nb and j != i
         const bool is_eq = kk > 0 && cand && key[s] == T;
         const uint32_t eq_mask = __ballot_sync(0xFFFFFFFFu, is_eq);
         const int eq_rank = eq_seen + __popc(eq_mask & lt);
@@ -181,16 +179,19 @@ __global__ void __launch_bounds__(256, 1) select_gemm_kernel(const float* __rest
 
     const int li = lane / 8, lj = lane % 8;
     auto load_chunk = [&](int jc, int cc, float* dst) {
-        // 256 key rows x 32 channels = 2048 float4, 8 per thread, coalesced along channels
+        // 256 key rows x 32 channels = 2048 x 16 B, 8 per thread, asynchronous copies
+        // (coalesced along channels; rows past nb are zero-filled)
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
             const int f = tid + 256 * r;
             const int row = f / 8, q4 = f % 8;
             const int j = jc + row;
-            const float4 v = j < nb ? __ldg(reinterpret_cast<const float4*>(km + static_cast<long long>(j) * D + cc * kSelCChunk) + q4)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-            *reinterpret_cast<float4*>(dst + row * kSelKStride + q4 * 4) = v;
+            const float* src = km + static_cast<long long>(j < nb ? j : 0) * D + cc * kSelCChunk + q4 * 4;
+            const uint32_t dst_s = smem_u32(dst + row * kSelKStride + q4 * 4);
+            const uint32_t bytes = j < nb ? 16u : 0u;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_s), "l"(src), "r"(bytes) : "memory");
         }
+        asm volatile("cp.async.commit_group;" ::: "memory");
     };
 
     for (int jc = 0; jc < nb; jc += kSelJChunk) {
@@ -200,11 +201,15 @@ __global__ void __launch_bounds__(256, 1) select_gemm_kernel(const float* __rest
 #pragma unroll
             for (int b = 0; b < 4; ++b) acc[a][b] = make_float2(0.f, 0.f);
         __syncthreads();  // previous chunk's readers are done with ks
-        load_chunk(jc, 0, ks);
+        if (jc == 0) load_chunk(0, 0, ks);  // later chunks' first slice was prefetched below
         for (int cc = 0; cc < D / kSelCChunk; ++cc) {
             float* cur = ks + (cc & 1) * kSelJChunk * kSelKStride;
-            __syncthreads();  // cur is filled; the other buffer is free
-            if (cc + 1 < D / kSelCChunk) load_chunk(jc, cc + 1, ks + ((cc + 1) & 1) * kSelJChunk * kSelKStride);
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+            __syncthreads();  // cur is filled for every thread; the other buffer is free
+            if (cc + 1 < D / kSelCChunk)
+                load_chunk(jc, cc + 1, ks + ((cc + 1) & 1) * kSelJChunk * kSelKStride);
+            else if (jc + kSelJChunk < nb)
+                load_chunk(jc + kSelJChunk, 0, ks + ((cc + 1) & 1) * kSelJChunk * kSelKStride);
 #pragma unroll
             for (int c = 0; c < kSelCChunk; c += 4) {
                 float4 qv[8], kv[4];
