@@ -205,8 +205,7 @@ sbsa_status launch_attn_t(const sbsa_shape* s, const void* q, const void* k, con
     auto kern = attn_kernel<D, BLK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "attention smem attribute");
-    const long long ctas = (p.units + 1) / 2;  // two query tiles per CTA
-    kern<<<static_cast<unsigned>(ctas), C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
+    kern<<<static_cast<unsigned>(p.units), C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
     e = cudaGetLastError();
     return e == cudaSuccess ? SBSA_OK : cuda_fail(e, "attention launch");
 }
