@@ -246,18 +246,19 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
             constexpr uint32_t idS = idesc_bf16_f32(128, BLK, false);
             constexpr uint32_t idO = idesc_bf16_f32(128, D, true);
             const uint32_t ring_addr = smem_u32(sRing);
-            const uint32_t q_addr = smem_u32(sQ);
+            const uint64_t qdesc0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
             int seq = 0;
             auto issue_qk = [&](int j) -> bool {
                 const int slot = seq % NS;
                 if (!wait(&kv_full[slot], (seq / NS) & 1)) return false;
                 tc_fence_after();
-                const uint32_t kaddr = ring_addr + slot * C::kTile;
+                const uint64_t kdesc0 = sdesc_sw128(ring_addr + slot * C::kTile, 16, 1024);
                 const uint32_t d_s = tmem + ((j & 1) ? C::kColS1 : C::kColS0);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t da = sdesc_sw128(q_addr + (kk / 4) * (128 * 128) + (kk % 4) * 32, 16, 1024);
-                    const uint64_t db = sdesc_sw128(kaddr + (kk / 4) * (BLK * 128) + (kk % 4) * 32, 16, 1024);
+                    // only the 14-bit start-address field (bytes / 16) moves between K steps
+                    const uint64_t da = qdesc0 + static_cast<uint64_t>(((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4);
+                    const uint64_t db = kdesc0 + static_cast<uint64_t>(((kk / 4) * (BLK * 128) + (kk % 4) * 32) >> 4);
                     umma_ss(d_s, da, db, idS, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&kv_empty[slot]);
@@ -274,12 +275,12 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
                 if (!(ok = wait(&kv_full[slot], (seq / NS) & 1))) break;
                 if (!(ok = wait(&p_full[j & 1], (j >> 1) & 1))) break;
                 tc_fence_after();
-                const uint32_t vaddr = ring_addr + slot * C::kTile;
+                const uint64_t vdesc0 = sdesc_sw128(ring_addr + slot * C::kTile, BLK * 128, 1024);
                 const uint32_t a_p = tmem + ((j & 1) ? C::kColS1 : C::kColS0);
                 const uint32_t d_o = tmem + ((j & 1) ? C::kColO1 : C::kColO0);
 #pragma unroll
                 for (int kk = 0; kk < BLK / 16; ++kk) {
-                    const uint64_t db = sdesc_sw128(vaddr + kk * 16 * 128, BLK * 128, 1024);
+                    const uint64_t db = vdesc0 + static_cast<uint64_t>((kk * 16 * 128) >> 4);
                     umma_ts(d_o, a_p + kk * 8, db, idO, (j > 1 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(&kv_empty[slot]);
