@@ -68,6 +68,24 @@ def layer_flops(wl: inputs.Workload, k: int) -> float:
     return 4.0 * wl.seq_len_padded * k * wl.block * wl.head_dim * wl.heads * wl.batch
 
 
+def max_over_ranks(pg, device, timings: dict) -> dict:
+    """Each timing (ms) replaced by its maximum over all ranks; one all-reduce for all.
+
+    Every rank calls this with the same keys in the same order.  `pg` is the
+    torch.distributed module (or None for a single process)."""
+    if pg is None:
+        return dict(timings)
+    names = sorted(timings)
+    t = torch.tensor([float(timings[n]) for n in names], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return {n: float(x) for n, x in zip(names, t.tolist())}
+
+
+def job_tflops(flops_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput: every rank's layer counted, divided by the slowest rank's time."""
+    return flops_per_rank * world / (ms / 1e3) / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -340,22 +358,14 @@ def run_gpu(args, wl):
         e2e_ms = e0.elapsed_time(e1) / n_e2e
         e2e = {"ms": e2e_ms, "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2}
 
-    def max_over_ranks(x: float) -> float:
-        if pg is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
-
-    elapsed_ms = max_over_ranks(elapsed_ms)
-    att_avg = max_over_ranks(statistics.mean(att_ms))
-    pool_avg = max_over_ranks(statistics.mean(pool_ms))
-    sel_avg = max_over_ranks(statistics.mean(sel_ms))
-    forward_ms = max_over_ranks(forward_ms)
+    t = max_over_ranks(pg, dev, {"elapsed": elapsed_ms, "att": statistics.mean(att_ms),
+                                 "pool": statistics.mean(pool_ms), "sel": statistics.mean(sel_ms),
+                                 "forward": forward_ms, "e2e": e2e["ms"] if e2e is not None else 0.0})
+    elapsed_ms, att_avg, pool_avg, sel_avg, forward_ms = (t[n] for n in ("elapsed", "att", "pool", "sel", "forward"))
     if e2e is not None:
-        e2e["ms"] = max_over_ranks(e2e["ms"])
+        e2e["ms"] = t["e2e"]
     ms_step = elapsed_ms / args.steps
-    value = flops * ws_n / (ms_step / 1e3) / 1e12
+    value = job_tflops(flops, ws_n, ms_step)
 
     if rank == 0:
         peaks, peak_src = load_peaks()
@@ -388,7 +398,7 @@ def run_gpu(args, wl):
             "peaks": {"source": peak_src, **peaks},
         }
         if e2e is not None:
-            line["e2e"] = {"value": flops * ws_n / (e2e["ms"] / 1e3) / 1e12, "unit": "TFLOP/s",
+            line["e2e"] = {"value": job_tflops(flops, ws_n, e2e["ms"]), "unit": "TFLOP/s",
                            "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
                            "d2h_bytes_per_step": e2e["d2h_bytes_per_step"], "ms_per_step": e2e["ms"]}
         if ws_n == 1 and not args.no_cpu_baseline:
