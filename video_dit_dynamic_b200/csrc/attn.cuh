@@ -5,28 +5,35 @@
 // contribute nothing and the softmax is normalised over the kept keys only.
 //
 // One CTA per (b, h, query block): a 128-row query tile against its k kept key blocks.
-// 320 threads (ten warps):
+// 352 threads (eleven warps):
 //   warps 0-3 / 4-7 (softmax, two warpgroups): warpgroup g handles the kept blocks
-//       j = g, g+2, g+4, ...  Thread r owns query row r: it reads its row of
-//       S_j = Q K_j^T from TMEM, keeps its own running max m_g and sum l_g (log2
-//       domain), rescales its row of its own accumulator O_g in TMEM when m_g moves,
-//       and writes P_j = exp2(S_j*scale*log2e - m_g) as bf16 over the first BLK/2
-//       columns of S_j (P aliases S).  The two warpgroups never wait on each other per
-//       block; at the end each row merges (m_0, l_0, O_0) and (m_1, l_1, O_1) exactly:
+//       j = g, g+2, g+4, ...  Thread r owns query row r.  It copies its row of
+//       S_j = Q K_j^T out of TMEM and at once hands the S buffer back, keeps its own
+//       running max m_g and sum l_g (log2 domain), rescales its row of its own
+//       accumulator O_g in TMEM when m_g moves, and writes P_j = exp2(S_j*scale*log2e - m_g)
+//       as bf16 into the warpgroup's shared-memory P buffer (the layout a K-major
+//       tcgen05 operand with 128-byte swizzle reads).  The two warpgroups never wait on
+//       each other per block; at the end each row merges (m_0, l_0, O_0) and
+//       (m_1, l_1, O_1) exactly:
 //       O = (2^(m_0-M) O_0 + 2^(m_1-M) O_1) / (2^(m_0-M) l_0 + 2^(m_1-M) l_1), M = max.
-//   warp 8 streams Q and the K_j / V_j tiles with TMA (128-byte swizzle) through a ring
-//       of shared-memory slots.
-//   warp 9 allocates 512 TMEM columns and one of its threads issues tcgen05.mma:
-//       S_j = Q K_j^T (both operands in shared memory) into S buffer j&1, and
-//       O_{j&1} += P_j V_j (P from TMEM, V an MN-major shared-memory operand).
-// Tensor-core order: QK_0, QK_1, PV_0, QK_2, PV_1, QK_3, ... so S_{j+1} is computed
-// while a warpgroup works on S_j.  MMAs execute in issue order: QK_{j+2} may reuse S
-// buffer j&1 (and the aliased P_j) once PV_j is issued, and the commit that signals
-// S_{j+2} also proves PV_j done, so O_{j&1} is stable when its warpgroup rescales it.
-// The producer loads K_0, K_1, V_0, K_2, V_1, ... - the same order - over one ring.
+//   warp 8 streams Q and the K_j / V_j tiles with TMA (128-byte swizzle) into a K ring
+//       and a V ring of shared-memory slots.
+//   warp 9 allocates 512 TMEM columns; one of its threads issues every S_j = Q K_j^T
+//       (both operands in shared memory) into S buffer j&1.
+//   warp 10: one thread issues every O_{j&1} += P_j V_j (P and V in shared memory,
+//       V an MN-major operand).
+// Two issuing threads, each with a single MMA instruction site: a wait in one of them
+// (for a K tile, a free S buffer, a P block) leaves the other's MMAs to keep the
+// tensor pipe busy, where one thread alternating between the two kinds drains the
+// MMA queue at every switch and every wait.  Since the two threads' MMAs are not
+// ordered with respect to each other, every hand-over is an mbarrier:
+//   s_full[b]  QK_j done (commit)          -> softmax warpgroup b may read S_j
+//   s_free[b]  S_j copied to registers      -> QK_{j+2} may overwrite S buffer b
+//   p_full[b]  P_j stored (and O_b rescaled) -> PV_j may run
+//   pv_done[b] PV_j done (commit)          -> P buffer b is free and O_b is stable
 //
-// TMEM columns: S buffers at 0 and 128 (BLK fp32 columns each, P in the first BLK/2),
-// O_0 at 256 and O_1 at 384 (D columns each).  For BLK = 64 the 128-row Q tile also holds the next block's
+// TMEM columns: S buffers at 0 and 128 (BLK fp32 columns each), O_0 at 256 and O_1 at
+// 384 (D columns each).  For BLK = 64 the 128-row Q tile also holds the next block's
 // 64 rows; those rows are computed and discarded.
 //
 // Every wait is bounded (kWaitLimitNs); a wait that runs out latches SBSA_ERR_TIMEOUT,
@@ -88,24 +95,25 @@ template <int D, int BLK>
 struct AttnCfg {
     static constexpr int kTile = BLK * D * 2;        // bytes of one K or V tile
     static constexpr int kQBytes = 128 * D * 2;      // bytes of the Q tile
-    static constexpr int kSmemBudget = 216 * 1024;   // Q tile + ring
-    static constexpr int kStagesRaw = (kSmemBudget - kQBytes) / kTile;
-    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-    static constexpr int kRingOff = kQBytes;
-    static constexpr int kBarOff = kRingOff + kStages * kTile;
-    // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_ready[2], drain
-    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;
-    // after the barriers: tmem slot + abort flag (16 B), then the per-row (m, l) of
-    // each warpgroup for the final merge: [2][2][128] floats
-    static constexpr int kXchgOff = kBarOff + kNumBars * 8 + 16;
-    static constexpr int kXchgBytes = 2 * 2 * 128 * 4;
-    static constexpr int kSmemBytes = kXchgOff + kXchgBytes + 1024;  // + alignment slack
-    static constexpr int kThreads = 320;
-    static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
-    static_assert(kStages >= 2, "need at least two ring slots");
+    static constexpr int kPBytes = 128 * BLK * 2;    // bytes of one P block (bf16)
+    static constexpr int kSmemBudget = 224 * 1024;   // Q + two P buffers + the K and V rings
+    static constexpr int kStagesRaw = (kSmemBudget - kQBytes - 2 * kPBytes) / (2 * kTile);
+    static constexpr int kStages = kStagesRaw > 4 ? 4 : kStagesRaw;  // slots per ring
+    static constexpr int kPOff = kQBytes;
+    static constexpr int kKOff = kPOff + 2 * kPBytes;
+    static constexpr int kVOff = kKOff + kStages * kTile;
+    static constexpr int kBarOff = kVOff + kStages * kTile;
+    // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2],
+    // s_free[2], p_full[2], pv_done[2], drain[2]
+    static constexpr int kNumBars = 1 + 4 * kStages + 2 * 5;
+    static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // + tmem slot, flag, alignment slack
+    static constexpr int kThreads = 352;
+    static constexpr uint32_t kColS0 = 0, kColO0 = 256;  // S_b at b*128, O_g at 256 + g*128
+    static_assert(kStages >= 2, "need at least two slots per ring");
     static_assert(D == 64 || D == 128, "head_dim");
     static_assert(BLK == 64 || BLK == 128, "block_size");
     static_assert(kSmemBytes <= 232448, "shared memory");
+    static_assert(2 * 2 * 128 * 4 <= kPBytes, "merge exchange fits in a P buffer");
 };
 
 struct AttnParams {
@@ -125,7 +133,7 @@ __device__ __forceinline__ void softmax_pair_sync() {
 }
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CUtensorMap map_q,
+__global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CUtensorMap map_q,
                                                       const __grid_constant__ CUtensorMap map_k,
                                                       const __grid_constant__ CUtensorMap map_v,
                                                       const AttnParams p) {
@@ -135,18 +143,22 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
     extern __shared__ __align__(1024) uint8_t attn_smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(attn_smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;
-    uint8_t* sRing = smem + C::kRingOff;
+    uint8_t* sP = smem + C::kPOff;   // P_b at sP + b * kPBytes
+    uint8_t* sK = smem + C::kKOff;
+    uint8_t* sV = smem + C::kVOff;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
     uint64_t* q_full = bars;
-    uint64_t* kv_full = bars + 1;
-    uint64_t* kv_empty = kv_full + NS;
-    uint64_t* s_full = kv_empty + NS;
-    uint64_t* p_full = s_full + 2;
-    uint64_t* o_ready = p_full + 2;
-    uint64_t* drain = o_ready + 2;
+    uint64_t* k_full = bars + 1;
+    uint64_t* k_empty = k_full + NS;
+    uint64_t* v_full = k_empty + NS;
+    uint64_t* v_empty = v_full + NS;
+    uint64_t* s_full = v_empty + NS;
+    uint64_t* s_free = s_full + 2;
+    uint64_t* p_full = s_free + 2;
+    uint64_t* pv_done = p_full + 2;
+    uint64_t* drain = pv_done + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    float* xml = reinterpret_cast<float*>(smem + C::kXchgOff);  // [g][m, l][128]
 
     const int tid = threadIdx.x;
     const int warp = tid / 32;
@@ -164,13 +176,19 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
     if (tid == 256) {
         *abort_flag = 0;
         mbar_init(q_full, 1);
-        for (int s = 0; s < NS; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
+            mbar_init(&s_free[b], 128);
             mbar_init(&p_full[b], 128);
-            mbar_init(&o_ready[b], 1);
+            mbar_init(&pv_done[b], 1);
+            mbar_init(&drain[b], 1);
         }
-        mbar_init(drain, 1);
         fence_mbar_init();
         tma_prefetch_desc(&map_q);
         tma_prefetch_desc(&map_k);
@@ -195,12 +213,11 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
         if (!*abort_flag) give_up();
         return false;
     };
-    // ring position of the tiles, in the shared load / MMA order
-    //   K_0 -> 0, K_1 -> 1, and for j >= 0: V_j -> 2 + 2j, K_{j+2} -> 3 + 2j
-    // (when n == 1: K_0 -> 0, V_0 -> 1)
 
     if (warp == 8) {
         // ------------------------------------------------------------ TMA producer
+        // Order of need: K_0, K_1, then K_{j+2} (wanted as soon as S_j is copied out)
+        // before V_j (wanted when P_j is ready).
         if ((tid & 31) == 0 && n > 0) {
             const uint64_t pol_q = policy_evict_first();
             const uint64_t pol_kv = policy_evict_last();
@@ -209,51 +226,54 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
 #pragma unroll
             for (int a = 0; a < D / 64; ++a)
                 tma_load_2d(sQ + a * 128 * 128, &map_q, q_full, a * 64, row0 + qb * BLK, pol_q);
-            int seq = 0;
-            bool ok = true;
+            int kseq = 0, vseq = 0;
             auto load = [&](int j, bool is_v) -> bool {
+                int& seq = is_v ? vseq : kseq;
                 const int slot = seq % NS;
                 const uint32_t ph = (seq / NS) & 1;
-                if (!wait(&kv_empty[slot], ph ^ 1)) return false;
+                if (!wait(is_v ? &v_empty[slot] : &k_empty[slot], ph ^ 1)) return false;
                 int blk = __ldg(p.col_idx + rs + j);
                 if (blk < 0 || blk >= p.nb) blk = 0;  // masked by the softmax warps
-                uint8_t* dst = sRing + slot * C::kTile;
-                mbar_arrive_expect_tx(&kv_full[slot], C::kTile);
+                uint8_t* dst = (is_v ? sV : sK) + slot * C::kTile;
+                uint64_t* full = is_v ? &v_full[slot] : &k_full[slot];
+                mbar_arrive_expect_tx(full, C::kTile);
 #pragma unroll
                 for (int a = 0; a < D / 64; ++a)
-                    tma_load_2d(dst + a * BLK * 128, is_v ? &map_v : &map_k, &kv_full[slot], a * 64,
-                                row0 + blk * BLK, pol_kv);
+                    tma_load_2d(dst + a * BLK * 128, is_v ? &map_v : &map_k, full, a * 64, row0 + blk * BLK, pol_kv);
                 ++seq;
                 return true;
             };
-            ok = load(0, false);
+            bool ok = load(0, false);
             if (ok && n > 1) ok = load(1, false);
             for (int j = 0; ok && j < n; ++j) {
-                ok = load(j, true);
-                if (ok && j + 2 < n) ok = load(j + 2, false);
+                if (j + 2 < n) ok = load(j + 2, false);
+                if (ok) ok = load(j, true);
             }
             if (!ok) {
                 // drain: every issued copy must land before the CTA exits
                 volatile int never = 0;
                 mbar_wait_bounded(q_full, 0, &never, kWaitLimitNs);
-                for (int q = seq - NS < 0 ? 0 : seq - NS; q < seq; ++q)
-                    mbar_wait_bounded(&kv_full[q % NS], (q / NS) & 1, &never, kWaitLimitNs);
+                for (int q = kseq - NS < 0 ? 0 : kseq - NS; q < kseq; ++q)
+                    mbar_wait_bounded(&k_full[q % NS], (q / NS) & 1, &never, kWaitLimitNs);
+                for (int q = vseq - NS < 0 ? 0 : vseq - NS; q < vseq; ++q)
+                    mbar_wait_bounded(&v_full[q % NS], (q / NS) & 1, &never, kWaitLimitNs);
             }
         }
     } else if (warp == 9) {
-        // ------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------------ QK issuer
         if ((tid & 31) == 0 && n > 0) {
             constexpr uint32_t idS = idesc_bf16_f32(128, BLK, false);
-            constexpr uint32_t idO = idesc_bf16_f32(128, D, true);
-            const uint32_t ring_addr = smem_u32(sRing);
+            const uint32_t k_addr = smem_u32(sK);
             const uint64_t qdesc0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
-            int seq = 0;
-            auto issue_qk = [&](int j) -> bool {
-                const int slot = seq % NS;
-                if (!wait(&kv_full[slot], (seq / NS) & 1)) return false;
+            bool ok = wait(q_full, 0);
+            for (int j = 0; ok && j < n; ++j) {
+                const int slot = j % NS;
+                const int b = j & 1;
+                if (!(ok = wait(&k_full[slot], (j / NS) & 1))) break;
+                if (j >= 2 && !(ok = wait(&s_free[b], ((j - 2) >> 1) & 1))) break;
                 tc_fence_after();
-                const uint64_t kdesc0 = sdesc_sw128(ring_addr + slot * C::kTile, 16, 1024);
-                const uint32_t d_s = tmem + ((j & 1) ? C::kColS1 : C::kColS0);
+                const uint64_t kdesc0 = sdesc_sw128(k_addr + slot * C::kTile, 16, 1024);
+                const uint32_t d_s = tmem + C::kColS0 + b * 128;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     // only the 14-bit start-address field (bytes / 16) moves between K steps
@@ -261,37 +281,44 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
                     const uint64_t db = kdesc0 + static_cast<uint64_t>(((kk / 4) * (BLK * 128) + (kk % 4) * 32) >> 4);
                     umma_ss(d_s, da, db, idS, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&kv_empty[slot]);
-                umma_commit(&s_full[j & 1]);
-                ++seq;
-                return true;
-            };
-            bool ok = wait(q_full, 0) && issue_qk(0);
-            if (ok && n > 1) ok = issue_qk(1);
-            for (int j = 0; ok && j < n; ++j) {
-                // V_j first (normally loaded long ago; this wait overlaps QK_{j+1} on the
-                // tensor core), then the real dependency: P_j from the softmax warps
-                const int slot = seq % NS;
-                if (!(ok = wait(&kv_full[slot], (seq / NS) & 1))) break;
-                if (!(ok = wait(&p_full[j & 1], (j >> 1) & 1))) break;
-                tc_fence_after();
-                const uint64_t vdesc0 = sdesc_sw128(ring_addr + slot * C::kTile, BLK * 128, 1024);
-                const uint32_t a_p = tmem + ((j & 1) ? C::kColS1 : C::kColS0);
-                const uint32_t d_o = tmem + ((j & 1) ? C::kColO1 : C::kColO0);
-#pragma unroll
-                for (int kk = 0; kk < BLK / 16; ++kk) {
-                    const uint64_t db = vdesc0 + static_cast<uint64_t>((kk * 16 * 128) >> 4);
-                    umma_ts(d_o, a_p + kk * 8, db, idO, (j > 1 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(&kv_empty[slot]);
-                if (j + 2 >= n) umma_commit(&o_ready[j & 1]);  // last PV into O_{j&1}
-                ++seq;
-                if (j + 2 < n) ok = issue_qk(j + 2);
+                umma_commit(&k_empty[slot]);
+                umma_commit(&s_full[b]);
             }
             if (!ok) {
-                umma_commit(drain);  // wait for every MMA already issued
+                umma_commit(&drain[0]);  // wait for every MMA this thread issued
                 volatile int never = 0;
-                mbar_wait_bounded(drain, 0, &never, kWaitLimitNs);
+                mbar_wait_bounded(&drain[0], 0, &never, kWaitLimitNs);
+            }
+        }
+    } else if (warp == 10) {
+        // ------------------------------------------------------------ PV issuer
+        if ((tid & 31) == 0 && n > 0) {
+            constexpr uint32_t idO = idesc_bf16_f32(128, D, true);
+            const uint32_t v_addr = smem_u32(sV);
+            const uint64_t pdesc0 = sdesc_sw128(smem_u32(sP), 16, 1024);
+            bool ok = true;
+            for (int j = 0; ok && j < n; ++j) {
+                const int slot = j % NS;
+                const int b = j & 1;
+                if (!(ok = wait(&v_full[slot], (j / NS) & 1))) break;
+                if (!(ok = wait(&p_full[b], (j >> 1) & 1))) break;
+                tc_fence_after();
+                const uint64_t vdesc0 = sdesc_sw128(v_addr + slot * C::kTile, BLK * 128, 1024);
+                const uint64_t pdesc = pdesc0 + static_cast<uint64_t>((b * C::kPBytes) >> 4);
+                const uint32_t d_o = tmem + C::kColO0 + b * 128;
+#pragma unroll
+                for (int kk = 0; kk < BLK / 16; ++kk) {
+                    const uint64_t da = pdesc + static_cast<uint64_t>(((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4);
+                    const uint64_t db = vdesc0 + static_cast<uint64_t>((kk * 16 * 128) >> 4);
+                    umma_ss(d_o, da, db, idO, (j > 1 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(&v_empty[slot]);
+                umma_commit(&pv_done[b]);
+            }
+            if (!ok) {
+                umma_commit(&drain[1]);
+                volatile int never = 0;
+                mbar_wait_bounded(&drain[1], 0, &never, kWaitLimitNs);
             }
         }
     } else if (warp < 8) {
@@ -304,8 +331,12 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
         const bool row_valid = row_in_block && t < p.L;
         const float sl2 = p.scale_log2;  // |scale| * log2(e) > 0
         const float2 sl2x2 = make_float2(sl2, sl2);
-        const uint32_t s_col = tmem + lane_base + (g ? C::kColS1 : C::kColS0);
-        const uint32_t o_col = tmem + lane_base + (g ? C::kColO1 : C::kColO0);
+        const uint32_t s_col = tmem + lane_base + C::kColS0 + g * 128;
+        const uint32_t o_col = tmem + lane_base + C::kColO0 + g * 128;
+        // this row of P_g: 128-byte rows, 16-byte chunks swizzled by (row mod 8), one
+        // 16 KB region per 64 keys
+        const uint32_t p_row = smem_u32(sP + g * C::kPBytes) + r * 128;
+        const uint32_t p_swz = static_cast<uint32_t>(r & 7);
         float m = -INFINITY;  // running reference max (log2 domain), possibly stale by < 8
         float l = 0.f;        // this warpgroup's part of the row sum
         bool ok = true;
@@ -333,6 +364,9 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
 #pragma unroll
                 for (int e = 0; e < BLK; ++e) s[e] = __uint_as_float(raw[e]);
             }
+            // S_j is in registers: QK_{j+2} may overwrite the buffer
+            tc_fence_before();
+            mbar_arrive(&s_free[g]);
             if (p.neg_scale) {
 #pragma unroll
                 for (int e = 0; e < BLK; ++e) s[e] = -s[e];
@@ -393,9 +427,16 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
             const float2 s23 = __fadd2_rn(sum4[2], sum4[3]);
             const float2 sall = __fadd2_rn(s01, s23);
             l = l * alpha + (sall.x + sall.y);
-            tmem_st_cols<BLK / 2>(s_col, pk);  // P over the first BLK/2 columns of S
-            // O_g already holds every earlier PV of this warpgroup (the commit that
-            // signalled S_j covers them): rescale it now that P is out of registers
+            // PV_{j-2} must be done before P buffer g is overwritten or O_g rescaled
+            if (j >= 2) {
+                ok = wait_warp(&pv_done[g], ((j - 2) >> 1) & 1);
+                if (!ok) continue;
+            }
+#pragma unroll
+            for (int c = 0; c < BLK / 8; ++c) {
+                const uint32_t addr = p_row + (c / 8) * (128 * 128) + ((static_cast<uint32_t>(c & 7) ^ p_swz) << 4);
+                st_shared_v4(addr, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            }
             if (j > 1 && __any_sync(0xFFFFFFFFu, alpha != 1.f)) {
                 const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
@@ -410,23 +451,43 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
                     }
                     tmem_st_cols<(D < 64 ? D : 64)>(o_col + h, ov);
                 }
+                tmem_st_wait();
             }
-            tmem_st_wait();
+            fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&p_full[g]);
         }
         const bool has_blocks = g < n;
-        if (ok && has_blocks) ok = wait_warp(&o_ready[g], 0);
-        // ---- merge: row r of (m_0, l_0, O_0) and (m_1, l_1, O_1); warpgroup g writes
-        // output columns [g D/2, (g+1) D/2)
-        xml[(g * 2 + 0) * 128 + r] = has_blocks ? m : -INFINITY;
-        xml[(g * 2 + 1) * 128 + r] = has_blocks ? l : 0.f;
+        if (ok && has_blocks) {
+            const int j_last = g + ((n - 1 - g) & ~1);  // this warpgroup's last block
+            ok = wait_warp(&pv_done[g], (j_last >> 1) & 1);
+        }
         ok = __all_sync(0xFFFFFFFFu, ok);
+        // ---- merge: row r of (m_0, l_0, O_0) and (m_1, l_1, O_1); warpgroup g writes
+        // output columns [g D/2, (g+1) D/2).  The exchange goes through P buffer g,
+        // which no MMA reads any more once this warpgroup's last PV is done; after a
+        // failed wait it may still be read, so then nothing is exchanged.
+        float* xml_mine = reinterpret_cast<float*>(sP + g * C::kPBytes);
+        const float* xml_other = reinterpret_cast<const float*>(sP + (g ^ 1) * C::kPBytes);
+        if (ok) {
+            xml_mine[r] = has_blocks ? m : -INFINITY;
+            xml_mine[128 + r] = has_blocks ? l : 0.f;
+        }
         tc_fence_before();
         softmax_pair_sync();
         tc_fence_after();
-        const float m0 = xml[0 * 128 + r], l0 = xml[1 * 128 + r];
-        const float m1 = xml[2 * 128 + r], l1 = xml[3 * 128 + r];
+        // a failed wait anywhere in the pair is seen by both warpgroups: the flag is
+        // latched before the barrier
+        const bool pair_ok = ok && !*abort_flag;
+        float mg = -INFINITY, lg = 0.f, mo = -INFINITY, lo = 0.f;
+        if (pair_ok) {
+            mg = xml_mine[r];
+            lg = xml_mine[128 + r];
+            mo = xml_other[r];
+            lo = xml_other[128 + r];
+        }
+        const float m0 = g == 0 ? mg : mo, l0 = g == 0 ? lg : lo;
+        const float m1 = g == 0 ? mo : mg, l1 = g == 0 ? lo : lg;
         const float M = fmaxf(m0, m1);
         const float w0 = (m0 == -INFINITY) ? 0.f : ex2_approx(m0 - M);
         const float w1 = (m1 == -INFINITY) ? 0.f : ex2_approx(m1 - M);
@@ -435,14 +496,15 @@ __global__ void __launch_bounds__(320, 1) attn_kernel(const __grid_constant__ CU
         {
             // every lane of the warp runs the TMEM loads (warp-collective); only rows of
             // this query block are stored
-            const bool write_o = ok && any_pv && row_valid && lt > 0.f;
+            const bool read_o = __all_sync(0xFFFFFFFFu, pair_ok) && any_pv;
+            const bool write_o = read_o && row_valid && lt > 0.f;
             const float inv = write_o ? 1.f / lt : 0.f;
             const float c0 = w0 * inv, c1 = w1 * inv;
             const bool use1 = n > 1;  // O_1 holds data only if warpgroup 1 had a block
             uint32_t o0[HD], o1[HD];
-            if (ok && any_pv) {
+            if (read_o) {
                 tmem_ld_cols<HD>(tmem + lane_base + C::kColO0 + g * HD, o0);
-                if (use1) tmem_ld_cols<HD>(tmem + lane_base + C::kColO1 + g * HD, o1);
+                if (use1) tmem_ld_cols<HD>(tmem + lane_base + C::kColO0 + 128 + g * HD, o1);
             }
             if (row_in_block) {
                 uint4* dst = reinterpret_cast<uint4*>(p.o + (bh * p.Lp + t) * D + g * HD);
