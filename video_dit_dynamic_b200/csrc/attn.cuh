@@ -50,7 +50,7 @@
 // polynomial instead of the MUFU ex2 unit; the two run in parallel, so moving some of
 // the work off the MUFU unit (16 results/clk/SM) shortens the softmax.
 #ifndef SBSA_POLY_EXP2_EIGHTHS
-#define SBSA_POLY_EXP2_EIGHTHS 0
+#define SBSA_POLY_EXP2_EIGHTHS 2
 #endif
 
 namespace sbsa {
