@@ -377,12 +377,14 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                 for (int e = 0; e < BLK; ++e)
                     if (e >= nvalid) s[e] = -INFINITY;
             }
-            // block max: eight independent chains, then a tree
+            // block max: eight independent chains of three-input maxima, then a tree
             float mx8[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) mx8[c] = s[c];
+            for (int c = 0; c < 8; ++c) mx8[c] = fmaxf(s[c], s[c + 8]);
 #pragma unroll
-            for (int e = 8; e < BLK; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], s[e]);
+            for (int e = 16; e < BLK; e += 16)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) mx8[c] = fmax3(mx8[c], s[e + c], s[e + 8 + c]);
             const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                    fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;
             // Lazy rescaling: keep the old reference max unless the block's max exceeds
