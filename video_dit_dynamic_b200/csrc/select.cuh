@@ -46,18 +46,62 @@ __device__ __forceinline__ void select_row_topk(const uint32_t* __restrict__ key
         // pattern maps to 0, and it is clamped to 1)
         key[s] = (j < nb && j != i) ? max(keys_row[j], 1u) : 0u;
     }
+    // The (k-1)-th largest candidate key T: a search over the key range [lo, hi) with
+    // count(key >= lo) >= k-1 > count(key >= hi).  Each probe is placed where the
+    // counts at the two ends put it if the keys were spread evenly in between
+    // (interpolation), with a halving probe after any interpolation that did not at
+    // least halve the range, so the search never takes more than twice the 33 steps
+    // of plain bisection.  It stops early when exactly k-1 keys are >= the probe.
     uint32_t T = 0u;
     if (kk > 0) {
+        uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+        int nc = 0;
+#pragma unroll
+        for (int s = 0; s < KPL; ++s) {
+            if (key[s] != 0u) {
+                kmin = min(kmin, key[s]);
+                ++nc;
+            }
+            kmax = max(kmax, key[s]);
+        }
+        uint32_t lo = __reduce_min_sync(0xFFFFFFFFu, kmin);
+        const uint32_t top = __reduce_max_sync(0xFFFFFFFFu, kmax);
+        int c_lo = __reduce_add_sync(0xFFFFFFFFu, nc);  // candidates: count(key >= lo)
+        int c_hi = 0;
+        // hi = top + 1 as a 64-bit bound: top can be the largest key
+        uint64_t hi = static_cast<uint64_t>(top) + 1u;
+        bool halve = false;
+        T = lo;
 #pragma unroll 1
-        for (int bit = 31; bit >= 0; --bit) {
-            const uint32_t cand = T | (1u << bit);
+        for (int it = 0; it < 72 && hi - lo > 1u; ++it) {
+            const uint64_t range = hi - lo;
+            uint64_t off;
+            if (halve) {
+                off = range >> 1;
+            } else {
+                const float f = static_cast<float>(c_lo - kk) / static_cast<float>(c_lo - c_hi);
+                off = static_cast<uint64_t>(f * static_cast<float>(range));
+            }
+            off = off < 1u ? 1u : (off > range - 1u ? range - 1u : off);
+            const uint32_t cand = static_cast<uint32_t>(lo + off);
             // four independent partial counts keep the add chains short
             int c4[4] = {0, 0, 0, 0};
 #pragma unroll
             for (int s = 0; s < KPL; ++s) c4[s & 3] += key[s] >= cand ? 1 : 0;
             const int cnt = __reduce_add_sync(0xFFFFFFFFu, (c4[0] + c4[1]) + (c4[2] + c4[3]));
-            if (cnt >= kk) T = cand;
-            if (cnt == kk) break;  // {key >= cand} is exactly the top k-1
+            if (cnt == kk) {  // {key >= cand} is exactly the top k-1
+                T = cand;
+                break;
+            }
+            if (cnt > kk) {
+                lo = cand;
+                c_lo = cnt;
+            } else {
+                hi = cand;
+                c_hi = cnt;
+            }
+            T = lo;
+            halve = !halve && 2u * (hi - lo) > range;
         }
     }
     int n_gt = 0;
