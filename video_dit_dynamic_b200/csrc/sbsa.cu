@@ -108,6 +108,21 @@ sbsa_status make_map(CUtensorMap* m, const void* base, long long rows, int d, in
     return SBSA_OK;
 }
 
+// fp32 block means [rows][128] viewed as a 2D tensor, box = 32 channels (128 B) x box_rows
+sbsa_status make_map_means(CUtensorMap* m, const float* base, long long rows, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(SBSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {128 * 4};
+    cuuint32_t box[2] = {32, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SBSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return SBSA_OK;
+}
+
 std::atomic<unsigned int> g_epoch{1};
 
 // ---------------------------------------------------------------- launchers
@@ -157,16 +172,38 @@ sbsa_status launch_select_gemm(const sbsa_shape* s, const float* qm, const float
     return e == cudaSuccess ? SBSA_OK : cuda_fail(e, "select launch");
 }
 
+template <int KPL>
+sbsa_status launch_select_tc(const sbsa_shape* s, const float* qm, const float* km, int k, int32_t* rp, int32_t* ci,
+                             cudaStream_t st) {
+    const int nb = num_blocks(s);
+    CUtensorMap mq, mk;
+    sbsa_status r;
+    if ((r = make_map_means(&mq, qm, num_rows(s), kSelTcRows)) != SBSA_OK) return r;
+    if ((r = make_map_means(&mk, km, num_rows(s), 128)) != SBSA_OK) return r;
+    SelTcParams p;
+    p.nb = nb;
+    p.k_keep = k;
+    p.n_rows = num_rows(s);
+    p.epoch = g_epoch.fetch_add(1);
+    auto kern = select_tc_kernel<KPL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSelTcSmemBytes));
+    if (e != cudaSuccess) return cuda_fail(e, "select smem attribute");
+    const dim3 grid((nb + kSelTcRows - 1) / kSelTcRows, static_cast<unsigned>(s->batch * s->heads));
+    kern<<<grid, kSelTcThreads, kSelTcSmemBytes, st>>>(mq, mk, rp, ci, p);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? SBSA_OK : cuda_fail(e, "select launch");
+}
+
 template <int D>
 sbsa_status launch_select_d(const sbsa_shape* s, const float* qm, const float* km, int k, int32_t* rp, int32_t* ci,
                             cudaStream_t st) {
     const int nb = num_blocks(s);
     if constexpr (D == 128) {
-        // register-blocked GEMM path (head_dim 128, up to 1024 blocks)
-        if (nb <= 64) return launch_select_gemm<2>(s, qm, km, k, rp, ci, st);
-        if (nb <= 256) return launch_select_gemm<8>(s, qm, km, k, rp, ci, st);
-        if (nb <= 512) return launch_select_gemm<16>(s, qm, km, k, rp, ci, st);
-        if (nb <= 1024) return launch_select_gemm<32>(s, qm, km, k, rp, ci, st);
+        // tensor-core scores (head_dim 128, up to 1024 blocks)
+        if (nb <= 64) return launch_select_tc<2>(s, qm, km, k, rp, ci, st);
+        if (nb <= 256) return launch_select_tc<8>(s, qm, km, k, rp, ci, st);
+        if (nb <= 512) return launch_select_tc<16>(s, qm, km, k, rp, ci, st);
+        if (nb <= 1024) return launch_select_tc<32>(s, qm, km, k, rp, ci, st);
     }
     if (nb <= 64) return launch_select_t<D, 2>(s, qm, km, k, rp, ci, st);
     if (nb <= 256) return launch_select_t<D, 8>(s, qm, km, k, rp, ci, st);

@@ -17,6 +17,7 @@
 //            which yields the ascending order directly.
 #pragma once
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace sbsa {
 
@@ -290,6 +291,235 @@ __global__ void __launch_bounds__(256, 1) select_gemm_kernel(const float* __rest
 constexpr size_t select_gemm_smem_bytes(int KPL) {
     return (static_cast<size_t>(kSelQT) * kSelQStride + 2ull * kSelJChunk * kSelKStride) * 4 +
            static_cast<size_t>(kSelQT) * 32 * KPL * 4;
+}
+
+// ---------------------------------------------------------------- tensor-core scores
+// Scores of 32 query blocks against all key blocks of one (b, h) on the tensor cores, in
+// the transposed form S^T = Kmean . Qmean^T: M = 128 key blocks per tile (TMEM lane =
+// key block, column = query block), N = 32 query blocks, K = d = 128, kind::tf32.
+// fp32 accuracy from three products per K step: each mean x is split exactly into
+// x_t = x with its 13 low mantissa bits cleared (what the tensor core reads from a raw
+// fp32 operand: it truncates) and x_l = x - x_t; s = k_t.q_t + k_t.q_l + k_l.q_t drops
+// only k_l.q_l and the truncation of the small parts, about 2^-19 of |k||q| per product,
+// below the fp32 rounding of a 128-term sum.
+//
+// CTA = (b*h, 32 query blocks), 320 threads, two CTAs per SM:
+//   warp 8  : TMA of the raw means (box 32 channels x rows, 128-byte swizzle: the
+//             K-major operand layout): the Q tile once, then K chunks (128 key blocks x
+//             32 channels) through a two-slot ring.
+//   warp 9  : TMEM allocation (256 columns: 8 key tiles x 32 query blocks) and the thread
+//             that issues the MMAs, 12 per chunk ((k_t,q_t), (k_t,q_l), (k_l,q_t) at 4 K
+//             steps).
+//   warps 0-7: write q_l once and k_l of every chunk (two buffers); then read the scores
+//             out of TMEM into shared memory as order-preserving keys, 16 query rows at a
+//             time, and run the warp-per-row top-k.
+constexpr int kSelTcRows = 32;                  // query blocks per CTA
+constexpr int kSelTcThreads = 320;
+constexpr int kSelTcTile = 128 * 128;           // bytes of one K chunk (128 rows x 32 fp32)
+constexpr int kSelTcQBytes = 4 * 32 * 128;      // Q tile: 4 channel chunks x 32 rows x 128 B
+constexpr int kSelTcOffQ = 0, kSelTcOffQl = kSelTcQBytes, kSelTcOffX = 2 * kSelTcQBytes;
+constexpr int kSelTcOffXl = kSelTcOffX + 2 * kSelTcTile;
+constexpr int kSelTcOffBar = kSelTcOffXl + 2 * kSelTcTile;  // 96 KB of operands
+constexpr int kSelTcNumBars = 2 + 2 + 2 + 2 + 2 + 1;  // q_full, ql_full, x_full[2], x_empty[2], l_full[2], l_empty[2], done
+constexpr size_t kSelTcSmemBytes = kSelTcOffBar + kSelTcNumBars * 8 + 16 + 1024;
+
+constexpr uint32_t idesc_tf32_f32(int M, int N) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+__device__ __forceinline__ void umma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// x - (x with its 13 low mantissa bits cleared), for four floats
+__device__ __forceinline__ float4 tf32_low_part(float4 v) {
+    auto lo = [](float x) { return x - __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); };
+    return make_float4(lo(v.x), lo(v.y), lo(v.z), lo(v.w));
+}
+
+struct SelTcParams {
+    int nb, k_keep;
+    long long n_rows;
+    unsigned int epoch;
+};
+
+template <int KPL>
+__global__ void __launch_bounds__(kSelTcThreads, 2) select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
+                                                                    const __grid_constant__ CUtensorMap map_k,
+                                                                    int32_t* __restrict__ row_ptr,
+                                                                    int32_t* __restrict__ col_idx,
+                                                                    const SelTcParams p) {
+    constexpr int NBP = 32 * KPL;                 // key slots per row (>= nb)
+    constexpr int HALF = kSelTcRows / 2;          // query rows per top-k round
+    static_assert(HALF * NBP * 4 <= kSelTcOffBar, "keys of one round fit over the operand buffers");
+    extern __shared__ __align__(1024) uint8_t sel_tc_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sel_tc_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSelTcOffBar);
+    uint64_t* q_full = bars;
+    uint64_t* ql_full = bars + 1;
+    uint64_t* x_full = bars + 2;
+    uint64_t* x_empty = bars + 4;
+    uint64_t* l_full = bars + 6;
+    uint64_t* l_empty = bars + 8;
+    uint64_t* done = bars + 10;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kSelTcNumBars);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem);  // [HALF][NBP], after the MMAs
+
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    if (launch_aborted(p.epoch)) return;
+    const int nb = p.nb;
+    const long long bh = blockIdx.y;
+    const int i0 = blockIdx.x * kSelTcRows;
+    const int nq = min(kSelTcRows, nb - i0);
+    const int n_tiles = (nb + 127) / 128;
+    const int n_chunks = 4 * n_tiles;
+
+    if (tid == 256) {
+        *abort_flag = 0;
+        // ql_full and l_full[] count the 256 threads that write low parts; the rest one arrival
+        for (int b = 0; b < kSelTcNumBars; ++b)
+            mbar_init(&bars[b], (&bars[b] == ql_full || &bars[b] == &l_full[0] || &bars[b] == &l_full[1]) ? 256u : 1u);
+        fence_mbar_init();
+        tma_prefetch_desc(&map_q);
+        tma_prefetch_desc(&map_k);
+    }
+    if (warp == 9) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+        if (mbar_wait_bounded(bar, parity, abort_flag, kWaitLimitNs)) return true;
+        if (!*abort_flag) {
+            *abort_flag = 1;
+            abort_launch(p.epoch);
+        }
+        return false;
+    };
+    bool ok = true;
+
+    if (warp == 8) {
+        // ---------------------------------------------------------------- TMA
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_last();
+            const int row_q = static_cast<int>(bh * nb + i0), row_k = static_cast<int>(bh * nb);
+            mbar_arrive_expect_tx(q_full, kSelTcQBytes);
+#pragma unroll
+            for (int a = 0; a < 4; ++a) tma_load_2d(smem + kSelTcOffQ + a * 32 * 128, &map_q, q_full, 32 * a, row_q, pol);
+            int c = 0;
+            for (; c < n_chunks; ++c) {
+                const int b = c & 1;
+                if (c >= 2 && !(ok = wait(&x_empty[b], ((c - 2) >> 1) & 1))) break;
+                mbar_arrive_expect_tx(&x_full[b], kSelTcTile);
+                tma_load_2d(smem + kSelTcOffX + b * kSelTcTile, &map_k, &x_full[b], 32 * (c & 3), row_k + 128 * (c >> 2), pol);
+            }
+            if (!ok) {
+                volatile int never = 0;
+                mbar_wait_bounded(q_full, 0, &never, kWaitLimitNs);
+                for (int q = c - 2 < 0 ? 0 : c - 2; q < c; ++q) mbar_wait_bounded(&x_full[q & 1], (q >> 1) & 1, &never, kWaitLimitNs);
+            }
+        }
+    } else if (warp == 9) {
+        // ---------------------------------------------------------------- MMA
+        if (lane == 0) {
+            constexpr uint32_t id = idesc_tf32_f32(128, kSelTcRows);
+            const uint32_t q_addr = smem_u32(smem + kSelTcOffQ), ql_addr = smem_u32(smem + kSelTcOffQl);
+            const uint32_t x_addr = smem_u32(smem + kSelTcOffX), xl_addr = smem_u32(smem + kSelTcOffXl);
+            ok = wait(q_full, 0) && wait(ql_full, 0);
+            for (int c = 0; ok && c < n_chunks; ++c) {
+                const int b = c & 1, t = c >> 2, dc = c & 3;
+                if (!(ok = wait(&x_full[b], (c >> 1) & 1))) break;
+                if (!(ok = wait(&l_full[b], (c >> 1) & 1))) break;
+                tc_fence_after();
+                const uint32_t d = tmem + t * kSelTcRows;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t xa = sdesc_sw128(x_addr + b * kSelTcTile + ks * 32, 16, 1024);
+                    const uint64_t la = sdesc_sw128(xl_addr + b * kSelTcTile + ks * 32, 16, 1024);
+                    const uint64_t qb = sdesc_sw128(q_addr + dc * 32 * 128 + ks * 32, 16, 1024);
+                    const uint64_t lb = sdesc_sw128(ql_addr + dc * 32 * 128 + ks * 32, 16, 1024);
+                    umma_tf32_ss(d, xa, qb, id, (dc > 0 || ks > 0) ? 1u : 0u);
+                    umma_tf32_ss(d, xa, lb, id, 1u);
+                    umma_tf32_ss(d, la, qb, id, 1u);
+                }
+                umma_commit(&x_empty[b]);
+                umma_commit(&l_empty[b]);
+            }
+            umma_commit(done);  // every MMA this thread issued (also on the error path)
+            if (!ok) {
+                volatile int never = 0;
+                mbar_wait_bounded(done, 0, &never, kWaitLimitNs);
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- low parts
+        if ((ok = wait(q_full, 0))) {
+#pragma unroll
+            for (int u = 0; u < kSelTcQBytes / 16 / 256; ++u) {
+                const int f = tid + 256 * u;
+                const float4 v = reinterpret_cast<const float4*>(smem + kSelTcOffQ)[f];
+                reinterpret_cast<float4*>(smem + kSelTcOffQl)[f] = tf32_low_part(v);
+            }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(ql_full);
+        for (int c = 0; ok && c < n_chunks; ++c) {
+            const int b = c & 1;
+            if (!(ok = wait(&x_full[b], (c >> 1) & 1))) break;
+            float4 v[kSelTcTile / 16 / 256];
+#pragma unroll
+            for (int u = 0; u < kSelTcTile / 16 / 256; ++u)
+                v[u] = tf32_low_part(reinterpret_cast<const float4*>(smem + kSelTcOffX + b * kSelTcTile)[tid + 256 * u]);
+            if (c >= 2 && !(ok = wait(&l_empty[b], ((c - 2) >> 1) & 1))) break;
+#pragma unroll
+            for (int u = 0; u < kSelTcTile / 16 / 256; ++u)
+                reinterpret_cast<float4*>(smem + kSelTcOffXl + b * kSelTcTile)[tid + 256 * u] = v[u];
+            fence_proxy_async_smem();
+            mbar_arrive(&l_full[b]);
+        }
+    }
+    // ---------------------------------------------------------------- top-k
+    // every MMA is done once `done` completes; the operand buffers then hold keys
+    if (warp < 8 && ok) ok = wait(done, 0);
+    ok = __syncthreads_and(ok ? 1 : 0) != 0;
+    tc_fence_after();
+    if (ok && warp < 8) {
+        const int q4 = warp & 3;  // TMEM lane quarter of this warp
+        for (int round = 0; round < 2; ++round) {
+            const int r0 = round * HALF;
+            if (r0 < nq) {
+                // scores of key blocks 128 t + 32 q4 + lane for query rows r0 .. r0+15
+                for (int t = warp >> 2; t < n_tiles; t += 2) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem + (static_cast<uint32_t>(32 * q4) << 16) + t * kSelTcRows + r0, v);
+                    const int j = 128 * t + 32 * q4 + lane;
+                    if (j < NBP) {
+#pragma unroll
+                        for (int c = 0; c < HALF; ++c) keys[c * NBP + j] = order_key(__uint_as_float(v[c]));
+                    }
+                }
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            for (int r = r0 + warp; r < min(nq, r0 + HALF); r += 8)
+                select_row_topk<KPL>(keys + (r - r0) * NBP, nb, i0 + r, p.k_keep, bh * nb + i0 + r, row_ptr, col_idx);
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+        }
+    }
+    if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) row_ptr[p.n_rows] = static_cast<int32_t>(p.n_rows * p.k_keep);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
 }
 
 }  // namespace sbsa
