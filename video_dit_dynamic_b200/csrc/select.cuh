@@ -32,7 +32,7 @@ __device__ __forceinline__ uint32_t order_key(float s) {
 // j = l + 32 s.  The (k-1)-th largest key T is found by bisection on the key bits with
 // warp-wide counts, stopping early once exactly k-1 keys lie at or above the candidate.
 template <int KPL>
-__device__ __forceinline__ void select_row_topk(const uint32_t* __restrict__ keys_row, int nb, int i, int k_keep,
+__device__ __forceinline__ void select_row_topk(uint32_t* __restrict__ keys_row, int nb, int i, int k_keep,
                                                 long long row, int32_t* __restrict__ row_ptr,
                                                 int32_t* __restrict__ col_idx) {
     const int lane = threadIdx.x % 32;
@@ -42,7 +42,7 @@ __device__ __forceinline__ void select_row_topk(const uint32_t* __restrict__ key
 #pragma unroll
     for (int s = 0; s < KPL; ++s) {
         const int j = s * 32 + lane;
-        // non-candidates (padding, the diagonal) get key 0; every bisection candidate is
+        // non-candidates (padding, the diagonal) get key 0; every search candidate is
         // >= 1, so they never count (a real score's key is >= 1: only the all-ones NaN
         // pattern maps to 0, and it is clamped to 1)
         key[s] = (j < nb && j != i) ? max(keys_row[j], 1u) : 0u;
@@ -52,8 +52,10 @@ __device__ __forceinline__ void select_row_topk(const uint32_t* __restrict__ key
     // counts at the two ends put it if the keys were spread evenly in between
     // (interpolation), with a halving probe after any interpolation that did not at
     // least halve the range, so the search never takes more than twice the 33 steps
-    // of plain bisection.  It stops early when exactly k-1 keys are >= the probe.
+    // of plain bisection.  It stops early when exactly k-1 keys are >= the probe
+    // ("exact": then no key needs a tie decision).
     uint32_t T = 0u;
+    bool exact = kk == 0;
     if (kk > 0) {
         uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
         int nc = 0;
@@ -66,25 +68,25 @@ __device__ __forceinline__ void select_row_topk(const uint32_t* __restrict__ key
             kmax = max(kmax, key[s]);
         }
         uint32_t lo = __reduce_min_sync(0xFFFFFFFFu, kmin);
-        const uint32_t top = __reduce_max_sync(0xFFFFFFFFu, kmax);
+        // keys of finite scores are at most 0xFF7FFFFF, so hi = top + 1 fits in 32 bits
+        // (the clamp only matters for a NaN score, which the caller rules out)
+        uint32_t hi = min(__reduce_max_sync(0xFFFFFFFFu, kmax), 0xFFFFFFFEu) + 1u;
         int c_lo = __reduce_add_sync(0xFFFFFFFFu, nc);  // candidates: count(key >= lo)
         int c_hi = 0;
-        // hi = top + 1 as a 64-bit bound: top can be the largest key
-        uint64_t hi = static_cast<uint64_t>(top) + 1u;
         bool halve = false;
         T = lo;
 #pragma unroll 1
         for (int it = 0; it < 72 && hi - lo > 1u; ++it) {
-            const uint64_t range = hi - lo;
-            uint64_t off;
+            const uint32_t range = hi - lo;
+            uint32_t off;
             if (halve) {
                 off = range >> 1;
             } else {
-                const float f = static_cast<float>(c_lo - kk) / static_cast<float>(c_lo - c_hi);
-                off = static_cast<uint64_t>(f * static_cast<float>(range));
+                const float f = __fdividef(static_cast<float>(c_lo - kk), static_cast<float>(c_lo - c_hi));
+                off = static_cast<uint32_t>(f * static_cast<float>(range));
             }
-            off = off < 1u ? 1u : (off > range - 1u ? range - 1u : off);
-            const uint32_t cand = static_cast<uint32_t>(lo + off);
+            off = min(max(off, 1u), range - 1u);
+            const uint32_t cand = lo + off;
             // four independent partial counts keep the add chains short
             int c4[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -92,6 +94,7 @@ __device__ __forceinline__ void select_row_topk(const uint32_t* __restrict__ key
             const int cnt = __reduce_add_sync(0xFFFFFFFFu, (c4[0] + c4[1]) + (c4[2] + c4[3]));
             if (cnt == kk) {  // {key >= cand} is exactly the top k-1
                 T = cand;
+                exact = true;
                 break;
             }
             if (cnt > kk) {
@@ -102,33 +105,46 @@ __device__ __forceinline__ void select_row_topk(const uint32_t* __restrict__ key
                 c_hi = cnt;
             }
             T = lo;
-            halve = !halve && 2u * (hi - lo) > range;
+            halve = !halve && 2ull * (hi - lo) > range;
         }
     }
-    int n_gt = 0;
-    if (kk > 0) {
+    // Keys equal to T are kept lowest j first until k-1 are kept (only needed when the
+    // search ended on a key value with ties possible).
+    int need_eq = 0;
+    if (!exact) {
         int g4[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int s = 0; s < KPL; ++s) g4[s & 3] += key[s] > T ? 1 : 0;
-        n_gt = __reduce_add_sync(0xFFFFFFFFu, (g4[0] + g4[1]) + (g4[2] + g4[3]));
+        need_eq = kk - __reduce_add_sync(0xFFFFFFFFu, (g4[0] + g4[1]) + (g4[2] + g4[3]));
     }
-    const int need_eq = kk - n_gt;  // how many keys equal to T to keep (lowest j first)
-    int32_t* out = col_idx + row * k_keep;
+    // The kept j in ascending order: ballot prefix counts give each its position in a
+    // staging list over this row's own key buffer (every lane has read its keys), which
+    // then goes out with coalesced stores.
+    __syncwarp();
+    int32_t* stage = reinterpret_cast<int32_t*>(keys_row);
     int pos = 0, eq_seen = 0;
 #pragma unroll
     for (int s = 0; s < KPL; ++s) {
         const int j = s * 32 + lane;
         const bool cand = key[s] != 0u;  // j < nb and j != i
-        const bool is_eq = kk > 0 && cand && key[s] == T;
-        const uint32_t eq_mask = __ballot_sync(0xFFFFFFFFu, is_eq);
-        const int eq_rank = eq_seen + __popc(eq_mask & lt);
-        const bool keep = (j == i) || (kk > 0 && cand && key[s] > T) || (is_eq && eq_rank < need_eq);
+        bool keep;
+        if (exact) {
+            keep = (j == i) || (kk > 0 && cand && key[s] >= T);
+        } else {
+            const bool is_eq = cand && key[s] == T;
+            const uint32_t eq_mask = __ballot_sync(0xFFFFFFFFu, is_eq);
+            keep = (j == i) || (cand && key[s] > T) || (is_eq && eq_seen + __popc(eq_mask & lt) < need_eq);
+            eq_seen += __popc(eq_mask);
+        }
         const uint32_t m = __ballot_sync(0xFFFFFFFFu, keep);
-        if (keep) out[pos + __popc(m & lt)] = j;
+        if (keep) stage[pos + __popc(m & lt)] = j;
         pos += __popc(m);
-        eq_seen += __popc(eq_mask);
     }
+    __syncwarp();
+    int32_t* out = col_idx + row * k_keep;
+    for (int e = lane; e < k_keep; e += 32) out[e] = stage[e];
     if (lane == 0) row_ptr[row] = static_cast<int32_t>(row * k_keep);
+    __syncwarp();  // the staging area is reused by the caller
 }
 
 template <int D, int QT, int KPL>
@@ -306,7 +322,7 @@ constexpr size_t select_gemm_smem_bytes(int KPL) {
 // CTA = (b*h, 32 query blocks), 320 threads, two CTAs per SM:
 //   warp 8  : TMA of the raw means (box 32 channels x rows, 128-byte swizzle: the
 //             K-major operand layout): the Q tile once, then K chunks (128 key blocks x
-//             32 channels) through a two-slot ring.
+//             32 channels) through a three-slot ring.
 //   warp 9  : TMEM allocation (256 columns: 8 key tiles x 32 query blocks) and the thread
 //             that issues the MMAs, 12 per chunk ((k_t,q_t), (k_t,q_l), (k_l,q_t) at 4 K
 //             steps).
@@ -318,10 +334,15 @@ constexpr int kSelTcThreads = 320;
 constexpr int kSelTcTile = 128 * 128;           // bytes of one K chunk (128 rows x 32 fp32)
 constexpr int kSelTcQBytes = 4 * 32 * 128;      // Q tile: 4 channel chunks x 32 rows x 128 B
 constexpr int kSelTcOffQ = 0, kSelTcOffQl = kSelTcQBytes, kSelTcOffX = 2 * kSelTcQBytes;
-constexpr int kSelTcOffXl = kSelTcOffX + 2 * kSelTcTile;
-constexpr int kSelTcOffBar = kSelTcOffXl + 2 * kSelTcTile;  // 96 KB of operands
-constexpr int kSelTcNumBars = 2 + 2 + 2 + 2 + 2 + 1;  // q_full, ql_full, x_full[2], x_empty[2], l_full[2], l_empty[2], done
-constexpr size_t kSelTcSmemBytes = kSelTcOffBar + kSelTcNumBars * 8 + 16 + 1024;
+constexpr int kSelTcStages = 3;                // raw K chunks in flight
+constexpr int kSelTcOffXl = kSelTcOffX + kSelTcStages * kSelTcTile;
+constexpr int kSelTcOffBar = kSelTcOffXl + 2 * kSelTcTile;  // 112 KB of operands
+// q_full, ql_full, x_full[S], x_empty[S], l_full[2], l_empty[2], done
+constexpr int kSelTcNumBars = 2 + 2 * kSelTcStages + 2 + 2 + 1;
+// No alignment slack: two CTAs must fit in one SM's 228 KB.  Dynamic shared memory
+// starts 1024-byte aligned when the kernel has no static shared memory; the kernel
+// checks that, and if it ever is not, latches SBSA_ERR_TIMEOUT and returns at once.
+constexpr size_t kSelTcSmemBytes = kSelTcOffBar + kSelTcNumBars * 8 + 16;
 
 constexpr uint32_t idesc_tf32_f32(int M, int N) {
     return (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
@@ -357,21 +378,26 @@ __global__ void __launch_bounds__(kSelTcThreads, 2) select_tc_kernel(const __gri
     constexpr int HALF = kSelTcRows / 2;          // query rows per top-k round
     static_assert(HALF * NBP * 4 <= kSelTcOffBar, "keys of one round fit over the operand buffers");
     extern __shared__ __align__(1024) uint8_t sel_tc_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sel_tc_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = sel_tc_raw;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSelTcOffBar);
     uint64_t* q_full = bars;
     uint64_t* ql_full = bars + 1;
+    constexpr int S = kSelTcStages;
     uint64_t* x_full = bars + 2;
-    uint64_t* x_empty = bars + 4;
-    uint64_t* l_full = bars + 6;
-    uint64_t* l_empty = bars + 8;
-    uint64_t* done = bars + 10;
+    uint64_t* x_empty = x_full + S;
+    uint64_t* l_full = x_empty + S;
+    uint64_t* l_empty = l_full + 2;
+    uint64_t* done = l_empty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kSelTcNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem);  // [HALF][NBP], after the MMAs
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     if (launch_aborted(p.epoch)) return;
+    if (smem_u32(smem) & 1023u) {  // the swizzled operand layouts need 1024-byte alignment
+        if (tid == 0) abort_launch(p.epoch);
+        return;
+    }
     const int nb = p.nb;
     const long long bh = blockIdx.y;
     const int i0 = blockIdx.x * kSelTcRows;
@@ -416,15 +442,15 @@ __global__ void __launch_bounds__(kSelTcThreads, 2) select_tc_kernel(const __gri
             for (int a = 0; a < 4; ++a) tma_load_2d(smem + kSelTcOffQ + a * 32 * 128, &map_q, q_full, 32 * a, row_q, pol);
             int c = 0;
             for (; c < n_chunks; ++c) {
-                const int b = c & 1;
-                if (c >= 2 && !(ok = wait(&x_empty[b], ((c - 2) >> 1) & 1))) break;
+                const int b = c % S;
+                if (c >= S && !(ok = wait(&x_empty[b], ((c - S) / S) & 1))) break;
                 mbar_arrive_expect_tx(&x_full[b], kSelTcTile);
                 tma_load_2d(smem + kSelTcOffX + b * kSelTcTile, &map_k, &x_full[b], 32 * (c & 3), row_k + 128 * (c >> 2), pol);
             }
             if (!ok) {
                 volatile int never = 0;
                 mbar_wait_bounded(q_full, 0, &never, kWaitLimitNs);
-                for (int q = c - 2 < 0 ? 0 : c - 2; q < c; ++q) mbar_wait_bounded(&x_full[q & 1], (q >> 1) & 1, &never, kWaitLimitNs);
+                for (int q = c - S < 0 ? 0 : c - S; q < c; ++q) mbar_wait_bounded(&x_full[q % S], (q / S) & 1, &never, kWaitLimitNs);
             }
         }
     } else if (warp == 9) {
@@ -435,15 +461,15 @@ __global__ void __launch_bounds__(kSelTcThreads, 2) select_tc_kernel(const __gri
             const uint32_t x_addr = smem_u32(smem + kSelTcOffX), xl_addr = smem_u32(smem + kSelTcOffXl);
             ok = wait(q_full, 0) && wait(ql_full, 0);
             for (int c = 0; ok && c < n_chunks; ++c) {
-                const int b = c & 1, t = c >> 2, dc = c & 3;
-                if (!(ok = wait(&x_full[b], (c >> 1) & 1))) break;
-                if (!(ok = wait(&l_full[b], (c >> 1) & 1))) break;
+                const int b = c % S, lb = c & 1, t = c >> 2, dc = c & 3;
+                if (!(ok = wait(&x_full[b], (c / S) & 1))) break;
+                if (!(ok = wait(&l_full[lb], (c >> 1) & 1))) break;
                 tc_fence_after();
                 const uint32_t d = tmem + t * kSelTcRows;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     const uint64_t xa = sdesc_sw128(x_addr + b * kSelTcTile + ks * 32, 16, 1024);
-                    const uint64_t la = sdesc_sw128(xl_addr + b * kSelTcTile + ks * 32, 16, 1024);
+                    const uint64_t la = sdesc_sw128(xl_addr + lb * kSelTcTile + ks * 32, 16, 1024);
                     const uint64_t qb = sdesc_sw128(q_addr + dc * 32 * 128 + ks * 32, 16, 1024);
                     const uint64_t lb = sdesc_sw128(ql_addr + dc * 32 * 128 + ks * 32, 16, 1024);
                     umma_tf32_ss(d, xa, qb, id, (dc > 0 || ks > 0) ? 1u : 0u);
@@ -451,7 +477,7 @@ __global__ void __launch_bounds__(kSelTcThreads, 2) select_tc_kernel(const __gri
                     umma_tf32_ss(d, la, qb, id, 1u);
                 }
                 umma_commit(&x_empty[b]);
-                umma_commit(&l_empty[b]);
+                umma_commit(&l_empty[lb]);
             }
             umma_commit(done);  // every MMA this thread issued (also on the error path)
             if (!ok) {
@@ -472,18 +498,18 @@ __global__ void __launch_bounds__(kSelTcThreads, 2) select_tc_kernel(const __gri
         fence_proxy_async_smem();
         mbar_arrive(ql_full);
         for (int c = 0; ok && c < n_chunks; ++c) {
-            const int b = c & 1;
-            if (!(ok = wait(&x_full[b], (c >> 1) & 1))) break;
+            const int b = c % S, lb = c & 1;
+            if (!(ok = wait(&x_full[b], (c / S) & 1))) break;
             float4 v[kSelTcTile / 16 / 256];
 #pragma unroll
             for (int u = 0; u < kSelTcTile / 16 / 256; ++u)
                 v[u] = tf32_low_part(reinterpret_cast<const float4*>(smem + kSelTcOffX + b * kSelTcTile)[tid + 256 * u]);
-            if (c >= 2 && !(ok = wait(&l_empty[b], ((c - 2) >> 1) & 1))) break;
+            if (c >= 2 && !(ok = wait(&l_empty[lb], ((c - 2) >> 1) & 1))) break;
 #pragma unroll
             for (int u = 0; u < kSelTcTile / 16 / 256; ++u)
-                reinterpret_cast<float4*>(smem + kSelTcOffXl + b * kSelTcTile)[tid + 256 * u] = v[u];
+                reinterpret_cast<float4*>(smem + kSelTcOffXl + lb * kSelTcTile)[tid + 256 * u] = v[u];
             fence_proxy_async_smem();
-            mbar_arrive(&l_full[b]);
+            mbar_arrive(&l_full[lb]);
         }
     }
     // ---------------------------------------------------------------- top-k
