@@ -41,7 +41,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="long122880",
                     help="tiny | 480p | 720p | long122880 | sweep<keep%%> e.g. sweep100")
@@ -105,13 +105,16 @@ def dist_env():
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+    """nvidia-smi sampling of SM clocks and throttle reasons.  Sampling starts before
+    the warm-up (nvidia-smi takes a moment to start) every 50 ms; only the samples whose
+    timestamps fall inside the timed region (mark_begin .. mark_end) are reported."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
         self.proc = None
+        self.t0 = self.t1 = None
         self.path = os.path.join("/tmp", f"sbsa_clocks_{os.getpid()}.csv")
         try:
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
@@ -125,11 +128,24 @@ class ClockSampler:
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
-        time.sleep(0.3)
+
+    def mark_begin(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    @staticmethod
+    def _epoch(stamp: str):
+        import datetime
+        try:
+            return datetime.datetime.strptime(stamp.strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
 
     def stop(self):
         if self.proc is None:
@@ -140,24 +156,28 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.f.close()
-        sm, mx, reasons = [], [], set()
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
             for line in f:
                 parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 7:
+                if len(parts) < 8:
                     continue
                 try:
-                    sm.append(float(parts[0]))
-                    mx.append(float(parts[1]))
+                    rows.append((self._epoch(parts[0]), float(parts[1]), float(parts[2]),
+                                 [n for n, v in zip(names, parts[4:8]) if v.lower() == "active"]))
                 except ValueError:
                     continue
-                for n, v in zip(names, parts[3:7]):
-                    if v.lower() == "active":
-                        reasons.add(n)
         os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        inside = [r for r in rows if r[0] is not None and self.t0 is not None and self.t1 is not None
+                  and self.t0 - 0.05 <= r[0] <= self.t1 + 0.05]
+        use = inside if inside else rows[-3:]
+        sm = [r[1] for r in use]
+        reasons = sorted({n for r in use for n in r[3]})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(r[2] for r in use) if use else None,
+                "reasons": reasons, "samples": len(sm),
+                "window": "timed region" if inside else "last samples (none inside the timed region)"}
 
 
 # ------------------------------------------------------------------ traffic record
@@ -303,13 +323,14 @@ def run_gpu(args, wl):
             pg.barrier()
         torch.cuda.synchronize(dev)
 
+    clocks = ClockSampler(local)
+    clocks.start()
     for _ in range(args.warmup):
         step()
     sbsa.sbsa_check(stream)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    clocks = ClockSampler(local)
-    clocks.start()
     barrier()
+    clocks.mark_begin()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
@@ -317,6 +338,7 @@ def run_gpu(args, wl):
         step(evs[i])
     t_end.record(stream)
     barrier()
+    clocks.mark_end()
     clk = clocks.stop()
     sbsa.sbsa_check(stream)
     elapsed_ms = t_start.elapsed_time(t_end)

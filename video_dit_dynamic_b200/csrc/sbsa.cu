@@ -159,20 +159,6 @@ sbsa_status launch_select_t(const sbsa_shape* s, const float* qm, const float* k
 }
 
 template <int KPL>
-sbsa_status launch_select_gemm(const sbsa_shape* s, const float* qm, const float* km, int k, int32_t* rp, int32_t* ci,
-                               cudaStream_t st) {
-    const int nb = num_blocks(s);
-    const size_t smem = select_gemm_smem_bytes(KPL);
-    auto kern = select_gemm_kernel<KPL>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return cuda_fail(e, "select smem attribute");
-    const dim3 grid((nb + kSelQT - 1) / kSelQT, static_cast<unsigned>(s->batch * s->heads));
-    kern<<<grid, 256, smem, st>>>(qm, km, nb, k, rp, ci, num_rows(s));
-    e = cudaGetLastError();
-    return e == cudaSuccess ? SBSA_OK : cuda_fail(e, "select launch");
-}
-
-template <int KPL>
 sbsa_status launch_select_tc(const sbsa_shape* s, const float* qm, const float* km, int k, int32_t* rp, int32_t* ci,
                              cudaStream_t st) {
     const int nb = num_blocks(s);

@@ -6,15 +6,17 @@
 // fp32.  Kept: j = i, plus the k-1 highest-scoring j != i, ties to the lower j; written
 // in ascending j order into a CSR list with a uniform row length k.
 //
-// One CTA per (b*h, tile of QT query blocks), 256 threads.
-//   scores : each thread takes one key block j at a time, holds kmean_j in registers
-//            and forms its dot product with the QT query means broadcast from shared
-//            memory; the fp32 scores go to shared memory as order-preserving uint32 keys.
-//   top-k  : one warp per query row.  Lane l holds keys j = l + 32 r.  The (k-1)-th
-//            largest key T is found by bisection on the key bits (warp-wide counts,
-//            early exit); then keys > T are kept, and keys == T in ascending j until k-1
-//            are kept; the output position of each kept j is a ballot prefix count,
-//            which yields the ascending order directly.
+// Two kernels share the top-k:
+//   select_tc_kernel (head_dim 128, nb <= 1024): scores on the tensor cores in tf32 with
+//     an exact three-product split, described above the kernel.
+//   select_kernel (other shapes): one CTA per (b*h, tile of QT query blocks); each thread
+//     takes one key block j at a time, holds kmean_j in registers and forms its dot
+//     product with the QT query means broadcast from shared memory.
+// Scores go to shared memory as order-preserving uint32 keys.  Top-k: one warp per
+// query row, lane l holding keys j = l + 32 r; the (k-1)-th largest key T comes from a
+// search with warp-wide counts; keys > T are kept, and keys == T in ascending j until
+// k-1 are kept; the output position of each kept j is a ballot prefix count, which
+// yields the ascending order directly.
 #pragma once
 #include "common.cuh"
 #include "ptx.cuh"
@@ -29,8 +31,8 @@ __device__ __forceinline__ uint32_t order_key(float s) {
 
 // Keep, for query block i, the diagonal and the k_keep-1 largest of the other keys
 // (ties: lower j), writing them in ascending j.  One warp; lane l holds keys
-// j = l + 32 s.  The (k-1)-th largest key T is found by bisection on the key bits with
-// warp-wide counts, stopping early once exactly k-1 keys lie at or above the candidate.
+// j = l + 32 s.  keys_row (shared memory, this row only) is reused as staging space
+// for the output list.
 template <int KPL>
 __device__ __forceinline__ void select_row_topk(uint32_t* __restrict__ keys_row, int nb, int i, int k_keep,
                                                 long long row, int32_t* __restrict__ row_ptr,
@@ -197,116 +199,6 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ q
     for (int r = warp; r < nq; r += blockDim.x / 32)
         select_row_topk<KPL>(keys + r * NBP, nb, i0 + r, k_keep, bh * nb + i0 + r, row_ptr, col_idx);
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) row_ptr[n_rows] = static_cast<int32_t>(n_rows * k_keep);
-}
-
-// Scores through a shared-memory, register-blocked fp32 GEMM, for nb <= 1024.
-// CTA = (b*h, 32 query blocks), 256 threads.  Key means stream through shared memory
-// in chunks of 256 key blocks x 32 channels.  Thread (warp w, lane l) owns query rows
-// {l/8 + 4 r : r < 8} and key blocks {256 c + 32 w + l%8 + 8 s : s < 4}; rows and key
-// blocks interleave so that each shared-memory load is conflict-free or broadcast.
-// Products accumulate over channel pairs with packed fp32x2 FMAs, (even, odd) channel
-// partial sums added at the end.  Then one warp per row selects as above.
-constexpr int kSelQT = 32;
-constexpr int kSelQStride = 132;  // floats per query-mean row in shared memory (128 + 4)
-constexpr int kSelKStride = 36;   // floats per key-mean row of a 32-channel chunk (32 + 4)
-constexpr int kSelJChunk = 256;
-constexpr int kSelCChunk = 32;
-
-template <int KPL>
-__global__ void __launch_bounds__(256, 1) select_gemm_kernel(const float* __restrict__ q_mean,
-                                                            const float* __restrict__ k_mean, int nb, int k_keep,
-                                                            int32_t* __restrict__ row_ptr,
-                                                            int32_t* __restrict__ col_idx, long long n_rows) {
-    constexpr int D = 128;
-    constexpr int NBP = 32 * KPL;
-    extern __shared__ __align__(16) uint8_t sel_smem[];
-    float* qs = reinterpret_cast<float*>(sel_smem);                        // [32][132]
-    float* ks = qs + kSelQT * kSelQStride;                                 // [2][256][36]
-    uint32_t* keys = reinterpret_cast<uint32_t*>(ks + 2 * kSelJChunk * kSelKStride);  // [32][NBP]
-
-    const long long bh = blockIdx.y;
-    const int i0 = blockIdx.x * kSelQT;
-    const int nq = min(kSelQT, nb - i0);
-    const float* qm = q_mean + (bh * nb + i0) * D;
-    const float* km = k_mean + bh * nb * D;
-    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-
-    // query means -> qs (rows past nq are zero)
-    for (int f = tid; f < kSelQT * D / 4; f += 256) {
-        const int r = f / (D / 4), c4 = f % (D / 4);
-        const float4 v = r < nq ? __ldg(reinterpret_cast<const float4*>(qm) + f) : make_float4(0.f, 0.f, 0.f, 0.f);
-        *reinterpret_cast<float4*>(qs + r * kSelQStride + c4 * 4) = v;
-    }
-
-    const int li = lane / 8, lj = lane % 8;
-    auto load_chunk = [&](int jc, int cc, float* dst) {
-        // 256 key rows x 32 channels = 2048 x 16 B, 8 per thread, asynchronous copies
-        // (coalesced along channels; rows past nb are zero-filled)
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const int f = tid + 256 * r;
-            const int row = f / 8, q4 = f % 8;
-            const int j = jc + row;
-            const float* src = km + static_cast<long long>(j < nb ? j : 0) * D + cc * kSelCChunk + q4 * 4;
-            const uint32_t dst_s = smem_u32(dst + row * kSelKStride + q4 * 4);
-            const uint32_t bytes = j < nb ? 16u : 0u;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_s), "l"(src), "r"(bytes) : "memory");
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-
-    for (int jc = 0; jc < nb; jc += kSelJChunk) {
-        float2 acc[8][4];
-#pragma unroll
-        for (int a = 0; a < 8; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b) acc[a][b] = make_float2(0.f, 0.f);
-        __syncthreads();  // previous chunk's readers are done with ks
-        if (jc == 0) load_chunk(0, 0, ks);  // later chunks' first slice was prefetched below
-        for (int cc = 0; cc < D / kSelCChunk; ++cc) {
-            float* cur = ks + (cc & 1) * kSelJChunk * kSelKStride;
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
-            __syncthreads();  // cur is filled for every thread; the other buffer is free
-            if (cc + 1 < D / kSelCChunk)
-                load_chunk(jc, cc + 1, ks + ((cc + 1) & 1) * kSelJChunk * kSelKStride);
-            else if (jc + kSelJChunk < nb)
-                load_chunk(jc + kSelJChunk, 0, ks + ((cc + 1) & 1) * kSelJChunk * kSelKStride);
-#pragma unroll
-            for (int c = 0; c < kSelCChunk; c += 4) {
-                float4 qv[8], kv[4];
-#pragma unroll
-                for (int a = 0; a < 8; ++a)
-                    qv[a] = *reinterpret_cast<const float4*>(qs + (li + 4 * a) * kSelQStride + cc * kSelCChunk + c);
-#pragma unroll
-                for (int b = 0; b < 4; ++b)
-                    kv[b] = *reinterpret_cast<const float4*>(cur + (warp * 32 + lj + 8 * b) * kSelKStride + c);
-#pragma unroll
-                for (int a = 0; a < 8; ++a)
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        acc[a][b] = __ffma2_rn(make_float2(qv[a].x, qv[a].y), make_float2(kv[b].x, kv[b].y), acc[a][b]);
-                        acc[a][b] = __ffma2_rn(make_float2(qv[a].z, qv[a].w), make_float2(kv[b].z, kv[b].w), acc[a][b]);
-                    }
-            }
-        }
-#pragma unroll
-        for (int a = 0; a < 8; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int j = jc + warp * 32 + lj + 8 * b;
-                if (j < NBP) keys[(li + 4 * a) * NBP + j] = order_key(acc[a][b].x + acc[a][b].y);
-            }
-    }
-    __syncthreads();
-
-    for (int r = warp; r < nq; r += 8)
-        select_row_topk<KPL>(keys + r * NBP, nb, i0 + r, k_keep, bh * nb + i0 + r, row_ptr, col_idx);
-    if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) row_ptr[n_rows] = static_cast<int32_t>(n_rows * k_keep);
-}
-
-constexpr size_t select_gemm_smem_bytes(int KPL) {
-    return (static_cast<size_t>(kSelQT) * kSelQStride + 2ull * kSelJChunk * kSelKStride) * 4 +
-           static_cast<size_t>(kSelQT) * 32 * KPL * 4;
 }
 
 // ---------------------------------------------------------------- tensor-core scores
