@@ -46,8 +46,8 @@ def _random_means(B, H, nb, d, seed):
 
 
 @pytest.mark.parametrize("nb,k,d", [(1, 1, 64), (5, 2, 64), (33, 7, 128), (64, 64, 64), (100, 1, 128),
-                                    (257, 51, 128), (700, 70, 128), (960, 96, 128), (1500, 150, 64),
-                                    (2048, 205, 128)])
+                                    (96, 96, 128), (257, 51, 128), (700, 70, 128), (960, 96, 128),
+                                    (1024, 100, 128), (1500, 150, 64), (2048, 205, 128)])
 def test_select_matches_oracle(nb, k, d):
     B, H = 1, 2
     qm, km = _random_means(B, H, nb, d, seed=nb * 7 + k)
@@ -59,8 +59,9 @@ def test_select_matches_oracle(nb, k, d):
     pu.assert_selection_ok(ci.cpu().numpy().reshape(B, H, nb, k), ref, qn, kn, k)
 
 
-def test_select_exact_ties_prefer_lower_index():
-    nb, d, k = 40, 64, 4
+@pytest.mark.parametrize("d", [64, 128])
+def test_select_exact_ties_prefer_lower_index(d):
+    nb, k = 40, 4
     qm, km = _random_means(1, 1, nb, d, seed=5)
     km *= 0.01
     for j in (3, 17, 29, 31, 39):  # identical key blocks: exact ties in every row's ranking
@@ -69,10 +70,24 @@ def test_select_exact_ties_prefer_lower_index():
     _, ci = pu.gpu_select(s, qm, km, k)
     got = ci.cpu().numpy().reshape(nb, k)
     ref = oracle.select(qm.double().cpu().numpy(), km.double().cpu().numpy(), k)[0, 0]
-    # row 0: the five tied copies outscore every other block; the three lowest win
+    # row 0: the five tied copies outscore every other block; the three lowest win (exact
+    # ties survive the tensor-core path too: equal means give bit-equal scores)
     np.testing.assert_array_equal(got[0], ref[0])
     np.testing.assert_array_equal(got[0], [0, 3, 17, 29])
     np.testing.assert_array_equal(got, ref)
+
+
+@pytest.mark.parametrize("scale", [1e-3, 1e4])
+def test_select_scaled_means(scale):
+    """The tf32 split of the scores is exact at any magnitude: scaled means select alike."""
+    nb, k, d = 300, 30, 128
+    qm, km = _random_means(1, 2, nb, d, seed=11)
+    qm *= scale
+    km *= scale
+    s = sbsa.make_shape(1, 2, nb * 64, d, 64)
+    rp, ci = pu.gpu_select(s, qm, km, k)
+    qn, kn = qm.double().cpu().numpy(), km.double().cpu().numpy()
+    pu.assert_selection_ok(ci.cpu().numpy().reshape(1, 2, nb, k), oracle.select(qn, kn, k), qn, kn, k)
 
 
 def test_select_validate_csr_accepts_output():
