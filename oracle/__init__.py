@@ -54,6 +54,8 @@ def _load():
         lib.oracle_attention.argtypes = [I, I, I, I, I, I, P, P, P, I, P, P,
                                          ctypes.c_double, ctypes.c_long, P, P]
         lib.oracle_attention.restype = I
+        lib.oracle_rope.argtypes = [I, I, I, I, I, I, I, ctypes.c_double, P, I, P]
+        lib.oracle_rope.restype = None
         lib.oracle_set_threads.argtypes = [I]
         lib.oracle_threads_used.restype = I
         _lib = lib
@@ -98,6 +100,40 @@ def pool(x, L: int, blk: int) -> np.ndarray:
     out = np.empty((B, H, nb, d), dtype=np.float64)
     _load().oracle_pool(B, H, L, Lp, d, blk, _ptr(xa), dt, _ptr(out))
     return out
+
+
+def rope_pairs(d: int) -> tuple[int, int, int]:
+    """Rotation pairs per axis (frame, row, column) for head dim d (see sbsa_oracle.c)."""
+    ph = d // 6
+    return d // 2 - 2 * ph, ph, ph
+
+
+def rope(x, grid: tuple[int, int, int], theta: float = 10000.0) -> np.ndarray:
+    """3D RoPE of x [B][H][Lp][d] (fp64 result, same shape; bf16 given as uint16 bits)."""
+    a, dt = _as_input(x)
+    B, H, Lp, d = a.shape
+    out = np.empty((B, H, Lp, d), dtype=np.float64)
+    _load().oracle_rope(B, H, Lp, d, grid[0], grid[1], grid[2], float(theta), _ptr(a), dt, _ptr(out))
+    return out
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """fp64 -> nearest bf16, ties to even, rounded once from the fp64 value; returned
+    as uint16 bit patterns."""
+    f32 = np.asarray(x, dtype=np.float64)
+    # exact: split the fp64 value at bf16 precision with round-half-to-even
+    m, e = np.frexp(f32)                       # f = m * 2^e, 0.5 <= |m| < 1
+    q = np.rint(m * 256.0) / 256.0             # 8 significant bits, ties to even
+    r = np.ldexp(q, e).astype(np.float32)      # exactly representable in bf16
+    return (r.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def rope_pool(x, grid: tuple[int, int, int], L: int, blk: int, theta: float = 10000.0):
+    """Step 0 + step 1: rotated tensor as bf16 bits, and the block means of those bf16
+    values (what the attention then sees)."""
+    rot = rope(x, grid, theta)
+    bits = bf16_round(rot)
+    return bits, pool(bits, L, blk)
 
 
 def score_row(qmean_bh: np.ndarray, kmean_bh: np.ndarray, i: int):

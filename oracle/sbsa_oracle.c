@@ -24,6 +24,15 @@
  *              non-causal, scale 1/sqrt(d) unless given.  Two-pass softmax (max,
  *              then exp-sums), not the online form.
  *
+ *   0. rope    (next step on the path, fused with 1 in the library) [Card] bullet
+ *              高效推理算子 and [Guide] item 4 融合内核: 3D RoPE runs as a fused kernel.
+ *              The pages give no frequencies; the reading taken here is the usual 3D
+ *              split of the head dimension into rotation pairs (2p, 2p+1): the first
+ *              P_t = d/2 - 2*P_h pairs rotate with the frame index, the next
+ *              P_h = floor(d/6) with the row index, the last P_w = P_h with the column
+ *              index of the token on the (T, H, W) latent grid (row-major); pair q of an
+ *              axis with P pairs turns by angle pos * theta^(-q/P), theta = 10000.
+ *
  * Inputs are read as fp32, bf16 (raw 16-bit patterns, converted exactly) or fp64.
  * Tensors are row-major [B][H][Lp][d]; means are [B][H][nb][d]; col_idx is
  * [B][H][nb][k].  Padded tokens t >= L are ignored as keys and their query rows
@@ -80,6 +89,32 @@ void oracle_pool(int B, int H, int L, int Lp, int d, int blk,
             for (int t = t0; t < t1; ++t)
                 s += elem(x, dtype, ((size_t)bh * Lp + t) * d + c);
             out[r * d + c] = t1 > t0 ? s / (double)(t1 - t0) : 0.0;
+        }
+    }
+}
+
+/* Step 0: 3D RoPE of one tensor [B][H][Lp][d] over the (gt, gh, gw) grid, in fp64.
+ * Every token t < Lp is rotated by its grid position t -> (t / (gh*gw), (t / gw) % gh,
+ * t % gw), padded tokens included.  out has the input's shape. */
+void oracle_rope(int B, int H, int Lp, int d, int gt, int gh, int gw, double theta,
+                 const void *x, int dtype, double *out) {
+    (void)gt;
+    const int half = d / 2, ph = d / 6, pw = d / 6, pt = half - ph - pw;
+    long rows = (long)B * H * Lp;
+#pragma omp parallel for schedule(static) num_threads(oracle_threads_used())
+    for (long r = 0; r < rows; ++r) {
+        long t = r % Lp;
+        long pos[3] = {t / ((long)gh * gw), (t / gw) % gh, t % gw};
+        for (int p = 0; p < half; ++p) {
+            int axis = p < pt ? 0 : (p < pt + ph ? 1 : 2);
+            int q = axis == 0 ? p : (axis == 1 ? p - pt : p - pt - ph);
+            int np = axis == 0 ? pt : (axis == 1 ? ph : pw);
+            double ang = (double)pos[axis] * pow(theta, -(double)q / (double)np);
+            double c = cos(ang), sn = sin(ang);
+            double a = elem(x, dtype, (size_t)r * d + 2 * p);
+            double b = elem(x, dtype, (size_t)r * d + 2 * p + 1);
+            out[(size_t)r * d + 2 * p] = a * c - b * sn;
+            out[(size_t)r * d + 2 * p + 1] = a * sn + b * c;
         }
     }
 }

@@ -39,6 +39,16 @@ MUTANTS = {
                           "int u = cols[n / blk] * blk + (n + 1) % blk;\n            logit[n]"),
     # the scale is dropped
     "scale_dropped": ("logit[n] = s * scale;", "logit[n] = s;"),
+    # RoPE turns the wrong way round in the second component (a reflection, norms kept)
+    "rope_sin_sign": ("out[(size_t)r * d + 2 * p + 1] = a * sn + b * c;",
+                      "out[(size_t)r * d + 2 * p + 1] = -a * sn + b * c;"),
+    # RoPE pairs of the row and column axes swapped
+    "rope_axes_swapped": ("int axis = p < pt ? 0 : (p < pt + ph ? 1 : 2);",
+                          "int axis = p < pt ? 0 : (p < pt + ph ? 2 : 1);"),
+    # RoPE frequency exponent off by one pair
+    "rope_freq_off_by_one": ("pow(theta, -(double)q / (double)np)", "pow(theta, -(double)(q + 1) / (double)np)"),
+    # RoPE row index taken with the wrong divisor
+    "rope_row_position": ("(t / gw) % gh, t % gw}", "(t / gh) % gw, t % gw}"),
 }
 
 

@@ -308,3 +308,110 @@ def test_oracle_accepts_fp32_and_bf16_consistently():
     o2, c2, _, _ = oracle.forward(*as_bits, 64, 16, 2)
     np.testing.assert_array_equal(c1, c2)
     np.testing.assert_array_equal(o1, o2)
+
+
+# ---------------------------------------------------------------- step 0: 3D RoPE
+# The pages name a fused 3D RoPE kernel (page "知识卡片…", 方法/产品要点, bullet 高效推理算子;
+# page "单卡 RTX 5090 跑 Wan2.2-A14B…", 四步拆解 item 4) but give no frequencies; the
+# reading (pair split, theta) is stated in sbsa_oracle.c.  These pins fix that reading
+# with values worked out by hand and with properties a rotation must have.
+
+def _one_token_grid(d, pos, grid=(4, 4, 8)):
+    """x [1,1,Lp,d] with an impulse (1, 0) in every pair of the token at grid position pos."""
+    gt, gh, gw = grid
+    Lp = gt * gh * gw
+    x = np.zeros((1, 1, Lp, d))
+    t = (pos[0] * gh + pos[1]) * gw + pos[2]
+    x[0, 0, t, 0::2] = 1.0
+    return x, t
+
+
+def test_rope_hand_values_d12():
+    # d = 12: 6 pairs, 2 per axis.  theta^(-q/2) at q = 1 is 1/sqrt(10000) = 0.01 exactly,
+    # so the column pair q = 1 of a token in column 5 turns by 0.05 rad; q = 0 by 5 rad.
+    x, t = _one_token_grid(12, (0, 0, 5))
+    r = oracle.rope(x, (4, 4, 8))[0, 0, t]
+    cos5, sin5 = 0.28366218546322625, -0.9589242746631385          # cos 5, sin 5
+    cos005, sin005 = 0.9987502603949663, 0.04997916927067833      # cos 0.05, sin 0.05
+    np.testing.assert_allclose(r[8:10], [cos5, sin5], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(r[10:12], [cos005, sin005], rtol=0, atol=1e-15)
+    # frame and row pairs: that token is at frame 0, row 0 -> untouched
+    np.testing.assert_array_equal(r[0:8], [1, 0, 1, 0, 1, 0, 1, 0])
+
+
+def test_rope_hand_values_rows_and_frames_d12():
+    # frame pairs are the first two, row pairs the next two; q = 0 turns by pos rad
+    x, t = _one_token_grid(12, (2, 3, 0))
+    r = oracle.rope(x, (4, 4, 8))[0, 0, t]
+    np.testing.assert_allclose(r[0:2], [math.cos(2.0), math.sin(2.0)], atol=1e-15)
+    np.testing.assert_allclose(r[2:4], [math.cos(0.02), math.sin(0.02)], atol=1e-15)
+    np.testing.assert_allclose(r[4:6], [math.cos(3.0), math.sin(3.0)], atol=1e-15)
+    np.testing.assert_allclose(r[6:8], [math.cos(0.03), math.sin(0.03)], atol=1e-15)
+    np.testing.assert_array_equal(r[8:12], [1, 0, 1, 0])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_rope_axis_split(d):
+    # moving a token along one axis changes only that axis' pairs: frame pairs first,
+    # then row pairs, then column pairs (d=128: 22 + 21 + 21 pairs; d=64: 12 + 10 + 10)
+    pt, ph, pw = oracle.rope_pairs(d)
+    assert (pt, ph, pw) == ((22, 21, 21) if d == 128 else (12, 10, 10))
+    base = oracle.rope(_one_token_grid(d, (0, 0, 0))[0], (4, 4, 8))[0, 0, 0]
+    np.testing.assert_array_equal(base[0::2], 1.0)  # position 0: identity
+    for axis, (lo, hi) in enumerate([(0, pt), (pt, pt + ph), (pt + ph, pt + ph + pw)]):
+        pos = [0, 0, 0]
+        pos[axis] = 1
+        x, t = _one_token_grid(d, tuple(pos))
+        r = oracle.rope(x, (4, 4, 8))[0, 0, t]
+        moved = np.nonzero(np.abs(r[0::2] - 1.0) > 1e-13)[0]
+        assert moved.min() == lo and moved.max() == hi - 1
+
+
+def test_rope_preserves_pair_norms():
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((2, 3, 96, 128))
+    r = oracle.rope(x, (3, 4, 8))
+    n_in = np.hypot(x[..., 0::2], x[..., 1::2])
+    n_out = np.hypot(r[..., 0::2], r[..., 1::2])
+    np.testing.assert_allclose(n_out, n_in, rtol=1e-13)
+
+
+def test_rope_dot_product_depends_on_offset_only():
+    # <R(m) q, R(n) k> is unchanged when both positions move by the same offset on the
+    # grid: rotations that turn with the position make attention translation-invariant
+    rng = np.random.default_rng(22)
+    d, grid = 64, (4, 4, 8)
+    Lp = 4 * 4 * 8
+    q = np.zeros((1, 1, Lp, d))
+    k = np.zeros((1, 1, Lp, d))
+    qv, kv = rng.standard_normal(d), rng.standard_normal(d)
+
+    def t_of(p):
+        return (p[0] * 4 + p[1]) * 8 + p[2]
+
+    pairs = [((0, 1, 2), (1, 3, 5)), ((2, 0, 0), (3, 2, 3)), ((1, 1, 1), (2, 3, 4))]
+    dots = []
+    for a, b in pairs:
+        q[:] = 0.0
+        k[:] = 0.0
+        q[0, 0, t_of(a)] = qv
+        k[0, 0, t_of(b)] = kv
+        rq, rk = oracle.rope(q, grid)[0, 0, t_of(a)], oracle.rope(k, grid)[0, 0, t_of(b)]
+        dots.append(rq @ rk)
+    # the three pairs share the offset (1, 2, 3)
+    np.testing.assert_allclose(dots, dots[0], rtol=1e-12)
+    assert abs(dots[0] - qv @ kv) > 1e-3  # and the rotation is not the identity
+
+
+def test_rope_pool_means_are_means_of_rounded_outputs():
+    x = inputs.random_qkv(1, 2, 64, 12, seed=23, dtype=torch.bfloat16)[0]
+    bits, means = oracle.rope_pool(inputs.bf16_bits(x), (2, 4, 8), 60, 16)
+    vals = torch.from_numpy(bits.astype(np.int32) << 16).view(torch.float32).double().numpy()
+    ref = np.stack([vals[:, :, i * 16:min((i + 1) * 16, 60)].mean(axis=2) for i in range(4)], axis=2)
+    np.testing.assert_allclose(means, ref, rtol=1e-13, atol=1e-15)
+
+
+def test_bf16_rounding_ties_to_even():
+    # 1 + 2^-8 is halfway between bf16 1.0 and 1.0078125: to even (1.0); 1 + 3*2^-9 up
+    vals = np.array([1.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -9, 1.0 + 3 * 2.0 ** -8, -2.5, 0.0])
+    assert [int(b) for b in oracle.bf16_round(vals)] == [0x3F80, 0x3F80, 0x3F81, 0x3F82, 0xC020, 0x0000]
