@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--impl", default="sbsa", choices=["sbsa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-rope", action="store_true", help="skip timing the fused RoPE + pooling kernel")
     ap.add_argument("--cpu-units", type=int, default=16, help="attention units in the CPU sample")
     return ap.parse_args()
 
@@ -359,6 +360,29 @@ def run_gpu(args, wl):
     forward_ms = f0.elapsed_time(f1) / min(args.steps, 5)
     sbsa.sbsa_check(stream)
 
+    # the fused 3D RoPE + pooling kernel (the step before pooling in a DiT layer), timed
+    # on its own: it reads Q and K once and writes the rotated tensors and the means
+    rope = None
+    if not args.no_rope:
+        table = torch.empty(sbsa.sbsa_rope_table_floats(wl.head_dim, wl.grid), dtype=torch.float32, device=dev)
+        sbsa.sbsa_rope_table_init(wl.head_dim, wl.grid, 10000.0, table, stream=stream)
+        qo, ko = torch.empty_like(q), torch.empty_like(kt)
+        for _ in range(2):
+            sbsa.sbsa_rope_pool_qk(shape, wl.grid, table, q, kt, qo, ko, qm, km, stream=stream)
+        r0 = torch.cuda.Event(enable_timing=True)
+        r1 = torch.cuda.Event(enable_timing=True)
+        n_rope = 5
+        r0.record(stream)
+        for _ in range(n_rope):
+            sbsa.sbsa_rope_pool_qk(shape, wl.grid, table, q, kt, qo, ko, qm, km, stream=stream)
+        r1.record(stream)
+        torch.cuda.synchronize(dev)
+        sbsa.sbsa_check(stream)
+        rope_ms = r0.elapsed_time(r1) / n_rope
+        rope_bytes = 4 * q.numel() * 2 + 2 * qm.numel() * 4
+        rope = {"ms": rope_ms, "algorithmic_bytes": rope_bytes}
+        del qo, ko, table
+
     # end to end through the public API from pinned host buffers
     e2e = None
     if not args.no_e2e:
@@ -382,10 +406,13 @@ def run_gpu(args, wl):
 
     t = max_over_ranks(pg, dev, {"elapsed": elapsed_ms, "att": statistics.mean(att_ms),
                                  "pool": statistics.mean(pool_ms), "sel": statistics.mean(sel_ms),
-                                 "forward": forward_ms, "e2e": e2e["ms"] if e2e is not None else 0.0})
+                                 "forward": forward_ms, "e2e": e2e["ms"] if e2e is not None else 0.0,
+                                 "rope": rope["ms"] if rope is not None else 0.0})
     elapsed_ms, att_avg, pool_avg, sel_avg, forward_ms = (t[n] for n in ("elapsed", "att", "pool", "sel", "forward"))
     if e2e is not None:
         e2e["ms"] = t["e2e"]
+    if rope is not None:
+        rope["ms"] = t["rope"]
     ms_step = elapsed_ms / args.steps
     value = job_tflops(flops, ws_n, ms_step)
 
@@ -416,6 +443,11 @@ def run_gpu(args, wl):
                 "pool_plus_select_effective_GB/s": pool_bytes / ((pool_avg + sel_avg) / 1e3) / 1e9,
                 "attention": {"ms": att_avg, "TFLOP/s": att_tflops},
                 "sbsa_forward_ms": forward_ms,
+                **({"rope_pool": {"ms": rope["ms"], "GB/s": rope["algorithmic_bytes"] / (rope["ms"] / 1e3) / 1e9,
+                                  "hbm_frac": rope["algorithmic_bytes"] / (rope["ms"] / 1e3) / 1e9 / peaks["hbm_gbs"],
+                                  "algorithmic_bytes": rope["algorithmic_bytes"],
+                                  "note": "3D RoPE fused with pooling, timed alone (not part of the step)"}}
+                   if rope is not None else {}),
             },
             "peaks": {"source": peak_src, **peaks},
         }

@@ -91,6 +91,37 @@ size_t sbsa_workspace_bytes(const sbsa_shape *shape, int32_t k_keep);
 sbsa_status sbsa_pool_qk(const sbsa_shape *shape, const void *q, const void *k, float *q_mean, float *k_mean,
                          void *stream);
 
+/* Step 0 fused with step 1 -- 3D RoPE of Q and K, then their block means (pages
+ * "知识卡片…", 方法/产品要点, bullet 高效推理算子, and "单卡 RTX 5090 跑 Wan2.2-A14B…",
+ * 四步拆解 item 4: 3D RoPE as a fused kernel, fewer temporaries and memory round trips;
+ * here it is fused with the pooling that follows, so Q and K cross HBM once for both).
+ * The pages give no frequencies.  The rotation used: the head dimension is cut into
+ * pairs (2p, 2p+1); the first P_T = d/2 - 2*P_H pairs turn with the token's frame
+ * index, the next P_H = floor(d/6) with its row index, the last P_W = P_H with its
+ * column index on the (grid_t, grid_h, grid_w) latent grid, tokens in row-major order
+ * (d = 128: 22 + 21 + 21 pairs; d = 64: 12 + 10 + 10); pair q of an axis with P pairs
+ * turns by pos * theta^(-q/P):  (x, y) -> (x cos - y sin, x sin + y cos).
+ *
+ * sbsa_rope_table_floats: floats of the cos/sin table for a grid (0 if invalid).
+ * sbsa_rope_table_init: fills `table` (device, 8-byte aligned, that many floats) with
+ *   (cos, sin) pairs computed in double and rounded to fp32; theta > 1 (10000 usual).
+ *   One small launch; the table can be kept for every layer with the same grid.
+ * sbsa_rope_pool_qk: grid_t * grid_h * grid_w must equal seq_len.
+ *   q, k         : bf16 [B][H][Lp][d] (device) before the rotation.
+ *   q_out, k_out : bf16 [B][H][Lp][d] (device, written): rotated in fp32, rounded to
+ *                  bf16 (ties to even).  May be the same buffers as q, k (in place).
+ *                  Padded tokens t >= L are copied unrotated.
+ *   q_mean, k_mean: fp32 [B][H][nb][d] (device, written): means of the rotated bf16
+ *                  values over the valid tokens of each block, as sbsa_pool_qk of q_out
+ *                  and k_out would give.
+ * One kernel launch, HBM-bandwidth bound (reads Q and K once, writes them once). */
+size_t sbsa_rope_table_floats(int32_t head_dim, int32_t grid_t, int32_t grid_h, int32_t grid_w);
+sbsa_status sbsa_rope_table_init(int32_t head_dim, int32_t grid_t, int32_t grid_h, int32_t grid_w, double theta,
+                                 float *table, void *stream);
+sbsa_status sbsa_rope_pool_qk(const sbsa_shape *shape, int32_t grid_t, int32_t grid_h, int32_t grid_w,
+                              const float *table, const void *q, const void *k, void *q_out, void *k_out,
+                              float *q_mean, float *k_mean, void *stream);
+
 /* Step 2 -- block selection (same bullet: keep ~10-20% of the blocks, chosen per
  * input at run time).  For each (b, h, query block i): score_j = <q_mean_i, k_mean_j>
  * in fp32; keep j = i plus the k_keep-1 highest-scoring other blocks (ties: lower j);

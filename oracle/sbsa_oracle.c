@@ -94,16 +94,21 @@ void oracle_pool(int B, int H, int L, int Lp, int d, int blk,
 }
 
 /* Step 0: 3D RoPE of one tensor [B][H][Lp][d] over the (gt, gh, gw) grid, in fp64.
- * Every token t < Lp is rotated by its grid position t -> (t / (gh*gw), (t / gw) % gh,
- * t % gw), padded tokens included.  out has the input's shape. */
+ * Token t < L = gt*gh*gw is rotated by its grid position t -> (t / (gh*gw),
+ * (t / gw) % gh, t % gw); padded tokens (t >= L) have no position and are copied
+ * unrotated.  out has the input's shape. */
 void oracle_rope(int B, int H, int Lp, int d, int gt, int gh, int gw, double theta,
                  const void *x, int dtype, double *out) {
-    (void)gt;
     const int half = d / 2, ph = d / 6, pw = d / 6, pt = half - ph - pw;
+    const long L = (long)gt * gh * gw;
     long rows = (long)B * H * Lp;
 #pragma omp parallel for schedule(static) num_threads(oracle_threads_used())
     for (long r = 0; r < rows; ++r) {
         long t = r % Lp;
+        if (t >= L) {
+            for (int c = 0; c < d; ++c) out[(size_t)r * d + c] = elem(x, dtype, (size_t)r * d + c);
+            continue;
+        }
         long pos[3] = {t / ((long)gh * gw), (t / gw) % gh, t % gw};
         for (int p = 0; p < half; ++p) {
             int axis = p < pt ? 0 : (p < pt + ph ? 1 : 2);

@@ -113,3 +113,20 @@ def test_binding_rejects_cpu_tensors(lib):
     m = torch.zeros(1, 1, 2, 64)
     with pytest.raises(TypeError):
         sbsa.sbsa_pool_qk(s, x, x, m, m, stream=0)
+
+
+def test_rope_table_size_and_argument_errors():
+    from video_dit_dynamic_b200 import sbsa
+    # d = 128: 22 frame, 21 row, 21 column pairs; (cos, sin) per grid position and pair
+    assert sbsa.sbsa_rope_table_floats(128, (24, 64, 80)) == 2 * (24 * 22 + 64 * 21 + 80 * 21)
+    assert sbsa.sbsa_rope_table_floats(64, (2, 3, 4)) == 2 * (2 * 12 + 3 * 10 + 4 * 10)
+    assert sbsa.sbsa_rope_table_floats(96, (2, 3, 4)) == 0
+    assert sbsa.sbsa_rope_table_floats(128, (0, 3, 4)) == 0
+    lib = sbsa.load()
+    s = sbsa.make_shape(1, 2, 120, 128, 64)
+    # grid does not cover seq_len: rejected before any pointer is looked at
+    st = lib.sbsa_rope_pool_qk(ctypes.byref(s), 2, 3, 4, None, None, None, None, None, None, None, None)
+    assert st == 1 and b"grid" in lib.sbsa_last_error_message()
+    st = lib.sbsa_rope_pool_qk(ctypes.byref(s), 2, 6, 10, None, None, None, None, None, None, None, None)
+    assert st == 1 and b"null" in lib.sbsa_last_error_message()
+    assert lib.sbsa_rope_table_init(128, 2, 6, 10, 1.0, None, None) == 1   # theta must exceed 1

@@ -18,6 +18,7 @@
 #include "common.cuh"
 #include "pool.cuh"
 #include "ptx.cuh"
+#include "rope.cuh"
 #include "select.cuh"
 
 namespace sbsa {
@@ -141,6 +142,30 @@ sbsa_status launch_pool(const sbsa_shape* s, const void* q, const void* k, float
     }
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? SBSA_OK : cuda_fail(e, "pool launch");
+}
+
+sbsa_status launch_rope_pool(const sbsa_shape* s, int gt, int gh, int gw, const float2* table, const void* q,
+                             const void* k, void* qo, void* ko, float* qm, float* km, cudaStream_t st) {
+    const long long units = num_rows(s);
+    const dim3 grid(static_cast<unsigned>(2 * units));
+    const int L = s->seq_len, Lp = s->seq_len_padded, nb = num_blocks(s);
+    auto q4 = static_cast<const uint4*>(q);
+    auto k4 = static_cast<const uint4*>(k);
+    auto qo4 = static_cast<uint4*>(qo);
+    auto ko4 = static_cast<uint4*>(ko);
+    if (s->head_dim == 128) {
+        if (s->block_size == 128)
+            rope_pool_kernel<128, 128><<<grid, 256, 0, st>>>(q4, k4, qo4, ko4, table, qm, km, L, Lp, nb, gh, gw, gt, units);
+        else
+            rope_pool_kernel<128, 64><<<grid, 256, 0, st>>>(q4, k4, qo4, ko4, table, qm, km, L, Lp, nb, gh, gw, gt, units);
+    } else {
+        if (s->block_size == 128)
+            rope_pool_kernel<64, 128><<<grid, 256, 0, st>>>(q4, k4, qo4, ko4, table, qm, km, L, Lp, nb, gh, gw, gt, units);
+        else
+            rope_pool_kernel<64, 64><<<grid, 256, 0, st>>>(q4, k4, qo4, ko4, table, qm, km, L, Lp, nb, gh, gw, gt, units);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SBSA_OK : cuda_fail(e, "rope+pool launch");
 }
 
 template <int D, int KPL>
@@ -325,7 +350,7 @@ using namespace sbsa;
 
 extern "C" {
 
-int32_t sbsa_version(void) { return 100; }
+int32_t sbsa_version(void) { return 200; }
 
 const char* sbsa_status_string(sbsa_status st) {
     switch (st) {
@@ -363,6 +388,44 @@ sbsa_status sbsa_pool_qk(const sbsa_shape* shape, const void* q, const void* k, 
     if (!aligned16(q) || !aligned16(k) || !aligned16(q_mean) || !aligned16(k_mean))
         return fail(SBSA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
     if ((r = launch_pool(shape, q, k, q_mean, k_mean, static_cast<cudaStream_t>(stream))) != SBSA_OK) return r;
+    return ok();
+}
+
+size_t sbsa_rope_table_floats(int32_t head_dim, int32_t grid_t, int32_t grid_h, int32_t grid_w) {
+    if ((head_dim != 64 && head_dim != 128) || grid_t < 1 || grid_h < 1 || grid_w < 1) return 0;
+    return static_cast<size_t>(2 * rope_table_entries(head_dim, grid_t, grid_h, grid_w));
+}
+
+sbsa_status sbsa_rope_table_init(int32_t head_dim, int32_t grid_t, int32_t grid_h, int32_t grid_w, double theta,
+                                 float* table, void* stream) {
+    if (sbsa_rope_table_floats(head_dim, grid_t, grid_h, grid_w) == 0)
+        return fail(SBSA_ERR_INVALID_ARG, "head_dim must be 64 or 128 and the grid sizes >= 1");
+    if (!(theta > 1.0) || !std::isfinite(theta)) return fail(SBSA_ERR_INVALID_ARG, "theta must be finite and > 1");
+    if (!table || (reinterpret_cast<uintptr_t>(table) & 7u)) return fail(SBSA_ERR_INVALID_ARG, "table must be 8-byte aligned");
+    const long long n = rope_table_entries(head_dim, grid_t, grid_h, grid_w);
+    rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        head_dim, grid_t, grid_h, grid_w, theta, reinterpret_cast<float2*>(table), n);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
+    return ok();
+}
+
+sbsa_status sbsa_rope_pool_qk(const sbsa_shape* shape, int32_t grid_t, int32_t grid_h, int32_t grid_w,
+                              const float* table, const void* q, const void* k, void* q_out, void* k_out,
+                              float* q_mean, float* k_mean, void* stream) {
+    sbsa_status r = check_shape(shape);
+    if (r != SBSA_OK) return r;
+    if (grid_t < 1 || grid_h < 1 || grid_w < 1 ||
+        static_cast<long long>(grid_t) * grid_h * grid_w != static_cast<long long>(shape->seq_len))
+        return fail(SBSA_ERR_INVALID_ARG, "grid_t * grid_h * grid_w must equal seq_len");
+    if (!q || !k || !q_out || !k_out || !q_mean || !k_mean || !table) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out) || !aligned16(q_mean) ||
+        !aligned16(k_mean))
+        return fail(SBSA_ERR_INVALID_ARG, "tensors and means must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(table) & 7u) return fail(SBSA_ERR_INVALID_ARG, "table must be 8-byte aligned");
+    if ((r = launch_rope_pool(shape, grid_t, grid_h, grid_w, reinterpret_cast<const float2*>(table), q, k, q_out,
+                              k_out, q_mean, k_mean, static_cast<cudaStream_t>(stream))) != SBSA_OK)
+        return r;
     return ok();
 }
 

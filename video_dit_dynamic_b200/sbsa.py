@@ -23,7 +23,8 @@ STATUS_NAMES = {0: "SBSA_OK", 1: "SBSA_ERR_INVALID_ARG", 2: "SBSA_ERR_UNSUPPORTE
 # Every symbol include/sbsa.h declares.
 EXPORTS = ("sbsa_version", "sbsa_status_string", "sbsa_last_error_message", "sbsa_keep_blocks",
            "sbsa_workspace_bytes", "sbsa_pool_qk", "sbsa_select_blocks", "sbsa_attention_fwd", "sbsa_forward",
-           "sbsa_check", "sbsa_validate_csr", "sbsa_forward_noalloc")
+           "sbsa_check", "sbsa_validate_csr", "sbsa_forward_noalloc", "sbsa_rope_table_floats",
+           "sbsa_rope_table_init", "sbsa_rope_pool_qk")
 
 
 class SbsaError(RuntimeError):
@@ -84,8 +85,12 @@ def load(path: str | None = None):
     lib.sbsa_forward_noalloc.argtypes = [SP, P, P, P, I32, ctypes.c_float, P, P, P]
     lib.sbsa_check.argtypes = [P]
     lib.sbsa_validate_csr.argtypes = [SP, P, P, ctypes.c_int64, I32, P]
+    lib.sbsa_rope_table_floats.argtypes = [I32, I32, I32, I32]
+    lib.sbsa_rope_table_floats.restype = SZ
+    lib.sbsa_rope_table_init.argtypes = [I32, I32, I32, I32, ctypes.c_double, P, P]
+    lib.sbsa_rope_pool_qk.argtypes = [SP, I32, I32, I32, P, P, P, P, P, P, P, P]
     for name in ("sbsa_pool_qk", "sbsa_select_blocks", "sbsa_attention_fwd", "sbsa_forward", "sbsa_check",
-                 "sbsa_validate_csr", "sbsa_forward_noalloc"):
+                 "sbsa_validate_csr", "sbsa_forward_noalloc", "sbsa_rope_table_init", "sbsa_rope_pool_qk"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -144,6 +149,30 @@ def sbsa_pool_qk(shape: Shape, q, k, q_mean, k_mean, stream=None):
     _raise_on(load().sbsa_pool_qk(ctypes.byref(shape), _dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"),
                                   _dev(q_mean, torch.float32, "q_mean"), _dev(k_mean, torch.float32, "k_mean"),
                                   _stream(stream)))
+
+
+def sbsa_rope_table_floats(head_dim: int, grid) -> int:
+    return int(load().sbsa_rope_table_floats(int(head_dim), int(grid[0]), int(grid[1]), int(grid[2])))
+
+
+def sbsa_rope_table_init(head_dim: int, grid, theta: float, table, stream=None):
+    _check_numel(table, sbsa_rope_table_floats(head_dim, grid), "table")
+    _raise_on(load().sbsa_rope_table_init(int(head_dim), int(grid[0]), int(grid[1]), int(grid[2]), float(theta),
+                                          _dev(table, torch.float32, "table"), _stream(stream)))
+
+
+def sbsa_rope_pool_qk(shape: Shape, grid, table, q, k, q_out, k_out, q_mean, k_mean, stream=None):
+    n_in = shape.batch * shape.heads * shape.seq_len_padded * shape.head_dim
+    n_out = shape.batch * shape.heads * shape.num_blocks * shape.head_dim
+    for t, nm, n in ((q, "q", n_in), (k, "k", n_in), (q_out, "q_out", n_in), (k_out, "k_out", n_in),
+                     (q_mean, "q_mean", n_out), (k_mean, "k_mean", n_out)):
+        _check_numel(t, n, nm)
+    _check_numel(table, sbsa_rope_table_floats(shape.head_dim, grid), "table")
+    _raise_on(load().sbsa_rope_pool_qk(ctypes.byref(shape), int(grid[0]), int(grid[1]), int(grid[2]),
+                                       _dev(table, torch.float32, "table"), _dev(q, torch.bfloat16, "q"),
+                                       _dev(k, torch.bfloat16, "k"), _dev(q_out, torch.bfloat16, "q_out"),
+                                       _dev(k_out, torch.bfloat16, "k_out"), _dev(q_mean, torch.float32, "q_mean"),
+                                       _dev(k_mean, torch.float32, "k_mean"), _stream(stream)))
 
 
 def sbsa_select_blocks(shape: Shape, q_mean, k_mean, k_keep: int, row_ptr, col_idx, stream=None):
