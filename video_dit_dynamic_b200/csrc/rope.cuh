@@ -15,13 +15,15 @@
 // cos/sin come from a table built once per grid (rope_table_kernel, in double).
 // Padded tokens (t >= L) have no grid position; they are passed through unrotated.
 //
-// HBM-bound: one CTA per (tensor, b, h, block), 256 threads; thread t owns the 16-byte
-// chunk t % (d/8) (four rotation pairs) of rows t / (d/8), t / (d/8) + 256/(d/8), ...,
-// issues all of its loads before the first use, rotates in fp32, rounds to bf16 (ties
-// to even), stores, and sums the rounded values of the valid rows for the mean.
+// HBM-bound: one CTA per (tensor, b, h, block), 256 threads.  The block's tile comes in
+// and goes out with one bulk copy each; thread t owns the 16-byte chunk t % (d/8)
+// (four rotation pairs) of rows t / (d/8), t / (d/8) + 256/(d/8), ..., rotates it in
+// fp32, rounds to bf16 (ties to even) in place, and sums the rounded values of the
+// valid rows for the mean.
 #pragma once
 #include "common.cuh"
 #include "pool.cuh"
+#include "ptx.cuh"
 
 namespace sbsa {
 
@@ -63,25 +65,42 @@ __global__ void rope_table_kernel(int d, int gt, int gh, int gw, double theta, f
     table[e] = make_float2(static_cast<float>(c), static_cast<float>(s));
 }
 
-__device__ __forceinline__ void st_global_v4(void* p, const uint4& v) {
-    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+__device__ __forceinline__ void bulk_load_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
 }
+__device__ __forceinline__ void bulk_store_s2g(void* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
+                 "r"(bytes)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_store_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
 
-// in and out may be the same tensor (each 16-byte chunk is read, then written, by one
-// thread), so they carry no __restrict__.
+// The block's BLK x d bf16 tile is contiguous in memory: one bulk copy brings it into
+// shared memory, the threads rotate it in place, and one bulk copy writes it back, so
+// no register holds data in flight and many CTAs share an SM.  in and out may be the
+// same tensor (each tile is read completely before it is written), so they carry no
+// __restrict__.
 template <int D, int BLK>
 __global__ void __launch_bounds__(256) rope_pool_kernel(const uint4* q_in, const uint4* k_in, uint4* q_out,
                                                         uint4* k_out, const float2* __restrict__ table,
                                                         float* __restrict__ q_mean, float* __restrict__ k_mean,
                                                         int L, int Lp, int nb, int gh, int gw, int gt,
-                                                        long long units_per_tensor) {
+                                                        long long units_per_tensor, unsigned int epoch) {
     using S = RopeSplit<D>;
     constexpr int CH = D / 8;          // 16-byte chunks (four pairs each) per row
     constexpr int RG = 256 / CH;       // row groups
     constexpr int ITER = BLK / RG;     // rows per thread
+    constexpr uint32_t kTileBytes = BLK * D * 2;
     static_assert(BLK % RG == 0, "block must be a multiple of the row-group count");
+    __shared__ __align__(128) uint4 tile[BLK * CH];
     __shared__ float red[8][D];
+    __shared__ __align__(8) uint64_t full;
 
     long long u = blockIdx.x;
     const bool is_k = u >= units_per_tensor;
@@ -90,16 +109,16 @@ __global__ void __launch_bounds__(256) rope_pool_kernel(const uint4* q_in, const
     const int i = static_cast<int>(u % nb);
     const int t0 = i * BLK;
     const int nvalid = min(BLK, L - t0);
-
     const long long base = (static_cast<long long>(bh) * Lp + t0) * CH;
-    const uint4* src = (is_k ? k_in : q_in) + base;
-    uint4* dst = (is_k ? k_out : q_out) + base;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&full, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(&full, kTileBytes);
+        bulk_load_g2s(tile, (is_k ? k_in : q_in) + base, kTileBytes, &full);
+    }
     const int c = threadIdx.x % CH;
     const int g = threadIdx.x / CH;
-
-    uint4 w[ITER];
-#pragma unroll
-    for (int it = 0; it < ITER; ++it) w[it] = ld_stream_v4(src + static_cast<long long>(g + it * RG) * CH + c);
 
     // the four pairs of this chunk: their axis (0 frame, 1 row, 2 column), the table
     // entry of position 0 and the entries per position step
@@ -121,18 +140,28 @@ __global__ void __launch_bounds__(256) rope_pool_kernel(const uint4* q_in, const
             step[j] = S::kW;
         }
     }
-
     // grid position of this thread's first row, then stepped by RG rows (t < L only:
     // padded tokens have no grid position and pass through unrotated)
     const int tf = t0 + g;
     int pf = tf / (gh * gw), ph = (tf / gw) % gh, pw = tf % gw;
+
+    __syncthreads();  // the barrier is initialised before anyone waits on it
+    volatile int never = 0;
+    if (!mbar_wait_bounded(&full, 0, &never, kWaitLimitNs)) {
+        if (threadIdx.x == 0) abort_launch(epoch);
+        // give the copy one more bounded wait to land before the shared memory is released
+        mbar_wait_bounded(&full, 0, &never, kWaitLimitNs);
+        return;
+    }
 
     float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
     for (int it = 0; it < ITER; ++it) {
         const int r = g + it * RG;
         const bool valid = r < nvalid;
-        const uint32_t in[4] = {w[it].x, w[it].y, w[it].z, w[it].w};
+        uint4& cell = tile[r * CH + c];
+        const uint4 w = cell;
+        const uint32_t in[4] = {w.x, w.y, w.z, w.w};
         uint32_t out[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -143,8 +172,9 @@ __global__ void __launch_bounds__(256) rope_pool_kernel(const uint4* q_in, const
             const float x = __uint_as_float(in[j] << 16), y = __uint_as_float(in[j] & 0xFFFF0000u);
             out[j] = pack_bf16x2(x * cs.x - y * cs.y, x * cs.y + y * cs.x);
         }
-        st_global_v4(dst + static_cast<long long>(r) * CH + c, make_uint4(out[0], out[1], out[2], out[3]));
-        if (valid) acc_bf16x8(a, make_uint4(out[0], out[1], out[2], out[3]));
+        const uint4 o = make_uint4(out[0], out[1], out[2], out[3]);
+        cell = o;
+        if (valid) acc_bf16x8(a, o);
         // advance the grid position by RG tokens
         pw += RG;
         while (pw >= gw) {
@@ -155,6 +185,9 @@ __global__ void __launch_bounds__(256) rope_pool_kernel(const uint4* q_in, const
             }
         }
     }
+    fence_proxy_async_smem();  // the rotated tile is read by the async proxy next
+    __syncthreads();
+    if (threadIdx.x == 0) bulk_store_s2g((is_k ? k_out : q_out) + base, tile, kTileBytes);
 
     // lanes that share a column chunk: lane ^ CH, lane ^ 2CH, ... within the warp
 #pragma unroll
@@ -175,6 +208,8 @@ __global__ void __launch_bounds__(256) rope_pool_kernel(const uint4* q_in, const
         float* m = (is_k ? k_mean : q_mean) + u * D;
         m[threadIdx.x] = s / static_cast<float>(nvalid);
     }
+    // the tile must stay in shared memory until the bulk store has read it
+    if (threadIdx.x == 0) bulk_store_wait_read();
 }
 
 }  // namespace sbsa

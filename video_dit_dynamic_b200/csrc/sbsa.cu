@@ -149,20 +149,21 @@ sbsa_status launch_rope_pool(const sbsa_shape* s, int gt, int gh, int gw, const 
     const long long units = num_rows(s);
     const dim3 grid(static_cast<unsigned>(2 * units));
     const int L = s->seq_len, Lp = s->seq_len_padded, nb = num_blocks(s);
+    const unsigned int epoch = g_epoch.fetch_add(1);
     auto q4 = static_cast<const uint4*>(q);
     auto k4 = static_cast<const uint4*>(k);
     auto qo4 = static_cast<uint4*>(qo);
     auto ko4 = static_cast<uint4*>(ko);
     if (s->head_dim == 128) {
         if (s->block_size == 128)
-            rope_pool_kernel<128, 128><<<grid, 256, 0, st>>>(q4, k4, qo4, ko4, table, qm, km, L, Lp, nb, gh, gw, gt, units);
+            rope_pool_kernel<128, 128><<<grid, 256, 0, st>>>(q4, k4, qo4, ko4, table, qm, km, L, Lp, nb, gh, gw, gt, units, epoch);
         else
-            rope_pool_kernel<128, 64><<<grid, 256, 0, st>>>(q4, k4, qo4, ko4, table, qm, km, L, Lp, nb, gh, gw, gt, units);
+            rope_pool_kernel<128, 64><<<grid, 256, 0, st>>>(q4, k4, qo4, ko4, table, qm, km, L, Lp, nb, gh, gw, gt, units, epoch);
     } else {
         if (s->block_size == 128)
-            rope_pool_kernel<64, 128><<<grid, 256, 0, st>>>(q4, k4, qo4, ko4, table, qm, km, L, Lp, nb, gh, gw, gt, units);
+            rope_pool_kernel<64, 128><<<grid, 256, 0, st>>>(q4, k4, qo4, ko4, table, qm, km, L, Lp, nb, gh, gw, gt, units, epoch);
         else
-            rope_pool_kernel<64, 64><<<grid, 256, 0, st>>>(q4, k4, qo4, ko4, table, qm, km, L, Lp, nb, gh, gw, gt, units);
+            rope_pool_kernel<64, 64><<<grid, 256, 0, st>>>(q4, k4, qo4, ko4, table, qm, km, L, Lp, nb, gh, gw, gt, units, epoch);
     }
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? SBSA_OK : cuda_fail(e, "rope+pool launch");
