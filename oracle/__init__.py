@@ -56,6 +56,12 @@ def _load():
         lib.oracle_attention.restype = I
         lib.oracle_rope.argtypes = [I, I, I, I, I, I, I, ctypes.c_double, P, I, P]
         lib.oracle_rope.restype = None
+        lib.oracle_e4m3_decode.argtypes = [I]
+        lib.oracle_e4m3_decode.restype = ctypes.c_double
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_encode.restype = I
+        lib.oracle_quantize_fp8.argtypes = [I, I, I, I, I, I, P, I, P, P, P]
+        lib.oracle_quantize_fp8.restype = None
         lib.oracle_set_threads.argtypes = [I]
         lib.oracle_threads_used.restype = I
         _lib = lib
@@ -134,6 +140,51 @@ def rope_pool(x, grid: tuple[int, int, int], L: int, blk: int, theta: float = 10
     rot = rope(x, grid, theta)
     bits = bf16_round(rot)
     return bits, pool(bits, L, blk)
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """e4m3 codes (uint8) -> values (fp64)."""
+    lib = _load()
+    table = np.array([lib.oracle_e4m3_decode(c) for c in range(256)], dtype=np.float64)
+    return table[np.asarray(codes, dtype=np.uint8)]
+
+
+def e4m3_encode(x: float) -> int:
+    """One fp32 value -> e4m3 code (nearest, ties to even, saturating at +-448)."""
+    return int(_load().oracle_e4m3_encode(float(np.float32(x))))
+
+
+def quantize_fp8(x, L: int, blk: int, smooth=None):
+    """Per-block FP8 codes [B,H,Lp,d] (uint8) and scales [B,H,nb] (fp32) of x, after
+    subtracting smooth [B,H,d] (fp32, optional) from every valid token."""
+    a, dt = _as_input(x)
+    B, H, Lp, d = a.shape
+    nb = Lp // blk
+    codes = np.empty((B, H, Lp, d), dtype=np.uint8)
+    scales = np.empty((B, H, nb), dtype=np.float32)
+    sm = None if smooth is None else np.ascontiguousarray(smooth, dtype=np.float32).reshape(B * H, d)
+    _load().oracle_quantize_fp8(B, H, L, Lp, d, blk, _ptr(a), dt, _ptr(sm) if sm is not None else None,
+                                _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def dequantize_fp8(codes: np.ndarray, scales: np.ndarray, blk: int) -> np.ndarray:
+    """codes [B,H,Lp,d] * their block's scale -> fp64."""
+    B, H, Lp, d = codes.shape
+    s = np.repeat(scales.astype(np.float64), blk, axis=2)[:, :, :Lp, None]
+    return e4m3_decode(codes) * s
+
+
+def attention_fp8(q_codes, q_scales, k_codes, k_scales, v, L: int, blk: int, row_ptr, col_idx,
+                  scale: float = 0.0, units=None) -> np.ndarray:
+    """The FP8 path: softmax attention over the kept blocks with Q and K dequantized from
+    their codes and block scales (K as quantized, i.e. already smoothed), V as given."""
+    qd = dequantize_fp8(q_codes, q_scales, blk)
+    kd = dequantize_fp8(k_codes, k_scales, blk)
+    va, dt = _as_input(v)
+    vd = va.astype(np.float64) if dt == F64 or dt == F32 else \
+        (va.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return attention(qd, kd, vd, L, blk, row_ptr, col_idx, scale, units)
 
 
 def score_row(qmean_bh: np.ndarray, kmean_bh: np.ndarray, i: int):

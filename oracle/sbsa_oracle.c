@@ -33,6 +33,17 @@
  *              index of the token on the (T, H, W) latent grid (row-major); pair q of an
  *              axis with P pairs turns by angle pos * theta^(-q/P), theta = 10000.
  *
+ *   fp8     (next step: the FP8 path of [Card], same bullet, and [Guide] item 3: the
+ *              sparse mask feeds an FP8 attention in the style of SageAttention2).  The
+ *              pages give no quantization detail; the reading taken here: K is first
+ *              smoothed by subtracting a per-(b,h) channel vector (the sequence mean of
+ *              K), which leaves softmax unchanged; then every block of Q and of K gets
+ *              one scale, amax/448 over its valid tokens, and its values become e4m3
+ *              codes (round to nearest even, saturating at +-448).  The code decision is
+ *              taken in fp32 arithmetic, the same operations the GPU performs, so codes
+ *              and scales match bit for bit.  Attention then runs on the dequantized
+ *              Q and K (code value * block scale) with V as given.
+ *
  * Inputs are read as fp32, bf16 (raw 16-bit patterns, converted exactly) or fp64.
  * Tensors are row-major [B][H][Lp][d]; means are [B][H][nb][d]; col_idx is
  * [B][H][nb][k].  Padded tokens t >= L are ignored as keys and their query rows
@@ -121,6 +132,71 @@ void oracle_rope(int B, int H, int Lp, int d, int gt, int gh, int gw, double the
             out[(size_t)r * d + 2 * p] = a * c - b * sn;
             out[(size_t)r * d + 2 * p + 1] = a * sn + b * c;
         }
+    }
+}
+
+/* e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no infinities; the
+ * largest finite value is 448) -> value.  Code 0x7F / 0xFF (NaN) decode to NaN. */
+double oracle_e4m3_decode(int code) {
+    int sgn = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);                 /* subnormal: m/8 * 2^-6 */
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+/* float -> e4m3 code, round to nearest (ties to even), saturating at +-448. */
+int oracle_e4m3_encode(float x) {
+    int sgn = signbit(x) ? 1 : 0;
+    double a = fabs((double)x);
+    if (a >= 448.0) return (sgn << 7) | 0x7E;
+    /* quantum: 2^(E-3) for a normal value in [2^E, 2^(E+1)), 2^-9 below 2^-6 */
+    int E = a > 0.0 ? (int)floor(log2(a)) : -7;
+    if (E < -6) E = -6;
+    double quantum = ldexp(1.0, E - 3);
+    double n = nearbyint(a / quantum);                   /* ties to even (default mode) */
+    double r = n * quantum;
+    if (r > 448.0) r = 448.0;
+    /* encode r */
+    if (r < ldexp(1.0, -6)) return (sgn << 7) | (int)(r / ldexp(1.0, -9));
+    int e = (int)floor(log2(r));
+    int m = (int)((r / ldexp(1.0, e) - 1.0) * 8.0);
+    return (sgn << 7) | ((e + 7) << 3) | m;
+}
+
+/* FP8 quantization of one tensor [B][H][Lp][d] per block of blk tokens.  smooth is
+ * [B*H][d] fp32 (or NULL): y = x - smooth[bh] in fp32 for valid tokens, 0 for padded
+ * ones; amax = max |y| over the block; inv = 448 / amax and scale = amax / 448 in fp32
+ * (inv = scale = 1 for an all-zero block); code = e4m3(y * inv) in fp32.  codes has
+ * the input's shape; scales is [B*H*nb] fp32. */
+void oracle_quantize_fp8(int B, int H, int L, int Lp, int d, int blk, const void *x, int dtype,
+                         const float *smooth, uint8_t *codes, float *scales) {
+    int nb = Lp / blk;
+    long units = (long)B * H * nb;
+#pragma omp parallel for schedule(static) num_threads(oracle_threads_used())
+    for (long u = 0; u < units; ++u) {
+        long bh = u / nb;
+        int t0 = (int)(u % nb) * blk;
+        float amax = 0.0f;
+        for (int t = t0; t < t0 + blk && t < L; ++t)
+            for (int c = 0; c < d; ++c) {
+                float y = (float)elem(x, dtype, ((size_t)bh * Lp + t) * d + c) - (smooth ? smooth[bh * d + c] : 0.0f);
+                float ay = fabsf(y);
+                if (ay > amax) amax = ay;
+            }
+        float inv = amax > 0.0f ? 448.0f / amax : 1.0f;
+        scales[u] = amax > 0.0f ? amax / 448.0f : 1.0f;
+        for (int t = t0; t < t0 + blk; ++t)
+            for (int c = 0; c < d; ++c) {
+                size_t i = ((size_t)bh * Lp + t) * d + c;
+                if (t >= L) {
+                    codes[i] = 0;
+                    continue;
+                }
+                float y = (float)elem(x, dtype, i) - (smooth ? smooth[bh * d + c] : 0.0f);
+                codes[i] = (uint8_t)oracle_e4m3_encode(y * inv);
+            }
     }
 }
 

@@ -49,6 +49,12 @@ MUTANTS = {
     "rope_freq_off_by_one": ("pow(theta, -(double)q / (double)np)", "pow(theta, -(double)(q + 1) / (double)np)"),
     # RoPE row index taken with the wrong divisor
     "rope_row_position": ("(t / gw) % gh, t % gw}", "(t / gh) % gw, t % gw}"),
+    # large values mapped to the NaN pattern instead of saturating at 448
+    "fp8_no_saturation": ("if (a >= 448.0) return (sgn << 7) | 0x7E;", "if (a >= 480.0) return (sgn << 7) | 0x7F;"),
+    # e4m3 rounding half away from zero instead of to even
+    "fp8_round_half_up": ("double n = nearbyint(a / quantum);", "double n = floor(a / quantum + 0.5);"),
+    # padded tokens counted in the block's amax
+    "fp8_amax_counts_padding": ("for (int t = t0; t < t0 + blk && t < L; ++t)", "for (int t = t0; t < t0 + blk; ++t)"),
 }
 
 

@@ -415,3 +415,83 @@ def test_bf16_rounding_ties_to_even():
     # 1 + 2^-8 is halfway between bf16 1.0 and 1.0078125: to even (1.0); 1 + 3*2^-9 up
     vals = np.array([1.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -9, 1.0 + 3 * 2.0 ** -8, -2.5, 0.0])
     assert [int(b) for b in oracle.bf16_round(vals)] == [0x3F80, 0x3F80, 0x3F81, 0x3F82, 0xC020, 0x0000]
+
+
+# ---------------------------------------------------------------- FP8 path
+# FP8 attention in the style of SageAttention2 (page "知识卡片…", 方法/产品要点, bullet
+# 动态稀疏量化注意力; page "单卡 RTX 5090 跑 Wan2.2-A14B…", 四步拆解 item 3).  The reading
+# (smoothed K, one scale per block, e4m3 codes) is stated in sbsa_oracle.c.
+
+def test_e4m3_hand_values():
+    # e4m3: bias 7, 3 mantissa bits, largest 448 = 1.75 * 2^8, smallest 2^-9
+    cases = {448.0: 0x7E, 1.0: 0x38, 0.5: 0x30, 240.0: 0x77, 2.0 ** -6: 0x08, 7 * 2.0 ** -9: 0x07,
+             2.0 ** -9: 0x01, -448.0: 0xFE, 0.0: 0x00,
+             # halfway cases go to the even mantissa
+             1.0625: 0x38, 1.1875: 0x3A, 1.9375: 0x40, 1.5 * 2.0 ** -9: 0x02,
+             # beyond the largest finite value: saturate
+             500.0: 0x7E, -1e6: 0xFE}
+    for v, code in cases.items():
+        assert oracle.e4m3_encode(v) == code, (v, hex(oracle.e4m3_encode(v)), hex(code))
+
+
+def test_e4m3_codes_round_trip():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)  # 0x7F/0xFF: NaN
+    vals = oracle.e4m3_decode(codes)
+    assert vals.max() == 448.0 and vals.min() == -448.0
+    back = np.array([oracle.e4m3_encode(v) for v in vals])
+    # +0 and -0 both decode to a zero; everything else comes back to its own code
+    nz = codes != 0x80
+    np.testing.assert_array_equal(back[nz], codes[nz])
+    # the grid: 8 values per binade from 2^-6 on, 2^-9 steps below it
+    pos = np.sort(vals[vals > 0])
+    assert pos[0] == 2.0 ** -9 and np.allclose(np.diff(pos[:8]), 2.0 ** -9)
+
+
+def test_quantize_block_scale_and_error_bound():
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((1, 2, 96, 16)).astype(np.float32)
+    x[0, 1, 40:] *= 1e-3                 # a second block of a different magnitude
+    x[:, :, 90:] = 1000.0                # padded tokens hold junk larger than any valid value
+    codes, scales = oracle.quantize_fp8(x, 90, 32)
+    d = oracle.dequantize_fp8(codes, scales, 32)
+    for h in range(2):
+        for i in range(3):
+            blk = x[0, h, i * 32:min((i + 1) * 32, 90)]
+            amax = np.abs(blk).max()
+            assert scales[0, h, i] == np.float32(amax) / np.float32(448.0)
+            # the largest element lands on +-448 exactly
+            c = codes[0, h, i * 32:min((i + 1) * 32, 90)]
+            assert np.isin(c, [0x7E, 0xFE]).any()
+            # within half a quantum: 2^-4 relative in the normal range, 2^-10 * scale below
+            err = np.abs(d[0, h, i * 32:min((i + 1) * 32, 90)] - blk)
+            assert np.all(err <= np.maximum(np.abs(blk) * 2.0 ** -4, scales[0, h, i] * 2.0 ** -10) * (1 + 1e-6))
+    # padded tokens (t >= 90) are code 0 and do not enter the block's amax
+    assert np.all(codes[:, :, 90:] == 0)
+
+
+def test_smoothing_leaves_attention_unchanged():
+    # subtracting one vector from every key adds a per-query constant to the logits
+    q, k, v = (t.numpy() for t in inputs.random_qkv(1, 2, 64, 16, L=60, seed=32, dtype=torch.float64))
+    mean_k = k[:, :, :60].mean(axis=2, keepdims=True)
+    rp = oracle.uniform_row_ptr(1, 2, 4, 2)
+    col = oracle.select(oracle.pool(q, 60, 16), oracle.pool(k, 60, 16), 2)
+    a = oracle.attention(q, k, v, 60, 16, rp, col)
+    b = oracle.attention(q, k - mean_k, v, 60, 16, rp, col)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_fp8_attention_is_close_to_exact_attention():
+    q, k, v = inputs.random_qkv(1, 2, 128, 64, L=120, seed=33, dtype=torch.bfloat16)
+    qb, kb, vb = (inputs.bf16_bits(t) for t in (q, k, v))
+    kf = (kb.astype(np.uint32) << 16).view(np.float32)
+    smooth = kf[:, :, :120].astype(np.float64).mean(axis=2).astype(np.float32)
+    qc, qs = oracle.quantize_fp8(qb, 120, 32)
+    kc, ks = oracle.quantize_fp8(kb, 120, 32, smooth)
+    rp = oracle.uniform_row_ptr(1, 2, 4, 2)
+    col = oracle.select(oracle.pool(qb, 120, 32), oracle.pool(kb, 120, 32), 2)
+    exact = oracle.attention(qb, kb, vb, 120, 32, rp, col)
+    fp8 = oracle.attention_fp8(qc, qs, kc, ks, vb, 120, 32, rp, col)
+    err = np.abs(fp8 - exact)[:, :, :120]
+    # logits of d = 64 products of ~N(0,1) values with 2^-4 relative errors per factor
+    assert err.max() < 0.1 and err.mean() < 0.01
+    assert err.max() > 0  # and the quantization does something
