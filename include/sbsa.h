@@ -151,6 +151,33 @@ sbsa_status sbsa_select_blocks(const sbsa_shape *shape, const float *q_mean, con
 sbsa_status sbsa_attention_fwd(const sbsa_shape *shape, const void *q, const void *k, const void *v,
                                const int32_t *row_ptr, const int32_t *col_idx, float scale, void *o, void *stream);
 
+/* The FP8 path (pages "知识卡片…", 方法/产品要点, bullet 动态稀疏量化注意力, and "单卡 RTX
+ * 5090 跑 Wan2.2-A14B…", 四步拆解 item 3: the sparse mask feeds an FP8 attention in the
+ * style of SageAttention2).  The pages give no quantization detail; what is built:
+ * K smoothed by its sequence mean (softmax is unchanged by subtracting one vector from
+ * every key), one scale per block of Q and of K, e4m3 codes, S = Q.K^T on e4m3 tensor
+ * cores with fp32 accumulation, and the rest (softmax, P.V in bf16) as in step 3.
+ * head_dim 128 only.
+ *
+ * sbsa_key_mean: out fp32 [B][H][d] (device, written) = sum over blocks of
+ *   (valid tokens of the block) * k_mean[b,h,block,:] / L, i.e. the mean of K over the
+ *   valid tokens, from the block means of sbsa_pool_qk.
+ * sbsa_quantize_qk_fp8: q, k bf16 [B][H][Lp][d]; k_smooth fp32 [B][H][d] or NULL (no
+ *   smoothing); q8, k8 uint8 [B][H][Lp][d] (device, written) e4m3 codes; q_scale,
+ *   k_scale fp32 [B][H][nb] (device, written).  Per block, in fp32: y = x - smooth (K
+ *   only), amax = max |y| over the valid tokens, code = e4m3(y * (448 / amax)) with
+ *   round-to-nearest-even and saturation at +-448, scale = amax / 448 (1 for an all-zero
+ *   block); padded tokens get code 0.  One launch, HBM-bandwidth bound.
+ * sbsa_attention_fwd_fp8: as sbsa_attention_fwd, with q8/k8 and their block scales in
+ *   place of q/k: the logits are scale * (q8 . k8) * q_scale[query block] *
+ *   k_scale[key block].  v and o are bf16 as before. */
+sbsa_status sbsa_key_mean(const sbsa_shape *shape, const float *k_mean, float *out, void *stream);
+sbsa_status sbsa_quantize_qk_fp8(const sbsa_shape *shape, const void *q, const void *k, const float *k_smooth,
+                                 void *q8, void *k8, float *q_scale, float *k_scale, void *stream);
+sbsa_status sbsa_attention_fwd_fp8(const sbsa_shape *shape, const void *q8, const void *k8, const void *v,
+                                   const float *q_scale, const float *k_scale, const int32_t *row_ptr,
+                                   const int32_t *col_idx, float scale, void *o, void *stream);
+
 /* Steps 1-3 in one call on one stream: pool -> select -> attend, with the means and
  * the CSR lists carved out of `workspace` (device, 256-byte aligned, at least
  * sbsa_workspace_bytes(shape, k_keep) bytes).  If col_idx_out is non-NULL the

@@ -91,18 +91,27 @@ __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)
     else tmem_st16(taddr, r);
 }
 
-template <int D, int BLK>
+// FP8: Q and K arrive as e4m3 codes with one scale per block (fp8.cuh) and S = Q K^T
+// runs as kind::f8f6f4 MMAs (K = 32 per instruction, one 128-byte swizzle atom per row
+// at d = 128); the logit of block j is S * |scale| * log2(e) * q_scale * k_scale[j].
+// Everything from P on is the same as the bf16 form.
+template <int D, int BLK, bool FP8 = false>
 struct AttnCfg {
-    static constexpr int kTile = BLK * D * 2;        // bytes of one K or V tile
-    static constexpr int kQBytes = 128 * D * 2;      // bytes of the Q tile
+    static constexpr int kQKBytes = FP8 ? 1 : 2;     // bytes per Q/K element
+    static constexpr int kKTile = BLK * D * kQKBytes;  // bytes of one K tile
+    static constexpr int kVTile = BLK * D * 2;         // bytes of one V tile
+    static constexpr int kQBytes = 128 * D * kQKBytes;  // bytes of the Q tile
+    static constexpr int kQKAtoms = D * kQKBytes / 128;  // 128-byte swizzle atoms per Q/K row
+    static constexpr int kQKElemsPerAtom = 128 / kQKBytes;
+    static constexpr int kQKSteps = D / (FP8 ? 32 : 16);  // MMAs per S = Q K^T
     static constexpr int kPBytes = 128 * BLK * 2;    // bytes of one P block (bf16)
     static constexpr int kSmemBudget = 224 * 1024;   // Q + two P buffers + the K and V rings
-    static constexpr int kStagesRaw = (kSmemBudget - kQBytes - 2 * kPBytes) / (2 * kTile);
+    static constexpr int kStagesRaw = (kSmemBudget - kQBytes - 2 * kPBytes) / (kKTile + kVTile);
     static constexpr int kStages = kStagesRaw > 4 ? 4 : kStagesRaw;  // slots per ring
     static constexpr int kPOff = kQBytes;
     static constexpr int kKOff = kPOff + 2 * kPBytes;
-    static constexpr int kVOff = kKOff + kStages * kTile;
-    static constexpr int kBarOff = kVOff + kStages * kTile;
+    static constexpr int kVOff = kKOff + kStages * kKTile;
+    static constexpr int kBarOff = kVOff + kStages * kVTile;
     // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2],
     // s_free[2], p_full[2], pv_done[2], drain[2]
     static constexpr int kNumBars = 1 + 4 * kStages + 2 * 5;
@@ -114,6 +123,7 @@ struct AttnCfg {
     static_assert(BLK == 64 || BLK == 128, "block_size");
     static_assert(kSmemBytes <= 232448, "shared memory");
     static_assert(2 * 2 * 128 * 4 <= kPBytes, "merge exchange fits in a P buffer");
+    static_assert(!FP8 || D == 128, "the FP8 form needs d = 128 (one 128-byte atom per row)");
 };
 
 struct AttnParams {
@@ -125,19 +135,34 @@ struct AttnParams {
     float scale_log2;  // |scale| * log2(e)
     int neg_scale;     // 1 if scale < 0 (logits are then -|scale| * S)
     unsigned int epoch;
+    const float* q_scale;  // FP8 form: per (b, h, block) scales of the codes
+    const float* k_scale;
 };
+
+// e4m3 x e4m3 -> fp32 instruction descriptor (format 0 = E4M3 for both operands).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+__device__ __forceinline__ void umma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 
 // Synchronise the two softmax warpgroups (warps 0-7) on named barrier 1 (final merge).
 __device__ __forceinline__ void softmax_pair_sync() {
     asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
-template <int D, int BLK>
+template <int D, int BLK, bool FP8 = false>
 __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CUtensorMap map_q,
                                                       const __grid_constant__ CUtensorMap map_k,
                                                       const __grid_constant__ CUtensorMap map_v,
                                                       const AttnParams p) {
-    using C = AttnCfg<D, BLK>;
+    using C = AttnCfg<D, BLK, FP8>;
     constexpr int NS = C::kStages;
     constexpr int HD = D / 2;    // output columns each warpgroup writes in the merge
     extern __shared__ __align__(1024) uint8_t attn_smem_raw[];
@@ -224,8 +249,8 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
             const int row0 = static_cast<int>(bh * p.Lp);
             mbar_arrive_expect_tx(q_full, C::kQBytes);
 #pragma unroll
-            for (int a = 0; a < D / 64; ++a)
-                tma_load_2d(sQ + a * 128 * 128, &map_q, q_full, a * 64, row0 + qb * BLK, pol_q);
+            for (int a = 0; a < C::kQKAtoms; ++a)
+                tma_load_2d(sQ + a * 128 * 128, &map_q, q_full, a * C::kQKElemsPerAtom, row0 + qb * BLK, pol_q);
             int kseq = 0, vseq = 0;
             auto load = [&](int j, bool is_v) -> bool {
                 int& seq = is_v ? vseq : kseq;
@@ -234,12 +259,18 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                 if (!wait(is_v ? &v_empty[slot] : &k_empty[slot], ph ^ 1)) return false;
                 int blk = __ldg(p.col_idx + rs + j);
                 if (blk < 0 || blk >= p.nb) blk = 0;  // masked by the softmax warps
-                uint8_t* dst = (is_v ? sV : sK) + slot * C::kTile;
+                uint8_t* dst = is_v ? sV + slot * C::kVTile : sK + slot * C::kKTile;
                 uint64_t* full = is_v ? &v_full[slot] : &k_full[slot];
-                mbar_arrive_expect_tx(full, C::kTile);
+                mbar_arrive_expect_tx(full, is_v ? C::kVTile : C::kKTile);
+                if (is_v) {
 #pragma unroll
-                for (int a = 0; a < D / 64; ++a)
-                    tma_load_2d(dst + a * BLK * 128, is_v ? &map_v : &map_k, full, a * 64, row0 + blk * BLK, pol_kv);
+                    for (int a = 0; a < D / 64; ++a)
+                        tma_load_2d(dst + a * BLK * 128, &map_v, full, a * 64, row0 + blk * BLK, pol_kv);
+                } else {
+#pragma unroll
+                    for (int a = 0; a < C::kQKAtoms; ++a)
+                        tma_load_2d(dst + a * BLK * 128, &map_k, full, a * C::kQKElemsPerAtom, row0 + blk * BLK, pol_kv);
+                }
                 ++seq;
                 return true;
             };
@@ -262,7 +293,7 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
     } else if (warp == 9) {
         // ------------------------------------------------------------ QK issuer
         if ((tid & 31) == 0 && n > 0) {
-            constexpr uint32_t idS = idesc_bf16_f32(128, BLK, false);
+            constexpr uint32_t idS = FP8 ? idesc_e4m3_f32(128, BLK) : idesc_bf16_f32(128, BLK, false);
             const uint32_t k_addr = smem_u32(sK);
             const uint64_t qdesc0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
             bool ok = wait(q_full, 0);
@@ -272,14 +303,16 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                 if (!(ok = wait(&k_full[slot], (j / NS) & 1))) break;
                 if (j >= 2 && !(ok = wait(&s_free[b], ((j - 2) >> 1) & 1))) break;
                 tc_fence_after();
-                const uint64_t kdesc0 = sdesc_sw128(k_addr + slot * C::kTile, 16, 1024);
+                const uint64_t kdesc0 = sdesc_sw128(k_addr + slot * C::kKTile, 16, 1024);
                 const uint32_t d_s = tmem + C::kColS0 + b * 128;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
+                for (int kk = 0; kk < C::kQKSteps; ++kk) {
                     // only the 14-bit start-address field (bytes / 16) moves between K steps
+                    // (32 bytes per step: 16 bf16 or 32 e4m3 elements)
                     const uint64_t da = qdesc0 + static_cast<uint64_t>(((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4);
                     const uint64_t db = kdesc0 + static_cast<uint64_t>(((kk / 4) * (BLK * 128) + (kk % 4) * 32) >> 4);
-                    umma_ss(d_s, da, db, idS, kk > 0 ? 1u : 0u);
+                    if constexpr (FP8) umma_f8_ss(d_s, da, db, idS, kk > 0 ? 1u : 0u);
+                    else umma_ss(d_s, da, db, idS, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&k_empty[slot]);
                 umma_commit(&s_full[b]);
@@ -303,7 +336,7 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                 if (!(ok = wait(&v_full[slot], (j / NS) & 1))) break;
                 if (!(ok = wait(&p_full[b], (j >> 1) & 1))) break;
                 tc_fence_after();
-                const uint64_t vdesc0 = sdesc_sw128(v_addr + slot * C::kTile, BLK * 128, 1024);
+                const uint64_t vdesc0 = sdesc_sw128(v_addr + slot * C::kVTile, BLK * 128, 1024);
                 const uint64_t pdesc = pdesc0 + static_cast<uint64_t>((b * C::kPBytes) >> 4);
                 const uint32_t d_o = tmem + C::kColO0 + b * 128;
 #pragma unroll
@@ -329,8 +362,9 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
         const int t = qb * BLK + r;
         const bool row_in_block = r < BLK;
         const bool row_valid = row_in_block && t < p.L;
-        const float sl2 = p.scale_log2;  // |scale| * log2(e) > 0
-        const float2 sl2x2 = make_float2(sl2, sl2);
+        // logit scale |scale| * log2(e) > 0; the FP8 form also folds in this query
+        // block's scale here and each key block's scale below
+        const float sl2_q = FP8 ? p.scale_log2 * __ldg(p.q_scale + unit) : p.scale_log2;
         const uint32_t s_col = tmem + lane_base + C::kColS0 + g * 128;
         const uint32_t o_col = tmem + lane_base + C::kColO0 + g * 128;
         // this row of P_g: 128-byte rows, 16-byte chunks swizzled by (row mod 8), one
@@ -348,9 +382,20 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
             return __all_sync(0xFFFFFFFFu, w);
         };
         int blk_next = g < n ? __ldg(p.col_idx + rs + g) : 0;
+        float ks_next = 1.f;
+        if constexpr (FP8) {
+            if (g < n && blk_next >= 0 && blk_next < p.nb) ks_next = __ldg(p.k_scale + bh * p.nb + blk_next);
+        }
         for (int j = g; j < n; j += 2) {
             const int blk = blk_next;
-            if (j + 2 < n) blk_next = __ldg(p.col_idx + rs + j + 2);
+            const float sl2 = sl2_q * ks_next;
+            const float2 sl2x2 = make_float2(sl2, sl2);
+            if (j + 2 < n) {
+                blk_next = __ldg(p.col_idx + rs + j + 2);
+                if constexpr (FP8) {
+                    ks_next = (blk_next >= 0 && blk_next < p.nb) ? __ldg(p.k_scale + bh * p.nb + blk_next) : 1.f;
+                }
+            }
             if (ok) ok = wait_warp(&s_full[g], (j >> 1) & 1);
             if (!ok) continue;
             tc_fence_after();

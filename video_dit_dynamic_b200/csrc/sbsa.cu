@@ -16,6 +16,7 @@
 #include "../../include/sbsa.h"
 #include "attn.cuh"
 #include "common.cuh"
+#include "fp8.cuh"
 #include "pool.cuh"
 #include "ptx.cuh"
 #include "rope.cuh"
@@ -109,6 +110,21 @@ sbsa_status make_map(CUtensorMap* m, const void* base, long long rows, int d, in
     return SBSA_OK;
 }
 
+// e4m3 codes [rows][128] viewed as a 2D tensor, box = 128 channels (128 B) x box_rows
+sbsa_status make_map_codes(CUtensorMap* m, const void* base, long long rows, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(SBSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {128};
+    cuuint32_t box[2] = {128, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SBSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return SBSA_OK;
+}
+
 // fp32 block means [rows][128] viewed as a 2D tensor, box = 32 channels (128 B) x box_rows
 sbsa_status make_map_means(CUtensorMap* m, const float* base, long long rows, int box_rows) {
     EncodeTiledFn enc = encode_fn();
@@ -167,6 +183,24 @@ sbsa_status launch_rope_pool(const sbsa_shape* s, int gt, int gh, int gw, const 
     }
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? SBSA_OK : cuda_fail(e, "rope+pool launch");
+}
+
+sbsa_status launch_quantize(const sbsa_shape* s, const void* q, const void* k, const float* smooth, void* q8,
+                            void* k8, float* qs, float* ks, cudaStream_t st) {
+    const long long units = num_rows(s);
+    const dim3 grid(static_cast<unsigned>(2 * units));
+    const int L = s->seq_len, Lp = s->seq_len_padded, nb = num_blocks(s);
+    const unsigned int epoch = g_epoch.fetch_add(1);
+    auto q4 = static_cast<const uint4*>(q);
+    auto k4 = static_cast<const uint4*>(k);
+    auto q2 = static_cast<uint2*>(q8);
+    auto k2 = static_cast<uint2*>(k8);
+    if (s->block_size == 128)
+        quantize_kernel<128, 128><<<grid, 256, 0, st>>>(q4, k4, smooth, q2, k2, qs, ks, L, Lp, nb, units, epoch);
+    else
+        quantize_kernel<128, 64><<<grid, 256, 0, st>>>(q4, k4, smooth, q2, k2, qs, ks, L, Lp, nb, units, epoch);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SBSA_OK : cuda_fail(e, "quantize launch");
 }
 
 template <int D, int KPL>
@@ -230,15 +264,21 @@ sbsa_status launch_select(const sbsa_shape* s, const float* qm, const float* km,
                               : launch_select_d<64>(s, qm, km, k, rp, ci, st);
 }
 
-template <int D, int BLK>
+template <int D, int BLK, bool FP8 = false>
 sbsa_status launch_attn_t(const sbsa_shape* s, const void* q, const void* k, const void* v, const int32_t* rp,
-                          const int32_t* ci, float scale, void* o, cudaStream_t st) {
-    using C = AttnCfg<D, BLK>;
+                          const int32_t* ci, float scale, void* o, cudaStream_t st, const float* q_scale = nullptr,
+                          const float* k_scale = nullptr) {
+    using C = AttnCfg<D, BLK, FP8>;
     const long long rows = static_cast<long long>(s->batch) * s->heads * s->seq_len_padded;
     CUtensorMap mq, mk, mv;
     sbsa_status r;
-    if ((r = make_map(&mq, q, rows, D, 128)) != SBSA_OK) return r;
-    if ((r = make_map(&mk, k, rows, D, BLK)) != SBSA_OK) return r;
+    if constexpr (FP8) {
+        if ((r = make_map_codes(&mq, q, rows, 128)) != SBSA_OK) return r;
+        if ((r = make_map_codes(&mk, k, rows, BLK)) != SBSA_OK) return r;
+    } else {
+        if ((r = make_map(&mq, q, rows, D, 128)) != SBSA_OK) return r;
+        if ((r = make_map(&mk, k, rows, D, BLK)) != SBSA_OK) return r;
+    }
     if ((r = make_map(&mv, v, rows, D, BLK)) != SBSA_OK) return r;
     AttnParams p;
     p.row_ptr = rp;
@@ -251,7 +291,9 @@ sbsa_status launch_attn_t(const sbsa_shape* s, const void* q, const void* k, con
     p.scale_log2 = std::fabs(scale) * 1.4426950408889634f;
     p.neg_scale = scale < 0.f ? 1 : 0;
     p.epoch = g_epoch.fetch_add(1);
-    auto kern = attn_kernel<D, BLK>;
+    p.q_scale = q_scale;
+    p.k_scale = k_scale;
+    auto kern = attn_kernel<D, BLK, FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "attention smem attribute");
     kern<<<static_cast<unsigned>(p.units), C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
@@ -427,6 +469,58 @@ sbsa_status sbsa_rope_pool_qk(const sbsa_shape* shape, int32_t grid_t, int32_t g
     if ((r = launch_rope_pool(shape, grid_t, grid_h, grid_w, reinterpret_cast<const float2*>(table), q, k, q_out,
                               k_out, q_mean, k_mean, static_cast<cudaStream_t>(stream))) != SBSA_OK)
         return r;
+    return ok();
+}
+
+sbsa_status sbsa_key_mean(const sbsa_shape* shape, const float* k_mean, float* out, void* stream) {
+    sbsa_status r = check_shape(shape);
+    if (r != SBSA_OK) return r;
+    if (!k_mean || !out) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    key_mean_kernel<<<static_cast<unsigned>(static_cast<long long>(shape->batch) * shape->heads), shape->head_dim, 0,
+                      static_cast<cudaStream_t>(stream)>>>(k_mean, out, shape->head_dim, num_blocks(shape),
+                                                            shape->block_size, shape->seq_len);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "key mean launch");
+    return ok();
+}
+
+sbsa_status sbsa_quantize_qk_fp8(const sbsa_shape* shape, const void* q, const void* k, const float* k_smooth,
+                                 void* q8, void* k8, float* q_scale, float* k_scale, void* stream) {
+    sbsa_status r = check_shape(shape);
+    if (r != SBSA_OK) return r;
+    if (shape->head_dim != 128) return fail(SBSA_ERR_UNSUPPORTED, "the FP8 path needs head_dim 128");
+    if (!q || !k || !q8 || !k8 || !q_scale || !k_scale) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(q8) || !aligned16(k8))
+        return fail(SBSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+    if (((reinterpret_cast<uintptr_t>(q_scale) | reinterpret_cast<uintptr_t>(k_scale) |
+          reinterpret_cast<uintptr_t>(k_smooth)) & 3u))
+        return fail(SBSA_ERR_INVALID_ARG, "scales and smoothing vector must be 4-byte aligned");
+    if ((r = launch_quantize(shape, q, k, k_smooth, q8, k8, q_scale, k_scale, static_cast<cudaStream_t>(stream))) !=
+        SBSA_OK)
+        return r;
+    return ok();
+}
+
+sbsa_status sbsa_attention_fwd_fp8(const sbsa_shape* shape, const void* q8, const void* k8, const void* v,
+                                   const float* q_scale, const float* k_scale, const int32_t* row_ptr,
+                                   const int32_t* col_idx, float scale, void* o, void* stream) {
+    sbsa_status r = check_shape(shape);
+    if (r != SBSA_OK) return r;
+    if (shape->head_dim != 128) return fail(SBSA_ERR_UNSUPPORTED, "the FP8 path needs head_dim 128");
+    if (!q8 || !k8 || !v || !o || !q_scale || !k_scale || !row_ptr || !col_idx)
+        return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(q8) || !aligned16(k8) || !aligned16(v) || !aligned16(o))
+        return fail(SBSA_ERR_INVALID_ARG, "q8, k8, v, o must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(row_ptr) | reinterpret_cast<uintptr_t>(col_idx) |
+         reinterpret_cast<uintptr_t>(q_scale) | reinterpret_cast<uintptr_t>(k_scale)) & 3u)
+        return fail(SBSA_ERR_INVALID_ARG, "row_ptr, col_idx and the scales must be 4-byte aligned");
+    if (!std::isfinite(scale)) return fail(SBSA_ERR_INVALID_ARG, "scale must be finite");
+    const float sc = resolve_scale(shape, scale);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    r = shape->block_size == 128
+            ? launch_attn_t<128, 128, true>(shape, q8, k8, v, row_ptr, col_idx, sc, o, st, q_scale, k_scale)
+            : launch_attn_t<128, 64, true>(shape, q8, k8, v, row_ptr, col_idx, sc, o, st, q_scale, k_scale);
+    if (r != SBSA_OK) return r;
     return ok();
 }
 

@@ -24,7 +24,8 @@ STATUS_NAMES = {0: "SBSA_OK", 1: "SBSA_ERR_INVALID_ARG", 2: "SBSA_ERR_UNSUPPORTE
 EXPORTS = ("sbsa_version", "sbsa_status_string", "sbsa_last_error_message", "sbsa_keep_blocks",
            "sbsa_workspace_bytes", "sbsa_pool_qk", "sbsa_select_blocks", "sbsa_attention_fwd", "sbsa_forward",
            "sbsa_check", "sbsa_validate_csr", "sbsa_forward_noalloc", "sbsa_rope_table_floats",
-           "sbsa_rope_table_init", "sbsa_rope_pool_qk")
+           "sbsa_rope_table_init", "sbsa_rope_pool_qk", "sbsa_key_mean", "sbsa_quantize_qk_fp8",
+           "sbsa_attention_fwd_fp8")
 
 
 class SbsaError(RuntimeError):
@@ -89,8 +90,12 @@ def load(path: str | None = None):
     lib.sbsa_rope_table_floats.restype = SZ
     lib.sbsa_rope_table_init.argtypes = [I32, I32, I32, I32, ctypes.c_double, P, P]
     lib.sbsa_rope_pool_qk.argtypes = [SP, I32, I32, I32, P, P, P, P, P, P, P, P]
+    lib.sbsa_key_mean.argtypes = [SP, P, P, P]
+    lib.sbsa_quantize_qk_fp8.argtypes = [SP, P, P, P, P, P, P, P, P]
+    lib.sbsa_attention_fwd_fp8.argtypes = [SP, P, P, P, P, P, P, P, ctypes.c_float, P, P]
     for name in ("sbsa_pool_qk", "sbsa_select_blocks", "sbsa_attention_fwd", "sbsa_forward", "sbsa_check",
-                 "sbsa_validate_csr", "sbsa_forward_noalloc", "sbsa_rope_table_init", "sbsa_rope_pool_qk"):
+                 "sbsa_validate_csr", "sbsa_forward_noalloc", "sbsa_rope_table_init", "sbsa_rope_pool_qk",
+                 "sbsa_key_mean", "sbsa_quantize_qk_fp8", "sbsa_attention_fwd_fp8"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -173,6 +178,48 @@ def sbsa_rope_pool_qk(shape: Shape, grid, table, q, k, q_out, k_out, q_mean, k_m
                                        _dev(k, torch.bfloat16, "k"), _dev(q_out, torch.bfloat16, "q_out"),
                                        _dev(k_out, torch.bfloat16, "k_out"), _dev(q_mean, torch.float32, "q_mean"),
                                        _dev(k_mean, torch.float32, "k_mean"), _stream(stream)))
+
+
+def sbsa_key_mean(shape: Shape, k_mean, out, stream=None):
+    rows = shape.batch * shape.heads
+    _check_numel(k_mean, rows * shape.num_blocks * shape.head_dim, "k_mean")
+    _check_numel(out, rows * shape.head_dim, "out")
+    _raise_on(load().sbsa_key_mean(ctypes.byref(shape), _dev(k_mean, torch.float32, "k_mean"),
+                                   _dev(out, torch.float32, "out"), _stream(stream)))
+
+
+def sbsa_quantize_qk_fp8(shape: Shape, q, k, k_smooth, q8, k8, q_scale, k_scale, stream=None):
+    n_in = shape.batch * shape.heads * shape.seq_len_padded * shape.head_dim
+    rows = shape.batch * shape.heads * shape.num_blocks
+    for t, nm in ((q, "q"), (k, "k"), (q8, "q8"), (k8, "k8")):
+        _check_numel(t, n_in, nm)
+    _check_numel(q_scale, rows, "q_scale")
+    _check_numel(k_scale, rows, "k_scale")
+    sm = None
+    if k_smooth is not None:
+        _check_numel(k_smooth, shape.batch * shape.heads * shape.head_dim, "k_smooth")
+        sm = _dev(k_smooth, torch.float32, "k_smooth")
+    _raise_on(load().sbsa_quantize_qk_fp8(ctypes.byref(shape), _dev(q, torch.bfloat16, "q"),
+                                          _dev(k, torch.bfloat16, "k"), sm, _dev(q8, torch.uint8, "q8"),
+                                          _dev(k8, torch.uint8, "k8"), _dev(q_scale, torch.float32, "q_scale"),
+                                          _dev(k_scale, torch.float32, "k_scale"), _stream(stream)))
+
+
+def sbsa_attention_fwd_fp8(shape: Shape, q8, k8, v, q_scale, k_scale, row_ptr, col_idx, scale: float, o,
+                           stream=None):
+    n_in = shape.batch * shape.heads * shape.seq_len_padded * shape.head_dim
+    rows = shape.batch * shape.heads * shape.num_blocks
+    for t, nm in ((q8, "q8"), (k8, "k8"), (v, "v"), (o, "o")):
+        _check_numel(t, n_in, nm)
+    _check_numel(q_scale, rows, "q_scale")
+    _check_numel(k_scale, rows, "k_scale")
+    _check_numel(row_ptr, rows + 1, "row_ptr")
+    _raise_on(load().sbsa_attention_fwd_fp8(ctypes.byref(shape), _dev(q8, torch.uint8, "q8"),
+                                            _dev(k8, torch.uint8, "k8"), _dev(v, torch.bfloat16, "v"),
+                                            _dev(q_scale, torch.float32, "q_scale"),
+                                            _dev(k_scale, torch.float32, "k_scale"),
+                                            _dev(row_ptr, torch.int32, "row_ptr"), _dev(col_idx, torch.int32, "col_idx"),
+                                            float(scale), _dev(o, torch.bfloat16, "o"), _stream(stream)))
 
 
 def sbsa_select_blocks(shape: Shape, q_mean, k_mean, k_keep: int, row_ptr, col_idx, stream=None):
