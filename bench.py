@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-rope", action="store_true", help="skip timing the fused RoPE + pooling kernel")
+    ap.add_argument("--no-fp8", action="store_true", help="skip timing the FP8 path")
     ap.add_argument("--cpu-units", type=int, default=16, help="attention units in the CPU sample")
     return ap.parse_args()
 
@@ -80,6 +81,25 @@ def max_over_ranks(pg, device, timings: dict) -> dict:
     t = torch.tensor([float(timings[n]) for n in names], dtype=torch.float64, device=device)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return {n: float(x) for n, x in zip(names, t.tolist())}
+
+
+def fp8_summary(fp8: dict, flops: float, pool_select_ms: float, peaks: dict) -> dict:
+    """Figures of the FP8 path.  Its attention does the Q.K^T half of the FLOPs in e4m3 and
+    the P.V half in bf16, so its tensor roofline is the harmonic mix of the fp8 peak
+    (measured bf16 peak x 2, the nominal 4.5 / 2.25 PFLOP/s ratio) and the bf16 peak:
+    flops / (flops/2 / fp8 + flops/2 / bf16) = 4/3 of the bf16 peak."""
+    bf16 = peaks["bf16_tflops"]
+    mixed = flops / (0.5 * flops / (2.0 * bf16) + 0.5 * flops / bf16)
+    att_tflops = flops / (fp8["att_ms"] / 1e3) / 1e12
+    quant_gbs = fp8["quant_bytes"] / (fp8["quant_ms"] / 1e3) / 1e9
+    layer_ms = pool_select_ms + fp8["quant_ms"] + fp8["att_ms"]
+    return {"attention": {"ms": fp8["att_ms"], "TFLOP/s": att_tflops, "mixed_peak": mixed,
+                          "frac": att_tflops / mixed, "kernel": "attn_kernel<128,128,fp8>"},
+            "key_mean_plus_quantize": {"ms": fp8["quant_ms"], "GB/s": quant_gbs,
+                                       "hbm_frac": quant_gbs / peaks["hbm_gbs"],
+                                       "algorithmic_bytes": fp8["quant_bytes"]},
+            "layer_ms": layer_ms, "layer_TFLOP/s": flops / (layer_ms / 1e3) / 1e12,
+            "note": "pool + select + key mean + quantize + fp8 attention, timed apart from the step"}
 
 
 def job_tflops(flops_per_rank: float, world: int, ms: float) -> float:
@@ -383,6 +403,41 @@ def run_gpu(args, wl):
         rope = {"ms": rope_ms, "algorithmic_bytes": rope_bytes}
         del qo, ko, table
 
+    # the FP8 path (key mean -> per-block e4m3 quantization of Q and smoothed K -> the
+    # attention with e4m3 Q.K^T products), timed on its own over the same selection
+    fp8 = None
+    if not args.no_fp8 and wl.head_dim == 128:
+        kbar = torch.empty(wl.batch * wl.heads * wl.head_dim, dtype=torch.float32, device=dev)
+        q8 = torch.empty(q.numel(), dtype=torch.uint8, device=dev)
+        k8 = torch.empty_like(q8)
+        qs = torch.empty(rows, dtype=torch.float32, device=dev)
+        ks = torch.empty_like(qs)
+        o8 = torch.empty_like(q)
+
+        def fp8_step(fe=None):
+            if fe: fe[0].record(stream)
+            sbsa.sbsa_key_mean(shape, km, kbar, stream=stream)
+            sbsa.sbsa_quantize_qk_fp8(shape, q, kt, kbar, q8, k8, qs, ks, stream=stream)
+            if fe: fe[1].record(stream)
+            sbsa.sbsa_attention_fwd_fp8(shape, q8, k8, v, qs, ks, rp, ci, 0.0, o8, stream=stream)
+            if fe: fe[2].record(stream)
+
+        sbsa.sbsa_pool_qk(shape, q, kt, qm, km, stream=stream)
+        sbsa.sbsa_select_blocks(shape, qm, km, k, rp, ci, stream=stream)
+        for _ in range(3):
+            fp8_step()
+        n_fp8 = max(3, min(args.steps, 10))
+        fes = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_fp8)]
+        for i in range(n_fp8):
+            fp8_step(fes[i])
+        torch.cuda.synchronize(dev)
+        sbsa.sbsa_check(stream)
+        fp8 = {"quant_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in fes),
+               "att_ms": statistics.mean(e[1].elapsed_time(e[2]) for e in fes),
+               # bf16 Q and K read, their codes written, the block means read for the key mean
+               "quant_bytes": 2 * q.numel() * 2 + 2 * q.numel() + 2 * rows * 4 + km.numel() * 4}
+        del kbar, q8, k8, qs, ks, o8
+
     # end to end through the public API from pinned host buffers
     e2e = None
     if not args.no_e2e:
@@ -407,12 +462,16 @@ def run_gpu(args, wl):
     t = max_over_ranks(pg, dev, {"elapsed": elapsed_ms, "att": statistics.mean(att_ms),
                                  "pool": statistics.mean(pool_ms), "sel": statistics.mean(sel_ms),
                                  "forward": forward_ms, "e2e": e2e["ms"] if e2e is not None else 0.0,
-                                 "rope": rope["ms"] if rope is not None else 0.0})
+                                 "rope": rope["ms"] if rope is not None else 0.0,
+                                 "fp8_quant": fp8["quant_ms"] if fp8 is not None else 0.0,
+                                 "fp8_att": fp8["att_ms"] if fp8 is not None else 0.0})
     elapsed_ms, att_avg, pool_avg, sel_avg, forward_ms = (t[n] for n in ("elapsed", "att", "pool", "sel", "forward"))
     if e2e is not None:
         e2e["ms"] = t["e2e"]
     if rope is not None:
         rope["ms"] = t["rope"]
+    if fp8 is not None:
+        fp8["quant_ms"], fp8["att_ms"] = t["fp8_quant"], t["fp8_att"]
     ms_step = elapsed_ms / args.steps
     value = job_tflops(flops, ws_n, ms_step)
 
@@ -448,6 +507,7 @@ def run_gpu(args, wl):
                                   "algorithmic_bytes": rope["algorithmic_bytes"],
                                   "note": "3D RoPE fused with pooling, timed alone (not part of the step)"}}
                    if rope is not None else {}),
+                **({"fp8": fp8_summary(fp8, flops, pool_avg + sel_avg, peaks)} if fp8 is not None else {}),
             },
             "peaks": {"source": peak_src, **peaks},
         }
