@@ -62,6 +62,16 @@ def _load():
         lib.oracle_e4m3_encode.restype = I
         lib.oracle_quantize_fp8.argtypes = [I, I, I, I, I, I, P, I, P, P, P]
         lib.oracle_quantize_fp8.restype = None
+        lib.oracle_e2m1_decode.argtypes = [I]
+        lib.oracle_e2m1_decode.restype = ctypes.c_double
+        lib.oracle_e2m1_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e2m1_encode.restype = I
+        lib.oracle_nvfp4_sf_offset.argtypes = [I, I, I]
+        lib.oracle_nvfp4_sf_offset.restype = ctypes.c_size_t
+        lib.oracle_nvfp4_quantize.argtypes = [I, I, P, I, P, P]
+        lib.oracle_nvfp4_quantize.restype = ctypes.c_float
+        lib.oracle_nvfp4_dequantize.argtypes = [I, I, P, P, ctypes.c_float, P]
+        lib.oracle_nvfp4_dequantize.restype = None
         lib.oracle_set_threads.argtypes = [I]
         lib.oracle_threads_used.restype = I
         _lib = lib
@@ -185,6 +195,57 @@ def attention_fp8(q_codes, q_scales, k_codes, k_scales, v, L: int, blk: int, row
     vd = va.astype(np.float64) if dt == F64 or dt == F32 else \
         (va.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     return attention(qd, kd, vd, L, blk, row_ptr, col_idx, scale, units)
+
+
+def e2m1_decode(codes: np.ndarray) -> np.ndarray:
+    """e2m1 codes (low 4 bits of each entry) -> values (fp64)."""
+    lib = _load()
+    table = np.array([lib.oracle_e2m1_decode(c) for c in range(16)], dtype=np.float64)
+    return table[np.asarray(codes) & 15]
+
+
+def e2m1_encode(x: float) -> int:
+    """One fp32 value -> e2m1 code (nearest, ties to the even code, saturating at +-6)."""
+    return int(_load().oracle_e2m1_encode(float(np.float32(x))))
+
+
+def nvfp4_sf_offset(r: int, kb: int, K: int) -> int:
+    """Byte offset of the scale of (row r, 16-element block kb) in a K-column scale array."""
+    return int(_load().oracle_nvfp4_sf_offset(r, kb, K))
+
+
+def nvfp4_sf_bytes(rows: int, K: int) -> int:
+    return (rows + 127) // 128 * 128 * (K // 16)
+
+
+def nvfp4_quantize(x):
+    """[rows, K] (bf16 bits, fp32 or fp64) -> (codes uint8 [rows, K/2], sf uint8, tensor scale s)."""
+    a, dt = _as_input(x)
+    rows, K = a.shape
+    if K % 64:
+        raise ValueError("K must be a multiple of 64")
+    codes = np.empty((rows, K // 2), dtype=np.uint8)
+    sf = np.empty(nvfp4_sf_bytes(rows, K), dtype=np.uint8)
+    s = _load().oracle_nvfp4_quantize(rows, K, _ptr(a), dt, _ptr(codes), _ptr(sf))
+    return codes, sf, float(np.float32(s))
+
+
+def nvfp4_dequantize(codes: np.ndarray, sf: np.ndarray, s: float) -> np.ndarray:
+    """codes [rows, K/2] + scales + tensor scale -> fp64 [rows, K]."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    rows, K = codes.shape[0], codes.shape[1] * 2
+    out = np.empty((rows, K), dtype=np.float64)
+    _load().oracle_nvfp4_dequantize(rows, K, _ptr(codes), _ptr(sf), ctypes.c_float(s), _ptr(out))
+    return out
+
+
+def nvfp4_gemm(a_codes, a_sf, a_s, b_codes, b_sf, b_s, bias=None) -> np.ndarray:
+    """C[M, N] = A_dec @ B_dec^T + bias[N] in fp64, A [M, K] and B [N, K] in NVFP4."""
+    c = nvfp4_dequantize(a_codes, a_sf, a_s) @ nvfp4_dequantize(b_codes, b_sf, b_s).T
+    if bias is not None:
+        c = c + np.asarray(bias, dtype=np.float64)[None, :]
+    return c
 
 
 def score_row(qmean_bh: np.ndarray, kmean_bh: np.ndarray, i: int):

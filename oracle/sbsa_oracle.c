@@ -44,6 +44,19 @@
  *              and scales match bit for bit.  Attention then runs on the dequantized
  *              Q and K (code value * block scale) with V as given.
  *
+ *   nvfp4   (next step: the linear layers around the attention, [Card] bullets NVFP4
+ *              量化感知训练 and 高效推理算子, and page "单卡 RTX 5090 跑 Wan2.2-A14B：720p 视频
+ *              生成只要 3.8 秒", 四步拆解 item 2: both GEMM operands in NVFP4 -- E2M1 values,
+ *              one FP8 E4M3 scale per 16 consecutive elements, one FP32 scale per tensor --
+ *              with FP32 accumulation, BF16 output and a column bias added in the epilogue).
+ *              The pages give no formula for the scales; the reading taken here: the
+ *              tensor scale s = 2688 / amax (2688 = 6 * 448, so the largest block scale
+ *              is 448 and its largest element 6); each block of 16 along a row gets
+ *              sf = e4m3((block amax / 6) * s); each element the e2m1 code of
+ *              x * (s / sf), nearest with ties to the even code, saturating at +-6.  All of
+ *              it in fp32 operations, the same the GPU performs.  A value decodes to
+ *              code * sf / s, and the GEMM is C = A_dec * B_dec^T + bias (per column).
+ *
  * Inputs are read as fp32, bf16 (raw 16-bit patterns, converted exactly) or fp64.
  * Tensors are row-major [B][H][Lp][d]; means are [B][H][nb][d]; col_idx is
  * [B][H][nb][k].  Padded tokens t >= L are ignored as keys and their query rows
@@ -198,6 +211,89 @@ void oracle_quantize_fp8(int B, int H, int L, int Lp, int d, int blk, const void
                 codes[i] = (uint8_t)oracle_e4m3_encode(y * inv);
             }
     }
+}
+
+/* e2m1 (1 sign, 2 exponent bits with bias 1, 1 mantissa bit, no infinities or NaN):
+ * magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 for codes 0..7; bit 3 is the sign. */
+double oracle_e2m1_decode(int code) {
+    int sgn = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return sgn ? -v : v;
+}
+
+/* float -> e2m1 code: nearest grid value, a tie going to the even code (mantissa bit
+ * 0), saturating at +-6.  The grid step is 0.5 below 2, 1 in [2, 4) and 2 in [4, 6];
+ * inside each range the code is (range offset) + n with n = value / step, so the even
+ * n of nearbyint (ties to even in the default rounding mode) is the even code. */
+int oracle_e2m1_encode(float x) {
+    int sgn = signbit(x) ? 1 : 0;
+    double a = fabs((double)x);
+    if (a >= 6.0) return (sgn << 3) | 7;
+    double step = a < 2.0 ? 0.5 : (a < 4.0 ? 1.0 : 2.0);
+    double r = nearbyint(a / step) * step;
+    int code;
+    if (r < 2.0) code = (int)(r * 2.0);      /* 0, 0.5, 1, 1.5 -> 0..3 */
+    else if (r < 4.0) code = (int)r + 2;     /* 2, 3 -> 4, 5 */
+    else if (r < 6.0) code = 6;              /* 4 */
+    else code = 7;                           /* 6 */
+    return (sgn << 3) | code;
+}
+
+/* Byte offset of the scale of (row r, 16-element block kb) in a scale array for K
+ * columns: atoms of 128 rows x 4 blocks (512 bytes), the atoms of one 128-row group
+ * consecutive along K, and inside an atom row r at (r % 32) * 16 + ((r % 128) / 32) * 4,
+ * block kb at + kb % 4. */
+size_t oracle_nvfp4_sf_offset(int r, int kb, int K) {
+    size_t atom = (size_t)(r / 128) * (size_t)(K / 64) + (size_t)(kb / 4);
+    return atom * 512 + (size_t)(r % 32) * 16 + (size_t)((r % 128) / 32) * 4 + (size_t)(kb % 4);
+}
+
+/* NVFP4 quantization of a row-major [rows][K] matrix (K a multiple of 64).  codes is
+ * [rows][K/2]: element 2i of a row in the low nibble of byte i, 2i+1 in the high
+ * nibble.  sf holds ceil(rows/128)*128 * K/16 bytes in the layout of
+ * oracle_nvfp4_sf_offset; rows beyond `rows` get scale 0.  Returns the tensor scale
+ * s = 2688 / amax (1 when the tensor is all zero). */
+float oracle_nvfp4_quantize(int rows, int K, const void *x, int dtype, uint8_t *codes, uint8_t *sf) {
+    float amax = 0.0f;
+    for (size_t i = 0; i < (size_t)rows * K; ++i) {
+        float a = fabsf((float)elem(x, dtype, i));
+        if (a > amax) amax = a;
+    }
+    const float s = amax > 0.0f ? 2688.0f / amax : 1.0f;
+    const int rows_p = (rows + 127) / 128 * 128;
+    memset(sf, 0, (size_t)rows_p * (K / 16));
+#pragma omp parallel for schedule(static) num_threads(oracle_threads_used())
+    for (int r = 0; r < rows; ++r) {
+        for (int kb = 0; kb < K / 16; ++kb) {
+            float bmax = 0.0f;
+            for (int c = kb * 16; c < kb * 16 + 16; ++c) {
+                float a = fabsf((float)elem(x, dtype, (size_t)r * K + c));
+                if (a > bmax) bmax = a;
+            }
+            float scaled = (bmax / 6.0f) * s;
+            int code_sf = oracle_e4m3_encode(scaled);
+            sf[oracle_nvfp4_sf_offset(r, kb, K)] = (uint8_t)code_sf;
+            float sf_f = (float)oracle_e4m3_decode(code_sf);
+            float inv = sf_f > 0.0f ? s / sf_f : 0.0f;
+            for (int c = kb * 16; c < kb * 16 + 16; c += 2) {
+                int lo = oracle_e2m1_encode((float)elem(x, dtype, (size_t)r * K + c) * inv);
+                int hi = oracle_e2m1_encode((float)elem(x, dtype, (size_t)r * K + c + 1) * inv);
+                codes[((size_t)r * K + c) / 2] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+    }
+    return s;
+}
+
+/* Decoded NVFP4 matrix in fp64: out[r][c] = e2m1(code) * e4m3(sf) / s. */
+void oracle_nvfp4_dequantize(int rows, int K, const uint8_t *codes, const uint8_t *sf, float s, double *out) {
+    for (int r = 0; r < rows; ++r)
+        for (int c = 0; c < K; ++c) {
+            uint8_t byte = codes[((size_t)r * K + c) / 2];
+            int code = (c & 1) ? (byte >> 4) : (byte & 15);
+            double scale = oracle_e4m3_decode(sf[oracle_nvfp4_sf_offset(r, c / 16, K)]);
+            out[(size_t)r * K + c] = oracle_e2m1_decode(code) * scale / (double)s;
+        }
 }
 
 /* Step 2, part a: one row of the block-score matrix, s_j = sum_c qm[i,c]*km[j,c],

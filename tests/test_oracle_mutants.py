@@ -55,6 +55,21 @@ MUTANTS = {
     "fp8_round_half_up": ("double n = nearbyint(a / quantum);", "double n = floor(a / quantum + 0.5);"),
     # padded tokens counted in the block's amax
     "fp8_amax_counts_padding": ("for (int t = t0; t < t0 + blk && t < L; ++t)", "for (int t = t0; t < t0 + blk; ++t)"),
+    # e2m1 rounding half away from zero instead of to the even code
+    "fp4_round_half_up": ("double r = nearbyint(a / step) * step;", "double r = floor(a / step + 0.5) * step;"),
+    # the two elements of a byte swapped between the nibbles
+    "fp4_nibble_order": ("codes[((size_t)r * K + c) / 2] = (uint8_t)(lo | (hi << 4));",
+                         "codes[((size_t)r * K + c) / 2] = (uint8_t)(hi | (lo << 4));"),
+    # scale layout: the row's 32-group and lane swapped inside an atom
+    "fp4_sf_layout": ("(size_t)(r % 32) * 16 + (size_t)((r % 128) / 32) * 4", "(size_t)(r % 32) * 4 + (size_t)((r % 128) / 32) * 16"),
+    # tensor scale without the e2m1 maximum (448 / amax instead of 6 * 448 / amax)
+    "fp4_tensor_scale": ("const float s = amax > 0.0f ? 2688.0f / amax : 1.0f;",
+                         "const float s = amax > 0.0f ? 448.0f / amax : 1.0f;"),
+    # block scale from the block's amax without dividing by the e2m1 maximum
+    "fp4_block_scale": ("float scaled = (bmax / 6.0f) * s;", "float scaled = bmax * s / 448.0f;"),
+    # decoded values not divided by the tensor scale
+    "fp4_dequant_no_tensor_scale": ("out[(size_t)r * K + c] = oracle_e2m1_decode(code) * scale / (double)s;",
+                                    "out[(size_t)r * K + c] = oracle_e2m1_decode(code) * scale;"),
 }
 
 

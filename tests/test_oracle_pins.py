@@ -495,3 +495,135 @@ def test_fp8_attention_is_close_to_exact_attention():
     # logits of d = 64 products of ~N(0,1) values with 2^-4 relative errors per factor
     assert err.max() < 0.1 and err.mean() < 0.01
     assert err.max() > 0  # and the quantization does something
+
+
+# ---------------------------------------------------------------- NVFP4 (linear layers)
+
+def test_e2m1_hand_values():
+    # e2m1: bias 1, one mantissa bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6
+    exact = {0.0: 0x0, 0.5: 0x1, 1.0: 0x2, 1.5: 0x3, 2.0: 0x4, 3.0: 0x5, 4.0: 0x6, 6.0: 0x7,
+             -0.5: 0x9, -1.5: 0xB, -3.0: 0xD, -6.0: 0xF}
+    for v, c in exact.items():
+        assert oracle.e2m1_encode(v) == c, v
+        assert oracle.e2m1_decode(np.array([c]))[0] == v
+    # halfway cases go to the even code (mantissa bit 0)
+    ties = {0.25: 0x0, 0.75: 0x2, 1.25: 0x2, 1.75: 0x4, 2.5: 0x4, 3.5: 0x6, 5.0: 0x6, -2.5: 0xC}
+    for v, c in ties.items():
+        assert oracle.e2m1_encode(v) == c, v
+    # nearest, not truncated; beyond 6 saturates
+    near = {0.26: 0x1, 1.3: 0x3, 2.6: 0x5, 5.1: 0x7, 6.5: 0x7, 1000.0: 0x7, -7.0: 0xF, 0.2: 0x0}
+    for v, c in near.items():
+        assert oracle.e2m1_encode(v) == c, v
+
+
+def test_e2m1_round_trip_and_nearest_by_brute_force():
+    codes = np.arange(16)
+    vals = oracle.e2m1_decode(codes)
+    for c, v in zip(codes, vals):
+        if c != 0x8:  # -0 encodes as +0's magnitude with the sign bit
+            assert oracle.e2m1_encode(v) == c
+    grid = np.unique(vals)
+    rng = np.random.default_rng(41)
+    for x in rng.uniform(-7, 7, 2000).astype(np.float32):
+        got = oracle.e2m1_decode(np.array([oracle.e2m1_encode(x)]))[0]
+        best = np.min(np.abs(grid - np.clip(x, -6, 6)))
+        assert abs(got - np.clip(x, -6, 6)) == best
+
+
+def test_nvfp4_sf_layout_hand_offsets():
+    K = 256  # 16 blocks per row, 4 atoms of 4 blocks per 128-row group
+    # (row, block) -> offset: atom = (row // 128) * (K // 64) + block // 4, then
+    # (row % 32) * 16 + ((row % 128) // 32) * 4 + block % 4 inside the 512-byte atom
+    cases = {(0, 0): 0, (0, 1): 1, (0, 3): 3, (0, 4): 512, (1, 0): 16, (31, 0): 496, (32, 0): 4,
+             (33, 1): 21, (127, 15): 3 * 512 + 31 * 16 + 3 * 4 + 3, (128, 0): 4 * 512, (200, 6): 5 * 512 + 8 * 16 + 2 * 4 + 2}
+    for (r, kb), off in cases.items():
+        assert oracle.nvfp4_sf_offset(r, kb, K) == off, (r, kb)
+
+
+def test_nvfp4_nibble_order_and_scales_by_hand():
+    # one row, 64 columns; amax 6 -> s = 2688/6 = 448; block 0 amax 6 -> sf = e4m3(448) = 0x7E
+    x = np.zeros((1, 64), dtype=np.float32)
+    x[0, 0], x[0, 1] = 0.5, 6.0          # codes 1 (low nibble) and 7 (high nibble): byte 0x71
+    x[0, 2], x[0, 3] = -1.0, 0.0         # codes 0xA and 0: byte 0x0A
+    x[0, 16] = 3.0                       # block 1: amax 3 -> sf = e4m3(0.5 * 448 = 224) = 0x76, code(6) = 7
+    codes, sf, s = oracle.nvfp4_quantize(x)
+    assert s == np.float32(448.0)
+    assert codes[0, 0] == 0x71 and codes[0, 1] == 0x0A and codes[0, 8] == 0x07
+    assert sf[0] == 0x7E and sf[1] == 0x76 and sf[2] == 0 and sf[3] == 0
+    # rows beyond the matrix (padding up to 128) have scale 0
+    assert np.all(sf[16:] == 0) and sf.size == 128 * 4
+
+
+def test_nvfp4_exactly_representable_inputs_round_trip():
+    # x = (e2m1 value) * 2^j with every block holding a +-6 * 2^j: all scales are exact
+    rng = np.random.default_rng(42)
+    rows, K = 130, 128
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], dtype=np.float64)
+    mag = rng.choice(grid, size=(rows, K)) * rng.choice([-1, 1], size=(rows, K))
+    j = rng.integers(-6, 3, size=(rows, K // 16))
+    j[0, 0] = 3  # the block holding the tensor amax 6 * 2^3
+    mag.reshape(rows, K // 16, 16)[:, :, 5] = 6.0
+    x = (mag.reshape(rows, K // 16, 16) * np.exp2(j)[:, :, None]).reshape(rows, K)
+    codes, sf, s = oracle.nvfp4_quantize(x.astype(np.float32))
+    np.testing.assert_array_equal(oracle.nvfp4_dequantize(codes, sf, s), x)
+
+
+def test_nvfp4_block_scale_and_error_bound():
+    rng = np.random.default_rng(43)
+    x = rng.standard_normal((40, 192)).astype(np.float32)
+    x[3, 16:32] *= 1e-3                    # a block far below the others
+    codes, sf, s = oracle.nvfp4_quantize(x)
+    amax = np.abs(x).max()
+    assert s == np.float32(2688.0) / np.float32(amax)
+    d = oracle.nvfp4_dequantize(codes, sf, s)
+    for r in range(40):
+        for kb in range(192 // 16):
+            blk = x[r, kb * 16:(kb + 1) * 16].astype(np.float64)
+            sfv = oracle.e4m3_decode(np.array([sf[oracle.nvfp4_sf_offset(r, kb, 192)]]))[0]
+            step = sfv / s  # the value of one e2m1 unit in this block
+            # the block scale is the e4m3 rounding of (block amax / 6) * s: within 2^-4
+            target = float(np.float32(np.float32(np.abs(blk).max()) / np.float32(6.0)) * np.float32(s))
+            assert abs(sfv - target) <= target * 2.0 ** -4
+            # every element is the nearest of the block's 15 grid values (of x clipped to +-6 steps)
+            grid = np.unique(np.concatenate([oracle.e2m1_decode(np.arange(16))])) * step
+            got = d[r, kb * 16:(kb + 1) * 16]
+            for xv, gv in zip(blk, got):
+                assert abs(gv - np.clip(xv, grid[0], grid[-1])) <= np.min(np.abs(grid - xv)) * (1 + 1e-6) + 1e-300
+
+
+def test_nvfp4_gemm_exact_and_closed_forms():
+    rng = np.random.default_rng(44)
+    M, N, K = 96, 160, 128             # non-square: a transposed operand cannot pass
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], dtype=np.float64)
+
+    def exact(rows):
+        v = rng.choice(grid, size=(rows, K)) * rng.choice([-1, 1], size=(rows, K))
+        v.reshape(rows, K // 16, 16)[:, :, 0] = 6.0
+        return (v.reshape(rows, K // 16, 16) * np.exp2(rng.integers(-3, 2, size=(rows, K // 16)))[:, :, None]
+                ).reshape(rows, K)
+
+    a, b = exact(M), exact(N)
+    bias = rng.standard_normal(N)
+    qa, qb = oracle.nvfp4_quantize(a.astype(np.float32)), oracle.nvfp4_quantize(b.astype(np.float32))
+    c = oracle.nvfp4_gemm(*qa, *qb, bias)
+    np.testing.assert_array_equal(c, a @ b.T + bias[None, :])
+    # A = 0: every row of C is the bias (a column vector of C per n)
+    z = oracle.nvfp4_quantize(np.zeros((M, K), dtype=np.float32))
+    np.testing.assert_array_equal(oracle.nvfp4_gemm(*z, *qb, bias), np.broadcast_to(bias, (M, N)))
+    # one-hot rows of A pick columns of B_dec
+    e = np.zeros((4, K), dtype=np.float32)
+    e[np.arange(4), [0, 17, 64, 127]] = 6.0
+    qe = oracle.nvfp4_quantize(e)
+    bd = oracle.nvfp4_dequantize(*qb)
+    np.testing.assert_array_equal(oracle.nvfp4_gemm(*qe, *qb), 6.0 * bd[:, [0, 17, 64, 127]].T)
+
+
+def test_nvfp4_gemm_close_to_unquantized():
+    rng = np.random.default_rng(45)
+    a = rng.standard_normal((64, 256)).astype(np.float32)
+    b = rng.standard_normal((128, 256)).astype(np.float32)
+    c = oracle.nvfp4_gemm(*oracle.nvfp4_quantize(a), *oracle.nvfp4_quantize(b))
+    ref = a.astype(np.float64) @ b.T.astype(np.float64)
+    rel = np.linalg.norm(c - ref) / np.linalg.norm(ref)
+    # per-element relative error of e2m1 with block scales is ~ 1/12 rms; two operands
+    assert 0.02 < rel < 0.2, rel
