@@ -50,6 +50,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-rope", action="store_true", help="skip timing the fused RoPE + pooling kernel")
     ap.add_argument("--no-fp8", action="store_true", help="skip timing the FP8 path")
+    ap.add_argument("--no-nvfp4", action="store_true", help="skip timing the NVFP4 linear layer")
     ap.add_argument("--cpu-units", type=int, default=16, help="attention units in the CPU sample")
     return ap.parse_args()
 
@@ -100,6 +101,24 @@ def fp8_summary(fp8: dict, flops: float, pool_select_ms: float, peaks: dict) -> 
                                        "algorithmic_bytes": fp8["quant_bytes"]},
             "layer_ms": layer_ms, "layer_TFLOP/s": flops / (layer_ms / 1e3) / 1e12,
             "note": "pool + select + key mean + quantize + fp8 attention, timed apart from the step"}
+
+
+def fp4_summary(fp4: dict, peaks: dict) -> dict:
+    """Figures of the NVFP4 linear layer.  Its GEMM is a dense contraction on the
+    block-scaled fp4 tensor cores, whose peak is taken as the measured bf16 peak x 4 (the
+    nominal 9 / 2.25 PFLOP/s ratio); the quantizer is bandwidth-bound."""
+    fp4_peak = 4.0 * peaks["bf16_tflops"]
+    tf = fp4["gemm_flop"] / (fp4["gemm_ms"] / 1e3) / 1e12
+    qgbs = fp4["quant_bytes"] / (fp4["quant_ms"] / 1e3) / 1e9
+    return {"shape": {"m": fp4["m"], "n": fp4["n"], "k": fp4["k"]},
+            "gemm": {"ms": fp4["gemm_ms"], "TFLOP/s": tf, "peak": fp4_peak, "frac": tf / fp4_peak,
+                     "kernel": "nvfp4_gemm_kernel", "algorithmic_flop": fp4["gemm_flop"],
+                     "algorithmic_bytes": fp4["gemm_bytes"],
+                     "GB/s": fp4["gemm_bytes"] / (fp4["gemm_ms"] / 1e3) / 1e9},
+            "amax_plus_quantize": {"ms": fp4["quant_ms"], "GB/s": qgbs, "hbm_frac": qgbs / peaks["hbm_gbs"],
+                                   "algorithmic_bytes": fp4["quant_bytes"]},
+            "layer_ms": fp4["quant_ms"] + fp4["gemm_ms"],
+            "note": "QKV projection of the same tokens, timed apart from the step"}
 
 
 def job_tflops(flops_per_rank: float, world: int, ms: float) -> float:
@@ -438,6 +457,54 @@ def run_gpu(args, wl):
                "quant_bytes": 2 * q.numel() * 2 + 2 * q.numel() + 2 * rows * 4 + km.numel() * 4}
         del kbar, q8, k8, qs, ks, o8
 
+    # the NVFP4 linear layer that feeds this attention: the fused QKV projection of the
+    # same tokens, [L, H*d] x [3*H*d, H*d]^T + bias.  The weights are quantized once; a
+    # step quantizes the activations (amax, then codes and scales) and runs the GEMM.
+    fp4 = None
+    if not args.no_nvfp4 and wl.head_dim * wl.heads % 256 == 0:
+        fm, fk = wl.seq_len_padded * wl.batch, wl.heads * wl.head_dim
+        fn = 3 * fk
+        g4 = torch.Generator(device=dev).manual_seed(100 + rank)
+        xa = torch.randn(fm, fk, generator=g4, device=dev).to(torch.bfloat16)
+        wb = (torch.randn(fn, fk, generator=g4, device=dev) * 0.02).to(torch.bfloat16)
+        bias4 = torch.randn(fn, generator=g4, device=dev)
+        a_amax = torch.empty(1, dtype=torch.float32, device=dev)
+        b_amax = torch.empty_like(a_amax)
+        a_codes = torch.empty(fm * fk // 2, dtype=torch.uint8, device=dev)
+        b_codes = torch.empty(fn * fk // 2, dtype=torch.uint8, device=dev)
+        a_sf = torch.empty(sbsa.sbsa_nvfp4_scale_bytes(fm, fk), dtype=torch.uint8, device=dev)
+        b_sf = torch.empty(sbsa.sbsa_nvfp4_scale_bytes(fn, fk), dtype=torch.uint8, device=dev)
+        c4 = torch.empty(fm, fn, dtype=torch.bfloat16, device=dev)
+        sbsa.sbsa_nvfp4_amax(wb, b_amax, stream=stream)
+        sbsa.sbsa_nvfp4_quantize(wb, b_amax, b_codes, b_sf, stream=stream)
+
+        def fp4_step(fe=None):
+            if fe: fe[0].record(stream)
+            sbsa.sbsa_nvfp4_amax(xa, a_amax, stream=stream)
+            sbsa.sbsa_nvfp4_quantize(xa, a_amax, a_codes, a_sf, stream=stream)
+            if fe: fe[1].record(stream)
+            sbsa.sbsa_nvfp4_gemm(fm, fn, fk, a_codes, a_sf, a_amax, b_codes, b_sf, b_amax, bias4, c4, stream=stream)
+            if fe: fe[2].record(stream)
+
+        for _ in range(3):
+            fp4_step()
+        n_fp4 = max(3, min(args.steps, 10))
+        fes = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_fp4)]
+        for i in range(n_fp4):
+            fp4_step(fes[i])
+        torch.cuda.synchronize(dev)
+        sbsa.sbsa_check(stream)
+        fp4 = {"quant_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in fes),
+               "gemm_ms": statistics.mean(e[1].elapsed_time(e[2]) for e in fes),
+               "m": fm, "n": fn, "k": fk,
+               # amax pass reads the activations, the quantizer reads them again and
+               # writes codes (k/2 bytes per row) and scales (k/16)
+               "quant_bytes": 2 * fm * fk * 2 + fm * fk // 2 + fm * fk // 16,
+               # the GEMM must read both operands' codes and scales and write C once
+               "gemm_bytes": (fm + fn) * (fk // 2 + fk // 16) + fm * fn * 2,
+               "gemm_flop": 2.0 * fm * fn * fk}
+        del xa, wb, bias4, a_codes, b_codes, a_sf, b_sf, c4
+
     # end to end through the public API from pinned host buffers
     e2e = None
     if not args.no_e2e:
@@ -464,7 +531,9 @@ def run_gpu(args, wl):
                                  "forward": forward_ms, "e2e": e2e["ms"] if e2e is not None else 0.0,
                                  "rope": rope["ms"] if rope is not None else 0.0,
                                  "fp8_quant": fp8["quant_ms"] if fp8 is not None else 0.0,
-                                 "fp8_att": fp8["att_ms"] if fp8 is not None else 0.0})
+                                 "fp8_att": fp8["att_ms"] if fp8 is not None else 0.0,
+                                 "fp4_quant": fp4["quant_ms"] if fp4 is not None else 0.0,
+                                 "fp4_gemm": fp4["gemm_ms"] if fp4 is not None else 0.0})
     elapsed_ms, att_avg, pool_avg, sel_avg, forward_ms = (t[n] for n in ("elapsed", "att", "pool", "sel", "forward"))
     if e2e is not None:
         e2e["ms"] = t["e2e"]
@@ -472,6 +541,8 @@ def run_gpu(args, wl):
         rope["ms"] = t["rope"]
     if fp8 is not None:
         fp8["quant_ms"], fp8["att_ms"] = t["fp8_quant"], t["fp8_att"]
+    if fp4 is not None:
+        fp4["quant_ms"], fp4["gemm_ms"] = t["fp4_quant"], t["fp4_gemm"]
     ms_step = elapsed_ms / args.steps
     value = job_tflops(flops, ws_n, ms_step)
 
@@ -508,6 +579,7 @@ def run_gpu(args, wl):
                                   "note": "3D RoPE fused with pooling, timed alone (not part of the step)"}}
                    if rope is not None else {}),
                 **({"fp8": fp8_summary(fp8, flops, pool_avg + sel_avg, peaks)} if fp8 is not None else {}),
+                **({"nvfp4_linear": fp4_summary(fp4, peaks)} if fp4 is not None else {}),
             },
             "peaks": {"source": peak_src, **peaks},
         }

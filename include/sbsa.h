@@ -178,6 +178,47 @@ sbsa_status sbsa_attention_fwd_fp8(const sbsa_shape *shape, const void *q8, cons
                                    const float *q_scale, const float *k_scale, const int32_t *row_ptr,
                                    const int32_t *col_idx, float scale, void *o, void *stream);
 
+/* ---- NVFP4 linear layers (the GEMMs around the attention) ---------------------------
+ * Page "知识卡片：600倍加速，720p视频实时生成！单卡也能带的动14B模型", 方法/产品要点, bullets
+ * NVFP4 量化感知训练 (E2M1 values, one FP8 scale per 16 consecutive elements, an FP32
+ * scale per tensor) and 高效推理算子 (both GEMM operands NVFP4 on the block-scaled tensor
+ * cores); page "单卡 RTX 5090 跑 Wan2.2-A14B：720p 视频生成只要 3.8 秒", 四步拆解 item 2
+ * (FP32 accumulation, BF16 output, column bias fused into the epilogue).
+ *
+ * Formats (the pages give no formula; this is the reading taken):
+ *   tensor scale s = 2688 / amax|x| (1 for an all-zero tensor), 2688 = 6 * 448;
+ *   block scale sf = e4m3((amax of the 16 elements / 6) * s), round to nearest even,
+ *   saturating; code = e2m1(x * (s / sf)), nearest even, saturating at +-6 (0 where
+ *   sf = 0); all in fp32, in this order.  Value = e2m1(code) * e4m3(sf) / s.
+ *   codes:  [rows][cols/2] bytes, row-major; element 2i of a row in the low nibble of
+ *           byte i.
+ *   scales: sbsa_nvfp4_scale_bytes(rows, cols) bytes; atoms of 128 rows x 4 blocks (512
+ *           bytes: row r at (r % 32) * 16 + ((r % 128) / 32) * 4, block kb at + kb % 4),
+ *           the cols/64 atoms of one 128-row group consecutive, groups in row order;
+ *           rows past the matrix (up to a multiple of 128) have scale 0.
+ * All pointers are device pointers owned by the caller; every call is asynchronous on
+ * `stream`; argument errors are returned before any launch, launch errors as
+ * SBSA_ERR_CUDA, and a kernel that gives up on a wait latches SBSA_ERR_TIMEOUT for
+ * sbsa_check.
+ *
+ * sbsa_nvfp4_scale_bytes: size of the scale array of a [rows][cols] matrix (cols a
+ *   multiple of 64), 0 for invalid sizes.
+ * sbsa_nvfp4_amax: *amax = max |x| over a bf16 [rows][cols] matrix (16-byte aligned,
+ *   cols a multiple of 8).  Resets *amax first, then one reduction launch.
+ * sbsa_nvfp4_quantize: bf16 [rows][cols] (cols a multiple of 64) -> codes and scales,
+ *   with the tensor scale taken from *amax (device, as written by sbsa_nvfp4_amax).
+ * sbsa_nvfp4_gemm: c[m][n] (bf16, row-major) = A B^T / (s_A s_B) + bias[n], A = [m][k]
+ *   and B = [n][k] as NVFP4 codes + scales, s_A and s_B from a_amax / b_amax (device).
+ *   bias ([n] fp32) may be NULL.  Needs k a multiple of 256, n a multiple of 8; m any.
+ *   Codes, scales and c 16-byte aligned. */
+size_t sbsa_nvfp4_scale_bytes(int64_t rows, int32_t cols);
+sbsa_status sbsa_nvfp4_amax(const void *x, int64_t rows, int32_t cols, float *amax, void *stream);
+sbsa_status sbsa_nvfp4_quantize(const void *x, int64_t rows, int32_t cols, const float *amax, void *codes,
+                                void *scales, void *stream);
+sbsa_status sbsa_nvfp4_gemm(int32_t m, int32_t n, int32_t k, const void *a, const void *a_scales, const float *a_amax,
+                            const void *b, const void *b_scales, const float *b_amax, const float *bias, void *c,
+                            void *stream);
+
 /* Steps 1-3 in one call on one stream: pool -> select -> attend, with the means and
  * the CSR lists carved out of `workspace` (device, 256-byte aligned, at least
  * sbsa_workspace_bytes(shape, k_keep) bytes).  If col_idx_out is non-NULL the

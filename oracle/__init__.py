@@ -68,7 +68,7 @@ def _load():
         lib.oracle_e2m1_encode.restype = I
         lib.oracle_nvfp4_sf_offset.argtypes = [I, I, I]
         lib.oracle_nvfp4_sf_offset.restype = ctypes.c_size_t
-        lib.oracle_nvfp4_quantize.argtypes = [I, I, P, I, P, P]
+        lib.oracle_nvfp4_quantize.argtypes = [I, I, P, I, ctypes.c_float, P, P]
         lib.oracle_nvfp4_quantize.restype = ctypes.c_float
         lib.oracle_nvfp4_dequantize.argtypes = [I, I, P, P, ctypes.c_float, P]
         lib.oracle_nvfp4_dequantize.restype = None
@@ -218,15 +218,17 @@ def nvfp4_sf_bytes(rows: int, K: int) -> int:
     return (rows + 127) // 128 * 128 * (K // 16)
 
 
-def nvfp4_quantize(x):
-    """[rows, K] (bf16 bits, fp32 or fp64) -> (codes uint8 [rows, K/2], sf uint8, tensor scale s)."""
+def nvfp4_quantize(x, amax=None):
+    """[rows, K] (bf16 bits, fp32 or fp64) -> (codes uint8 [rows, K/2], sf uint8, tensor scale s).
+
+    amax: the tensor's max |x| when x holds rows sampled from a larger tensor."""
     a, dt = _as_input(x)
     rows, K = a.shape
     if K % 64:
         raise ValueError("K must be a multiple of 64")
     codes = np.empty((rows, K // 2), dtype=np.uint8)
     sf = np.empty(nvfp4_sf_bytes(rows, K), dtype=np.uint8)
-    s = _load().oracle_nvfp4_quantize(rows, K, _ptr(a), dt, _ptr(codes), _ptr(sf))
+    s = _load().oracle_nvfp4_quantize(rows, K, _ptr(a), dt, -1.0 if amax is None else float(amax), _ptr(codes), _ptr(sf))
     return codes, sf, float(np.float32(s))
 
 

@@ -251,14 +251,16 @@ size_t oracle_nvfp4_sf_offset(int r, int kb, int K) {
 /* NVFP4 quantization of a row-major [rows][K] matrix (K a multiple of 64).  codes is
  * [rows][K/2]: element 2i of a row in the low nibble of byte i, 2i+1 in the high
  * nibble.  sf holds ceil(rows/128)*128 * K/16 bytes in the layout of
- * oracle_nvfp4_sf_offset; rows beyond `rows` get scale 0.  Returns the tensor scale
- * s = 2688 / amax (1 when the tensor is all zero). */
-float oracle_nvfp4_quantize(int rows, int K, const void *x, int dtype, uint8_t *codes, uint8_t *sf) {
+ * oracle_nvfp4_sf_offset; rows beyond `rows` get scale 0.  amax is max |x| over these rows,
+ * or amax_in when that is >= 0 (rows sampled from a larger tensor).  Returns the tensor
+ * scale s = 2688 / amax (1 when the tensor is all zero). */
+float oracle_nvfp4_quantize(int rows, int K, const void *x, int dtype, float amax_in, uint8_t *codes, uint8_t *sf) {
     float amax = 0.0f;
     for (size_t i = 0; i < (size_t)rows * K; ++i) {
         float a = fabsf((float)elem(x, dtype, i));
         if (a > amax) amax = a;
     }
+    if (amax_in >= 0.0f) amax = amax_in; /* rows sampled from a larger tensor: its amax */
     const float s = amax > 0.0f ? 2688.0f / amax : 1.0f;
     const int rows_p = (rows + 127) / 128 * 128;
     memset(sf, 0, (size_t)rows_p * (K / 16));

@@ -130,3 +130,25 @@ def test_rope_table_size_and_argument_errors():
     st = lib.sbsa_rope_pool_qk(ctypes.byref(s), 2, 6, 10, None, None, None, None, None, None, None, None)
     assert st == 1 and b"null" in lib.sbsa_last_error_message()
     assert lib.sbsa_rope_table_init(128, 2, 6, 10, 1.0, None, None) == 1   # theta must exceed 1
+
+
+def test_nvfp4_sizes_and_argument_errors():
+    from video_dit_dynamic_b200 import sbsa
+    # scale bytes: rows padded to 128, one byte per 16 columns
+    assert sbsa.sbsa_nvfp4_scale_bytes(1, 64) == 128 * 4
+    assert sbsa.sbsa_nvfp4_scale_bytes(300, 512) == 384 * 32
+    assert sbsa.sbsa_nvfp4_scale_bytes(122880, 5120) == 122880 * 320
+    assert sbsa.sbsa_nvfp4_scale_bytes(10, 100) == 0 and sbsa.sbsa_nvfp4_scale_bytes(0, 64) == 0
+    lib = sbsa.load()
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: every call below fails its argument checks
+    assert lib.sbsa_nvfp4_gemm(128, 256, 256, None, fake, fake, fake, fake, fake, None, fake, None) == 1
+    assert b"null" in lib.sbsa_last_error_message()
+    for m, n, k in ((0, 256, 256), (128, 250, 256), (128, 256, 320), (128, 256, 128)):
+        st = lib.sbsa_nvfp4_gemm(m, n, k, fake, fake, fake, fake, fake, fake, None, fake, None)
+        assert st == 1, (m, n, k)
+    # misaligned codes
+    st = lib.sbsa_nvfp4_gemm(128, 256, 256, ctypes.c_void_p((1 << 20) + 8), fake, fake, fake, fake, fake, None,
+                             fake, None)
+    assert st == 1 and b"aligned" in lib.sbsa_last_error_message()
+    assert lib.sbsa_nvfp4_quantize(fake, 10, 100, fake, fake, fake, None) == 1
+    assert lib.sbsa_nvfp4_amax(fake, 10, 12, fake, None) == 1

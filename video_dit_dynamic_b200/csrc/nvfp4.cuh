@@ -1,0 +1,415 @@
+// NVFP4 linear layer (the GEMMs around the attention): both operands in NVFP4 -- E2M1
+// values, one E4M3 scale per 16 consecutive elements of a row, one FP32 scale per
+// tensor -- multiplied on the tcgen05 block-scaled tensor cores with FP32 accumulation,
+// BF16 output and a per-column bias added in the epilogue (page "知识卡片：600倍加速，
+// 720p视频实时生成！单卡也能带的动14B模型", 方法/产品要点, bullets NVFP4 量化感知训练 and
+// 高效推理算子; page "单卡 RTX 5090 跑 Wan2.2-A14B：720p 视频生成只要 3.8 秒", 四步拆解
+// item 2).
+//
+// Quantization (the pages give no formula; the plainest reading of their description):
+//   s     = 2688 / amax(|x|) over the tensor (1 for an all-zero tensor); 2688 = 6 * 448
+//   sf_b  = e4m3((amax of block b / 6) * s), nearest even, saturating
+//   code  = e2m1(x * (s / sf_b)), nearest even, saturating at +-6 (0 where sf_b = 0)
+// every step an fp32 operation in this order.  A value decodes to code * sf_b / s, so
+//   C[m][n] = (1 / (s_A s_B)) * sum_k code_A sf_A code_B sf_B + bias[n].
+//
+// Layouts:
+//   codes  [rows][K/2] bytes, element 2i of a row in the low nibble of byte i;
+//   scales atoms of 128 rows x 4 blocks (512 bytes; row r at (r % 32) * 16 +
+//          ((r % 128) / 32) * 4, block kb at + kb % 4), the K/64 atoms of one 128-row
+//          group consecutive; rows padded to a multiple of 128 (scale 0).  One atom is
+//          exactly what tcgen05.cp.32x128b.warpx4 moves into four TMEM columns, where the
+//          block-scaled MMA reads the scales of row r from column r / 32.
+#pragma once
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "rope.cuh"
+#include "tmem_wide.cuh"
+
+namespace sbsa {
+
+constexpr float kNvfp4Range = 2688.f;  // largest e2m1 (6) x largest e4m3 (448)
+
+__device__ __forceinline__ float nvfp4_tensor_scale(float amax) {
+    return amax > 0.f ? __fdiv_rn(kNvfp4Range, amax) : 1.f;
+}
+
+// e4m3 code (non-negative, finite) -> its exact fp32 value, from the format: bias 7,
+// three mantissa bits, subnormals m * 2^-9.
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+    const uint32_t e = (code >> 3) & 15u, m = code & 7u;
+    return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : static_cast<float>(m) * 0.001953125f;
+}
+
+// Eight floats -> eight e2m1 codes, v[0] in the lowest nibble (nearest even, saturating).
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return r;
+}
+
+__host__ __device__ constexpr size_t nvfp4_scale_offset(long long r, int kb, int K) {
+    return (static_cast<size_t>(r / 128) * static_cast<size_t>(K / 64) + static_cast<size_t>(kb / 4)) * 512 +
+           static_cast<size_t>(r % 32) * 16 + static_cast<size_t>((r % 128) / 32) * 4 + static_cast<size_t>(kb % 4);
+}
+
+// ---------------------------------------------------------------- amax
+// max |x| over a bf16 tensor of n8 16-byte chunks.  The result is combined with an
+// atomicMax on the float's bit pattern (for non-negative floats the bit patterns order
+// like the values); *out must hold 0 before the launch.
+__global__ void __launch_bounds__(256) nvfp4_amax_kernel(const uint4* __restrict__ x, long long n8,
+                                                         unsigned int* __restrict__ out) {
+    __shared__ float red[8];
+    float m = 0.f;
+    for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n8; i += static_cast<long long>(gridDim.x) * 256) {
+        const uint4 w = __ldg(x + i);
+        const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            m = fmaxf(m, fabsf(__uint_as_float(v[j] << 16)));
+            m = fmaxf(m, fabsf(__uint_as_float(v[j] & 0xFFFF0000u)));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+    if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
+        atomicMax(out, __float_as_uint(m));
+    }
+}
+
+// ---------------------------------------------------------------- quantizer
+// One thread per (row, 16-element block) of a [rows][K] bf16 matrix: 32 bytes in,
+// 8 bytes of codes and one scale byte out.  Threads for the padding rows (up to a
+// multiple of 128) write scale 0.
+__global__ void __launch_bounds__(256) nvfp4_quantize_kernel(const uint4* __restrict__ x,
+                                                             const float* __restrict__ amax,
+                                                             uint2* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                             long long rows, int K, long long n_threads) {
+    const long long t = blockIdx.x * 256ll + threadIdx.x;
+    if (t >= n_threads) return;
+    const int kbs = K / 16;
+    const long long r = t / kbs;
+    const int kb = static_cast<int>(t % kbs);
+    const size_t off = nvfp4_scale_offset(r, kb, K);
+    if (r >= rows) {
+        scales[off] = 0;
+        return;
+    }
+    const float s = nvfp4_tensor_scale(__ldg(amax));
+    // row r, elements 16 kb .. 16 kb + 15 are 16-byte chunks 2 t and 2 t + 1
+    const uint4 w0 = __ldg(x + 2 * t), w1 = __ldg(x + 2 * t + 1);
+    const uint32_t in[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    float v[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        v[2 * j] = __uint_as_float(in[j] << 16);
+        v[2 * j + 1] = __uint_as_float(in[j] & 0xFFFF0000u);
+    }
+    float bmax = 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) bmax = fmaxf(bmax, fabsf(v[j]));
+    const float scaled = __fmul_rn(__fdiv_rn(bmax, 6.f), s);
+    uint16_t sf2;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(sf2) : "f"(0.f), "f"(scaled));
+    const uint32_t sf = sf2 & 0xFFu;
+    const float sf_f = e4m3_value(sf);
+    const float inv = sf_f > 0.f ? __fdiv_rn(s, sf_f) : 0.f;
+    float lo[8], hi[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        lo[j] = __fmul_rn(v[j], inv);
+        hi[j] = __fmul_rn(v[8 + j], inv);
+    }
+    codes[t] = make_uint2(cvt_e2m1x8(lo), cvt_e2m1x8(hi));
+    scales[off] = static_cast<uint8_t>(sf);
+}
+
+// ---------------------------------------------------------------- GEMM
+// C[M][N] = alpha * A[M][K] B[N][K]^T + bias[N], A and B NVFP4 (K-major), C bf16.
+//
+// Persistent: one CTA per SM walks output tiles of 128 x 256 (tile index t -> row
+// tile t / tiles_n, column tile t % tiles_n, so the CTAs running at one time share a
+// few A row tiles and all of B in L2).  320 threads:
+//   warp 0     TMA producer: per K-tile of 256 elements one stage of A (128 rows x
+//              128 bytes), B (256 x 128 bytes), their scale atoms (2 KB and 4 KB,
+//              contiguous in global memory, one bulk copy per 128-row group) through a
+//              four-stage ring;
+//   warp 1     TMEM allocation and the one thread that issues everything on the
+//              tensor pipe: per K-tile, twelve tcgen05.cp of scale atoms into TMEM and
+//              four block-scaled MMAs (M = 128, N = 256, K = 64).  tcgen05.cp and
+//              tcgen05.mma from one thread execute in issue order, so a TMEM scale
+//              region can be refilled right after the MMAs that read it were issued
+//              (issuing the next K-tile's copies ahead of the current MMAs was measured
+//              slower: it makes the MMAs wait for one more stage to land);
+//   warps 2-9  epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 and output columns
+//              128 ((w - 2) / 4) .. + 127 of the tile, applies alpha and the bias in
+//              fp32, rounds to bf16, hands the accumulator back, then stores its rows.
+// TMEM: accumulator in columns 0-255; two scale regions of 48 columns at 256 and 304,
+// used by alternate K-tiles, each with the A scales (four columns per K step) and then
+// the B scales (eight per K step).
+struct Nvfp4GemmParams {
+    const uint8_t* sfa;
+    const uint8_t* sfb;
+    const float* amax_a;
+    const float* amax_b;
+    const float* bias;  // [N] or null
+    __nv_bfloat16* c;   // [M][N]
+    int M, N, K;
+    int tiles_m, tiles_n;
+    unsigned int epoch;
+};
+
+constexpr int kFp4TileM = 128;
+constexpr int kFp4TileN = 256;
+constexpr int kFp4TileK = 256;  // elements: 128 bytes of codes per row
+constexpr int kFp4Stages = 4;
+constexpr int kFp4ABytes = kFp4TileM * 128;
+constexpr int kFp4BBytes = kFp4TileN * 128;
+constexpr int kFp4SfaBytes = (kFp4TileM / 128) * 4 * 512;
+constexpr int kFp4SfbBytes = (kFp4TileN / 128) * 4 * 512;
+constexpr int kFp4StageBytes = kFp4ABytes + kFp4BBytes + kFp4SfaBytes + kFp4SfbBytes;
+constexpr int kFp4BarOff = kFp4Stages * kFp4StageBytes;
+constexpr int kFp4NumBars = 2 * kFp4Stages + 3;  // full[S], empty[S], acc_full, acc_empty, drain
+constexpr int kFp4SmemBytes = kFp4BarOff + kFp4NumBars * 8 + 16 + 1024;  // + tmem slot, flag, alignment slack
+constexpr int kFp4Threads = 320;
+constexpr uint32_t kFp4ColSf = 256;     // two scale regions of 48 columns, by K-tile parity
+constexpr uint32_t kFp4SfRegion = 48;   // A scales at +0 (16 columns), B scales at +16 (32 columns)
+static_assert(kFp4StageBytes % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
+static_assert(kFp4SmemBytes <= 232448, "shared memory");
+
+// kind::mxf4nvf4 instruction descriptor: E2M1 A and B (format 1), UE4M3 scales
+// (bit 23 = 0), both K-major, dense K = 64, scale-factor ids 0.
+__host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
+    return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// 32 rows x 16 bytes of shared memory into TMEM columns taddr .. taddr + 3 of every lane
+// quarter (row i of the source goes to lane i of each quarter).
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Descriptor of a 512-byte scale atom: no swizzle, 8-row x 16-byte core matrices 128
+// bytes apart (both offsets 128: the atom is one core matrix wide).
+__device__ __forceinline__ uint64_t sdesc_atom(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(128 >> 4) << 16;
+    d |= static_cast<uint64_t>(128 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm100; layout type 0 = no swizzle
+    return d;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
+                                                                    const __grid_constant__ CUtensorMap map_b,
+                                                                    const Nvfp4GemmParams p) {
+    extern __shared__ __align__(1024) uint8_t fp4_smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fp4_smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kFp4BarOff);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + kFp4Stages;
+    uint64_t* acc_full = bars + 2 * kFp4Stages;
+    uint64_t* acc_empty = acc_full + 1;
+    uint64_t* drain = acc_full + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kFp4NumBars);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (launch_aborted(p.epoch)) return;
+    const int num_tiles = p.tiles_m * p.tiles_n;
+    const int k_tiles = p.K / kFp4TileK;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int s = 0; s < kFp4Stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 8);
+        mbar_init(drain, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&map_a);
+        tma_prefetch_desc(&map_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    auto give_up = [&]() {
+        *abort_flag = 1;
+        abort_launch(p.epoch);
+    };
+    auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+        if (mbar_wait_bounded(bar, parity, abort_flag, kWaitLimitNs)) return true;
+        if (!*abort_flag) give_up();
+        return false;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const uint64_t pol_a = policy_evict_normal();
+            const uint64_t pol_b = policy_evict_last();
+            const size_t k_atoms = static_cast<size_t>(p.K / 64);
+            const int n_groups = (p.N + 127) / 128;
+            int it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                const int tm = tile / p.tiles_n;
+                const int tn = tile % p.tiles_n;
+                const int g0 = tn * (kFp4TileN / 128);
+                const int ng = min(kFp4TileN / 128, n_groups - g0);  // B scale groups that exist
+                for (int kt = 0; kt < k_tiles; ++kt, ++it) {
+                    const int s = it % kFp4Stages;
+                    if (!(ok = wait(&empty[s], ((it / kFp4Stages) & 1) ^ 1))) break;
+                    uint8_t* st = smem + s * kFp4StageBytes;
+                    mbar_arrive_expect_tx(&full[s], kFp4ABytes + kFp4BBytes + kFp4SfaBytes + ng * 2048);
+                    tma_load_2d(st, &map_a, &full[s], kt * 128, tm * kFp4TileM, pol_a);
+                    tma_load_2d(st + kFp4ABytes, &map_b, &full[s], kt * 128, tn * kFp4TileN, pol_b);
+                    bulk_load_g2s(st + kFp4ABytes + kFp4BBytes, p.sfa + (static_cast<size_t>(tm) * k_atoms + 4 * kt) * 512,
+                                  2048, &full[s]);
+                    for (int g = 0; g < ng; ++g)
+                        bulk_load_g2s(st + kFp4ABytes + kFp4BBytes + kFp4SfaBytes + g * 2048,
+                                      p.sfb + (static_cast<size_t>(g0 + g) * k_atoms + 4 * kt) * 512, 2048, &full[s]);
+                }
+            }
+            if (!ok) {
+                // every issued copy must land before the CTA exits
+                volatile int never = 0;
+                for (int q = it - kFp4Stages < 0 ? 0 : it - kFp4Stages; q < it; ++q)
+                    mbar_wait_bounded(&full[q % kFp4Stages], (q / kFp4Stages) & 1, &never, kWaitLimitNs);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ tensor-pipe issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_nvfp4(kFp4TileM, kFp4TileN);
+            int it = 0, tcount = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++tcount) {
+                // the epilogue must have read the previous tile's accumulator out of TMEM
+                if (tcount > 0 && !(ok = wait(acc_empty, (tcount - 1) & 1))) break;
+                tc_fence_after();
+                for (int kt = 0; kt < k_tiles; ++kt, ++it) {
+                    const int s = it % kFp4Stages;
+                    if (!(ok = wait(&full[s], (it / kFp4Stages) & 1))) break;
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(smem + s * kFp4StageBytes);
+                    const uint32_t sfa = st + kFp4ABytes + kFp4BBytes;
+                    const uint32_t sfb = sfa + kFp4SfaBytes;
+                    // consecutive K-tiles use different TMEM scale regions
+                    const uint32_t t_sfa = tmem + kFp4ColSf + (it & 1) * kFp4SfRegion;
+                    const uint32_t t_sfb = t_sfa + 16;
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb) {
+                        tmem_cp_32x128b_warpx4(t_sfa + 4 * kb, sdesc_atom(sfa + kb * 512));
+                        tmem_cp_32x128b_warpx4(t_sfb + 8 * kb, sdesc_atom(sfb + kb * 512));
+                        tmem_cp_32x128b_warpx4(t_sfb + 8 * kb + 4, sdesc_atom(sfb + 2048 + kb * 512));
+                    }
+                    const uint64_t a0 = sdesc_sw128(st, 16, 1024);
+                    const uint64_t b0 = sdesc_sw128(st + kFp4ABytes, 16, 1024);
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb) {
+                        // K = 64 codes = 32 bytes per step inside the 128-byte swizzled row
+                        umma_nvfp4(tmem, a0 + static_cast<uint64_t>((kb * 32) >> 4), b0 + static_cast<uint64_t>((kb * 32) >> 4),
+                                   idesc, t_sfa + 4 * kb, t_sfb + 8 * kb, (kt | kb) ? 1u : 0u);
+                    }
+                    umma_commit(&empty[s]);
+                }
+                if (ok) umma_commit(acc_full);
+            }
+            if (!ok) {
+                umma_commit(drain);  // wait for every MMA this thread issued
+                volatile int never = 0;
+                mbar_wait_bounded(drain, 0, &never, kWaitLimitNs);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;
+        const int half = (warp - 2) >> 2;
+        const uint32_t t_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(half * 128);
+        const float alpha = __frcp_rn(__fmul_rn(nvfp4_tensor_scale(__ldg(p.amax_a)), nvfp4_tensor_scale(__ldg(p.amax_b))));
+        int tcount = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
+            const int tm = tile / p.tiles_n;
+            const int tn = tile % p.tiles_n;
+            const bool ok = __all_sync(0xFFFFFFFFu, wait(acc_full, tcount & 1));
+            if (!ok) break;
+            tc_fence_after();
+            const int n0 = tn * kFp4TileN + half * 128;
+            // this warp's 128 columns in two 64-column TMEM loads
+            uint32_t packed[64];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t raw[64];
+                tmem_ld64(t_row + c * 64, raw);
+#pragma unroll
+                for (int e = 0; e < 64; e += 2) {
+                    const int n = n0 + c * 64 + e;
+                    const float b0 = (p.bias && n < p.N) ? __ldg(p.bias + n) : 0.f;
+                    const float b1 = (p.bias && n + 1 < p.N) ? __ldg(p.bias + n + 1) : 0.f;
+                    packed[c * 32 + e / 2] = pack_bf16x2(fmaf(__uint_as_float(raw[e]), alpha, b0),
+                                                         fmaf(__uint_as_float(raw[e + 1]), alpha, b1));
+                }
+            }
+            // the accumulator is in registers: the next tile's MMAs may overwrite it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+            const long long m = static_cast<long long>(tm) * kFp4TileM + quarter * 32 + lane;
+            if (m < p.M) {
+                uint4* dst = reinterpret_cast<uint4*>(p.c + m * p.N + n0);
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    if (n0 + 8 * j < p.N)
+                        dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace sbsa

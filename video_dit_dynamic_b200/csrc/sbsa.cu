@@ -1,6 +1,7 @@
 // C ABI of the sbsa library (declared in include/sbsa.h): argument checking, tensor-map
 // encoding, workspace carving and kernel launches.  All compute is in the kernels of
-// pool.cuh, select.cuh and attn.cuh; nothing here touches tensor data on the host.
+// pool.cuh, select.cuh, attn.cuh, rope.cuh, fp8.cuh and nvfp4.cuh; nothing here touches tensor
+// data on the host.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -17,6 +18,7 @@
 #include "attn.cuh"
 #include "common.cuh"
 #include "fp8.cuh"
+#include "nvfp4.cuh"
 #include "pool.cuh"
 #include "ptx.cuh"
 #include "rope.cuh"
@@ -138,6 +140,29 @@ sbsa_status make_map_means(CUtensorMap* m, const float* base, long long rows, in
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(SBSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
     return SBSA_OK;
+}
+
+// NVFP4 codes [rows][K/2] bytes, box = 128 bytes (256 codes) x box_rows, 128-byte swizzle;
+// rows beyond the matrix read as zero codes.
+sbsa_status make_map_fp4(CUtensorMap* m, const void* base, long long rows, int K, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(SBSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+    cuuint32_t box[2] = {128, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SBSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return SBSA_OK;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 148;
+    return n > 0 ? n : 148;
 }
 
 std::atomic<unsigned int> g_epoch{1};
@@ -521,6 +546,85 @@ sbsa_status sbsa_attention_fwd_fp8(const sbsa_shape* shape, const void* q8, cons
             ? launch_attn_t<128, 128, true>(shape, q8, k8, v, row_ptr, col_idx, sc, o, st, q_scale, k_scale)
             : launch_attn_t<128, 64, true>(shape, q8, k8, v, row_ptr, col_idx, sc, o, st, q_scale, k_scale);
     if (r != SBSA_OK) return r;
+    return ok();
+}
+
+size_t sbsa_nvfp4_scale_bytes(int64_t rows, int32_t cols) {
+    if (rows < 1 || cols < 64 || cols % 64) return 0;
+    return static_cast<size_t>((rows + 127) / 128 * 128) * static_cast<size_t>(cols / 16);
+}
+
+sbsa_status sbsa_nvfp4_amax(const void* x, int64_t rows, int32_t cols, float* amax, void* stream) {
+    if (!x || !amax) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (rows < 1 || cols < 8 || cols % 8) return fail(SBSA_ERR_INVALID_ARG, "rows >= 1 and cols a multiple of 8 required");
+    if (!aligned16(x) || (reinterpret_cast<uintptr_t>(amax) & 3u))
+        return fail(SBSA_ERR_INVALID_ARG, "x must be 16-byte and amax 4-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), st);
+    if (e != cudaSuccess) return cuda_fail(e, "amax reset");
+    const long long n8 = rows * static_cast<long long>(cols) / 8;
+    const long long want = (n8 + 255) / 256;
+    const unsigned grid = static_cast<unsigned>(want < 8LL * sm_count() ? want : 8LL * sm_count());
+    nvfp4_amax_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(x), n8, reinterpret_cast<unsigned int*>(amax));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+    return ok();
+}
+
+sbsa_status sbsa_nvfp4_quantize(const void* x, int64_t rows, int32_t cols, const float* amax, void* codes,
+                                void* scales, void* stream) {
+    if (!x || !amax || !codes || !scales) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (rows < 1 || cols < 64 || cols % 64) return fail(SBSA_ERR_INVALID_ARG, "rows >= 1 and cols a multiple of 64 required");
+    if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(amax) & 3u))
+        return fail(SBSA_ERR_INVALID_ARG, "x and codes must be 16-byte aligned, amax 4-byte aligned");
+    const long long rows_p = (rows + 127) / 128 * 128;
+    const long long n_threads = rows_p * (cols / 16);
+    const long long grid = (n_threads + 255) / 256;
+    if (grid > 0x7FFFFFFFLL) return fail(SBSA_ERR_UNSUPPORTED, "matrix too large");
+    nvfp4_quantize_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(x), amax, static_cast<uint2*>(codes), static_cast<uint8_t*>(scales), rows, cols,
+        n_threads);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "nvfp4 quantize launch");
+    return ok();
+}
+
+sbsa_status sbsa_nvfp4_gemm(int32_t m, int32_t n, int32_t k, const void* a, const void* a_scales, const float* a_amax,
+                            const void* b, const void* b_scales, const float* b_amax, const float* bias, void* c,
+                            void* stream) {
+    if (!a || !a_scales || !a_amax || !b || !b_scales || !b_amax || !c) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (m < 1 || n < 8 || n % 8 || k < kFp4TileK || k % kFp4TileK)
+        return fail(SBSA_ERR_INVALID_ARG, "need m >= 1, n a multiple of 8, k a multiple of 256");
+    if (!aligned16(a) || !aligned16(b) || !aligned16(c) || !aligned16(a_scales) || !aligned16(b_scales))
+        return fail(SBSA_ERR_INVALID_ARG, "codes, scales and c must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(a_amax) | reinterpret_cast<uintptr_t>(b_amax) |
+         reinterpret_cast<uintptr_t>(bias)) & 3u)
+        return fail(SBSA_ERR_INVALID_ARG, "amax and bias must be 4-byte aligned");
+    CUtensorMap ma, mb;
+    sbsa_status r;
+    if ((r = make_map_fp4(&ma, a, m, k, kFp4TileM)) != SBSA_OK) return r;
+    if ((r = make_map_fp4(&mb, b, n, k, kFp4TileN)) != SBSA_OK) return r;
+    Nvfp4GemmParams p;
+    p.sfa = static_cast<const uint8_t*>(a_scales);
+    p.sfb = static_cast<const uint8_t*>(b_scales);
+    p.amax_a = a_amax;
+    p.amax_b = b_amax;
+    p.bias = bias;
+    p.c = static_cast<__nv_bfloat16*>(c);
+    p.M = m;
+    p.N = n;
+    p.K = k;
+    p.tiles_m = (m + kFp4TileM - 1) / kFp4TileM;
+    p.tiles_n = (n + kFp4TileN - 1) / kFp4TileN;
+    p.epoch = g_epoch.fetch_add(1);
+    const long long tiles = static_cast<long long>(p.tiles_m) * p.tiles_n;
+    if (tiles > 0x7FFFFFFFLL) return fail(SBSA_ERR_UNSUPPORTED, "too many tiles");
+    const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
+    cudaError_t e = cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFp4SmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "nvfp4 gemm smem attribute");
+    nvfp4_gemm_kernel<<<grid, kFp4Threads, kFp4SmemBytes, static_cast<cudaStream_t>(stream)>>>(ma, mb, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "nvfp4 gemm launch");
     return ok();
 }
 

@@ -25,7 +25,8 @@ EXPORTS = ("sbsa_version", "sbsa_status_string", "sbsa_last_error_message", "sbs
            "sbsa_workspace_bytes", "sbsa_pool_qk", "sbsa_select_blocks", "sbsa_attention_fwd", "sbsa_forward",
            "sbsa_check", "sbsa_validate_csr", "sbsa_forward_noalloc", "sbsa_rope_table_floats",
            "sbsa_rope_table_init", "sbsa_rope_pool_qk", "sbsa_key_mean", "sbsa_quantize_qk_fp8",
-           "sbsa_attention_fwd_fp8")
+           "sbsa_attention_fwd_fp8", "sbsa_nvfp4_scale_bytes", "sbsa_nvfp4_amax", "sbsa_nvfp4_quantize",
+           "sbsa_nvfp4_gemm")
 
 
 class SbsaError(RuntimeError):
@@ -93,9 +94,15 @@ def load(path: str | None = None):
     lib.sbsa_key_mean.argtypes = [SP, P, P, P]
     lib.sbsa_quantize_qk_fp8.argtypes = [SP, P, P, P, P, P, P, P, P]
     lib.sbsa_attention_fwd_fp8.argtypes = [SP, P, P, P, P, P, P, P, ctypes.c_float, P, P]
+    lib.sbsa_nvfp4_scale_bytes.argtypes = [ctypes.c_int64, I32]
+    lib.sbsa_nvfp4_scale_bytes.restype = SZ
+    lib.sbsa_nvfp4_amax.argtypes = [P, ctypes.c_int64, I32, P, P]
+    lib.sbsa_nvfp4_quantize.argtypes = [P, ctypes.c_int64, I32, P, P, P, P]
+    lib.sbsa_nvfp4_gemm.argtypes = [I32, I32, I32, P, P, P, P, P, P, P, P, P]
     for name in ("sbsa_pool_qk", "sbsa_select_blocks", "sbsa_attention_fwd", "sbsa_forward", "sbsa_check",
                  "sbsa_validate_csr", "sbsa_forward_noalloc", "sbsa_rope_table_init", "sbsa_rope_pool_qk",
-                 "sbsa_key_mean", "sbsa_quantize_qk_fp8", "sbsa_attention_fwd_fp8"):
+                 "sbsa_key_mean", "sbsa_quantize_qk_fp8", "sbsa_attention_fwd_fp8", "sbsa_nvfp4_amax",
+                 "sbsa_nvfp4_quantize", "sbsa_nvfp4_gemm"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -220,6 +227,46 @@ def sbsa_attention_fwd_fp8(shape: Shape, q8, k8, v, q_scale, k_scale, row_ptr, c
                                             _dev(k_scale, torch.float32, "k_scale"),
                                             _dev(row_ptr, torch.int32, "row_ptr"), _dev(col_idx, torch.int32, "col_idx"),
                                             float(scale), _dev(o, torch.bfloat16, "o"), _stream(stream)))
+
+
+def sbsa_nvfp4_scale_bytes(rows: int, cols: int) -> int:
+    return int(load().sbsa_nvfp4_scale_bytes(rows, cols))
+
+
+def sbsa_nvfp4_amax(x, amax, stream=None):
+    """amax (1-element fp32 CUDA tensor) = max |x| over a bf16 [rows, cols] CUDA tensor."""
+    rows, cols = x.shape
+    _check_numel(amax, 1, "amax")
+    _raise_on(load().sbsa_nvfp4_amax(_dev(x, torch.bfloat16, "x"), rows, cols, _dev(amax, torch.float32, "amax"),
+                                     _stream(stream)))
+
+
+def sbsa_nvfp4_quantize(x, amax, codes, scales, stream=None):
+    """bf16 [rows, cols] -> codes (uint8, rows*cols/2) and scales (uint8, sbsa_nvfp4_scale_bytes)."""
+    rows, cols = x.shape
+    _check_numel(amax, 1, "amax")
+    _check_numel(codes, rows * cols // 2, "codes")
+    _check_numel(scales, sbsa_nvfp4_scale_bytes(rows, cols), "scales")
+    _raise_on(load().sbsa_nvfp4_quantize(_dev(x, torch.bfloat16, "x"), rows, cols, _dev(amax, torch.float32, "amax"),
+                                         _dev(codes, torch.uint8, "codes"), _dev(scales, torch.uint8, "scales"),
+                                         _stream(stream)))
+
+
+def sbsa_nvfp4_gemm(m: int, n: int, k: int, a, a_scales, a_amax, b, b_scales, b_amax, bias, c, stream=None):
+    """c [m, n] bf16 = A B^T / (s_A s_B) + bias, A [m, k] and B [n, k] as NVFP4 codes + scales."""
+    _check_numel(a, m * k // 2, "a")
+    _check_numel(b, n * k // 2, "b")
+    _check_numel(a_scales, sbsa_nvfp4_scale_bytes(m, k), "a_scales")
+    _check_numel(b_scales, sbsa_nvfp4_scale_bytes(n, k), "b_scales")
+    _check_numel(c, m * n, "c")
+    bp = None
+    if bias is not None:
+        _check_numel(bias, n, "bias")
+        bp = _dev(bias, torch.float32, "bias")
+    _raise_on(load().sbsa_nvfp4_gemm(m, n, k, _dev(a, torch.uint8, "a"), _dev(a_scales, torch.uint8, "a_scales"),
+                                     _dev(a_amax, torch.float32, "a_amax"), _dev(b, torch.uint8, "b"),
+                                     _dev(b_scales, torch.uint8, "b_scales"), _dev(b_amax, torch.float32, "b_amax"),
+                                     bp, _dev(c, torch.bfloat16, "c"), _stream(stream)))
 
 
 def sbsa_select_blocks(shape: Shape, q_mean, k_mean, k_keep: int, row_ptr, col_idx, stream=None):
