@@ -627,3 +627,54 @@ def test_nvfp4_gemm_close_to_unquantized():
     rel = np.linalg.norm(c - ref) / np.linalg.norm(ref)
     # per-element relative error of e2m1 with block scales is ~ 1/12 rms; two operands
     assert 0.02 < rel < 0.2, rel
+
+
+# ---------------------------------------------------------------- Light-Ulysses exchange
+
+def _bits_of(x):
+    return (np.asarray(x, dtype=np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_row_quantizer_scale_and_round_trip():
+    rng = np.random.default_rng(51)
+    rows = rng.standard_normal((33, 64)).astype(np.float32)
+    rows[4] = 0.0
+    codes, scales = oracle.quantize_rows_fp8(rows)
+    amax = np.abs(rows).max(axis=1)
+    np.testing.assert_array_equal(scales[amax > 0], (amax / np.float32(448.0)).astype(np.float32)[amax > 0])
+    assert scales[4] == 1.0 and np.all(codes[4] == 0)
+    # every row's largest element lands on +-448
+    assert np.all(np.isin(codes[amax > 0], [0x7E, 0xFE]).any(axis=1))
+    back = (oracle.dequantize_rows_bf16(codes, scales).astype(np.uint32) << 16).view(np.float32)
+    err = np.abs(back.astype(np.float64) - rows)
+    # e4m3 half-quantum (2^-4 relative, 2^-10 * scale below the normal range) + one bf16 rounding
+    bound = np.maximum(np.abs(rows) * 2.0 ** -4, scales[:, None] * 2.0 ** -10) * (1 + 2.0 ** -7) + np.abs(rows) * 2.0 ** -8
+    assert np.all(err <= bound)
+
+
+def test_ulysses_exchange_by_hand():
+    # G = 2 ranks, H = 2 heads, L = 4 tokens (2 per rank), d = 2; values exact in e4m3 and bf16:
+    # x[t, c, h, :] = [448 * s, 56 * s] with s = 2^-(t + c + h) (one row, one scale each)
+    G, H, L, d = 2, 2, 4, 2
+    x = np.zeros((L, 3, H, d), dtype=np.float32)
+    for t in range(L):
+        for c in range(3):
+            for h in range(H):
+                s = 2.0 ** -(t + c + h)
+                x[t, c, h] = [448.0 * s, -56.0 * s]
+    shards = [_bits_of(x[0:2]), _bits_of(x[2:4])]
+    out = oracle.ulysses_qkv(shards, H, L, Lp=6)
+    for r in range(G):
+        got = (out[r].astype(np.uint32) << 16).view(np.float32)
+        assert got.shape == (3, 1, 6, d)
+        # rank r holds head r of all four tokens, padded tokens 4 and 5 zero
+        for c in range(3):
+            for t in range(L):
+                np.testing.assert_array_equal(got[c, 0, t], x[t, c, r])
+            assert np.all(got[c, 0, 4:] == 0)
+    # the return exchange puts every head of a rank's own tokens back
+    o_shards = [out[r][0, :, :, :] for r in range(G)]  # the q rows of each rank's head, as "attention output"
+    back = oracle.ulysses_o(o_shards, H, L)
+    for r in range(G):
+        got = (back[r].astype(np.uint32) << 16).view(np.float32)
+        np.testing.assert_array_equal(got, x[2 * r:2 * r + 2, 0, :, :])
