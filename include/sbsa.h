@@ -219,6 +219,51 @@ sbsa_status sbsa_nvfp4_gemm(int32_t m, int32_t n, int32_t k, const void *a, cons
                             const void *b, const void *b_scales, const float *b_amax, const float *bias, void *c,
                             void *stream);
 
+/* ---- Light-Ulysses sequence parallelism ------------------------------------------------
+ * Page "知识卡片：600倍加速，720p视频实时生成！单卡也能带的动14B模型", 方法/产品要点, bullet
+ * Light-Ulysses 多卡并行; page "单卡 RTX 5090 跑 Wan2.2-A14B：720p 视频生成只要 3.8 秒",
+ * 四步拆解 item 4: Ulysses-style sequence parallelism with an FP8 payload, Q, K and V fused
+ * into one all-to-all, fused pre/post-processing kernels and a head-level pipeline.
+ * These calls are the pre/post-processing; the all-to-all itself is the caller's (NCCL).
+ *
+ * `world` ranks; before the attention rank r holds tokens [r L/world, (r+1) L/world), during
+ * it heads [r H/world, (r+1) H/world).  A head chunk (head0, head_chunk) selects heads
+ * head0 .. head0 + head_chunk - 1 of every rank's H/world (one step of the head-level
+ * pipeline; head0 = 0, head_chunk = H/world for the whole exchange).  Every row of
+ * head_dim = 128 values crosses as 128 e4m3 codes and one fp32 scale: scale = amax/448,
+ * code = e4m3(x * (448/amax)) in fp32, nearest even, saturating (an all-zero row: scale 1,
+ * codes 0); the receiver restores bf16(code * scale).
+ *
+ * Buffers: `send`/`recv` hold `world` equal slices in rank order, each slice its codes then
+ * its scales.  QKV slice for peer j: codes [L/world][3][head_chunk][128], scales
+ * [L/world][3][head_chunk] (fp32); O slice: codes [L/world][head_chunk][128], scales
+ * [L/world][head_chunk].  The all-to-all sends slice j of `send` to rank j and writes the
+ * slice from rank i at slice i of `recv`.
+ *   x: [L/world][3][H][128] bf16 (the fused QKV activation of this rank's tokens)
+ *   q, k, v, o: [H/world][tokens_padded][128] bf16 (the attention layout; unpack writes
+ *     the chunk's heads, tokens >= L as zero)
+ *   y: [L/world][H][128] bf16 (every head of this rank's tokens)
+ * Device pointers owned by the caller, 16-byte aligned; asynchronous on `stream`;
+ * argument errors before any launch.  *_bytes return 0 for invalid arguments. */
+typedef struct {
+    int32_t world;          /* ranks G */
+    int32_t tokens;         /* L, a multiple of world */
+    int32_t tokens_padded;  /* rows of the attention layout, >= L */
+    int32_t heads;          /* H, a multiple of world */
+    int32_t head_dim;       /* 128 */
+} sbsa_ulysses_shape;
+
+size_t sbsa_ulysses_qkv_bytes(const sbsa_ulysses_shape *shape, int32_t head_chunk);
+size_t sbsa_ulysses_o_bytes(const sbsa_ulysses_shape *shape, int32_t head_chunk);
+sbsa_status sbsa_ulysses_pack_qkv(const sbsa_ulysses_shape *shape, int32_t head0, int32_t head_chunk, const void *x,
+                                  void *send, void *stream);
+sbsa_status sbsa_ulysses_unpack_qkv(const sbsa_ulysses_shape *shape, int32_t head0, int32_t head_chunk,
+                                    const void *recv, void *q, void *k, void *v, void *stream);
+sbsa_status sbsa_ulysses_pack_o(const sbsa_ulysses_shape *shape, int32_t head0, int32_t head_chunk, const void *o,
+                                void *send, void *stream);
+sbsa_status sbsa_ulysses_unpack_o(const sbsa_ulysses_shape *shape, int32_t head0, int32_t head_chunk,
+                                  const void *recv, void *y, void *stream);
+
 /* Steps 1-3 in one call on one stream: pool -> select -> attend, with the means and
  * the CSR lists carved out of `workspace` (device, 256-byte aligned, at least
  * sbsa_workspace_bytes(shape, k_keep) bytes).  If col_idx_out is non-NULL the

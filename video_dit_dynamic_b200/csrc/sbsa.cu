@@ -1,7 +1,7 @@
 // C ABI of the sbsa library (declared in include/sbsa.h): argument checking, tensor-map
 // encoding, workspace carving and kernel launches.  All compute is in the kernels of
-// pool.cuh, select.cuh, attn.cuh, rope.cuh, fp8.cuh and nvfp4.cuh; nothing here touches tensor
-// data on the host.
+// pool.cuh, select.cuh, attn.cuh, rope.cuh, fp8.cuh, nvfp4.cuh and ulysses.cuh; nothing here
+// touches tensor data on the host.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -23,6 +23,7 @@
 #include "ptx.cuh"
 #include "rope.cuh"
 #include "select.cuh"
+#include "ulysses.cuh"
 
 namespace sbsa {
 namespace {
@@ -166,6 +167,30 @@ int sm_count() {
 }
 
 std::atomic<unsigned int> g_epoch{1};
+
+// Light-Ulysses dimensions of one head chunk, or an error
+sbsa_status ulysses_dims(const sbsa_ulysses_shape* s, int32_t head0, int32_t head_chunk, UlyssesDims* u) {
+    if (!s) return fail(SBSA_ERR_INVALID_ARG, "shape is NULL");
+    if (s->world < 1 || s->tokens < 1 || s->heads < 1) return fail(SBSA_ERR_INVALID_ARG, "world, tokens, heads >= 1");
+    if (s->head_dim != kUlyD) return fail(SBSA_ERR_UNSUPPORTED, "head_dim must be 128");
+    if (s->tokens % s->world || s->heads % s->world)
+        return fail(SBSA_ERR_INVALID_ARG, "tokens and heads must be multiples of world");
+    if (s->tokens_padded < s->tokens) return fail(SBSA_ERR_INVALID_ARG, "tokens_padded < tokens");
+    const int hg = s->heads / s->world;
+    if (head0 < 0 || head_chunk < 1 || head0 + head_chunk > hg)
+        return fail(SBSA_ERR_INVALID_ARG, "head chunk outside [0, heads / world)");
+    u->G = s->world;
+    u->Lr = s->tokens / s->world;
+    u->L = s->tokens;
+    u->Lp = s->tokens_padded;
+    u->H = s->heads;
+    u->Hg = hg;
+    u->h0 = head0;
+    u->hc = head_chunk;
+    return SBSA_OK;
+}
+
+bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
 
 // ---------------------------------------------------------------- launchers
 sbsa_status launch_pool(const sbsa_shape* s, const void* q, const void* k, float* qm, float* km, cudaStream_t st) {
@@ -547,6 +572,80 @@ sbsa_status sbsa_attention_fwd_fp8(const sbsa_shape* shape, const void* q8, cons
             : launch_attn_t<128, 64, true>(shape, q8, k8, v, row_ptr, col_idx, sc, o, st, q_scale, k_scale);
     if (r != SBSA_OK) return r;
     return ok();
+}
+
+size_t sbsa_ulysses_qkv_bytes(const sbsa_ulysses_shape* shape, int32_t head_chunk) {
+    UlyssesDims u;
+    if (ulysses_dims(shape, 0, head_chunk, &u) != SBSA_OK) return 0;
+    return static_cast<size_t>(u.G) * ulysses_qkv_slice_bytes(u);
+}
+
+size_t sbsa_ulysses_o_bytes(const sbsa_ulysses_shape* shape, int32_t head_chunk) {
+    UlyssesDims u;
+    if (ulysses_dims(shape, 0, head_chunk, &u) != SBSA_OK) return 0;
+    return static_cast<size_t>(u.G) * ulysses_o_slice_bytes(u);
+}
+
+sbsa_status sbsa_ulysses_pack_qkv(const sbsa_ulysses_shape* shape, int32_t head0, int32_t head_chunk, const void* x,
+                                  void* send, void* stream) {
+    UlyssesDims u;
+    sbsa_status r = ulysses_dims(shape, head0, head_chunk, &u);
+    if (r != SBSA_OK) return r;
+    if (!x || !send) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(x) || !aligned16(send)) return fail(SBSA_ERR_INVALID_ARG, "x and send must be 16-byte aligned");
+    const long long warps = static_cast<long long>(u.G) * u.Lr * 3 * u.hc;
+    const long long grid = (warps + kUlyWarps - 1) / kUlyWarps;
+    ulysses_pack_qkv_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<uint8_t*>(send), u);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "ulysses pack launch");
+}
+
+sbsa_status sbsa_ulysses_unpack_qkv(const sbsa_ulysses_shape* shape, int32_t head0, int32_t head_chunk,
+                                    const void* recv, void* q, void* k, void* v, void* stream) {
+    UlyssesDims u;
+    sbsa_status r = ulysses_dims(shape, head0, head_chunk, &u);
+    if (r != SBSA_OK) return r;
+    if (!recv || !q || !k || !v) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(recv) || !aligned16(q) || !aligned16(k) || !aligned16(v))
+        return fail(SBSA_ERR_INVALID_ARG, "recv, q, k, v must be 16-byte aligned");
+    const long long warps = static_cast<long long>(u.G) * u.Lr * 3 * u.hc + 3LL * u.hc * (u.Lp - u.L);
+    const long long grid = (warps + kUlyWarps - 1) / kUlyWarps;
+    ulysses_unpack_qkv_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint8_t*>(recv), static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k),
+        static_cast<__nv_bfloat16*>(v), u);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "ulysses unpack launch");
+}
+
+sbsa_status sbsa_ulysses_pack_o(const sbsa_ulysses_shape* shape, int32_t head0, int32_t head_chunk, const void* o,
+                                void* send, void* stream) {
+    UlyssesDims u;
+    sbsa_status r = ulysses_dims(shape, head0, head_chunk, &u);
+    if (r != SBSA_OK) return r;
+    if (!o || !send) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(o) || !aligned16(send)) return fail(SBSA_ERR_INVALID_ARG, "o and send must be 16-byte aligned");
+    const long long warps = static_cast<long long>(u.G) * u.Lr * u.hc;
+    const long long grid = (warps + kUlyWarps - 1) / kUlyWarps;
+    ulysses_pack_o_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<uint8_t*>(send), u);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "ulysses pack_o launch");
+}
+
+sbsa_status sbsa_ulysses_unpack_o(const sbsa_ulysses_shape* shape, int32_t head0, int32_t head_chunk,
+                                  const void* recv, void* y, void* stream) {
+    UlyssesDims u;
+    sbsa_status r = ulysses_dims(shape, head0, head_chunk, &u);
+    if (r != SBSA_OK) return r;
+    if (!recv || !y) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(recv) || !aligned16(y)) return fail(SBSA_ERR_INVALID_ARG, "recv and y must be 16-byte aligned");
+    const long long warps = static_cast<long long>(u.G) * u.Lr * u.hc;
+    const long long grid = (warps + kUlyWarps - 1) / kUlyWarps;
+    ulysses_unpack_o_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint8_t*>(recv), static_cast<__nv_bfloat16*>(y), u);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "ulysses unpack_o launch");
 }
 
 size_t sbsa_nvfp4_scale_bytes(int64_t rows, int32_t cols) {

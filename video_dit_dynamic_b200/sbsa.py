@@ -26,13 +26,19 @@ EXPORTS = ("sbsa_version", "sbsa_status_string", "sbsa_last_error_message", "sbs
            "sbsa_check", "sbsa_validate_csr", "sbsa_forward_noalloc", "sbsa_rope_table_floats",
            "sbsa_rope_table_init", "sbsa_rope_pool_qk", "sbsa_key_mean", "sbsa_quantize_qk_fp8",
            "sbsa_attention_fwd_fp8", "sbsa_nvfp4_scale_bytes", "sbsa_nvfp4_amax", "sbsa_nvfp4_quantize",
-           "sbsa_nvfp4_gemm")
+           "sbsa_nvfp4_gemm", "sbsa_ulysses_qkv_bytes", "sbsa_ulysses_o_bytes", "sbsa_ulysses_pack_qkv",
+           "sbsa_ulysses_unpack_qkv", "sbsa_ulysses_pack_o", "sbsa_ulysses_unpack_o")
 
 
 class SbsaError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
         self.status = status
+
+
+class UlyssesShape(ctypes.Structure):
+    _fields_ = [("world", ctypes.c_int32), ("tokens", ctypes.c_int32), ("tokens_padded", ctypes.c_int32),
+                ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
 
 
 class Shape(ctypes.Structure):
@@ -99,6 +105,17 @@ def load(path: str | None = None):
     lib.sbsa_nvfp4_amax.argtypes = [P, ctypes.c_int64, I32, P, P]
     lib.sbsa_nvfp4_quantize.argtypes = [P, ctypes.c_int64, I32, P, P, P, P]
     lib.sbsa_nvfp4_gemm.argtypes = [I32, I32, I32, P, P, P, P, P, P, P, P, P]
+    UP = ctypes.POINTER(UlyssesShape)
+    lib.sbsa_ulysses_qkv_bytes.argtypes = [UP, I32]
+    lib.sbsa_ulysses_qkv_bytes.restype = SZ
+    lib.sbsa_ulysses_o_bytes.argtypes = [UP, I32]
+    lib.sbsa_ulysses_o_bytes.restype = SZ
+    lib.sbsa_ulysses_pack_qkv.argtypes = [UP, I32, I32, P, P, P]
+    lib.sbsa_ulysses_unpack_qkv.argtypes = [UP, I32, I32, P, P, P, P, P]
+    lib.sbsa_ulysses_pack_o.argtypes = [UP, I32, I32, P, P, P]
+    lib.sbsa_ulysses_unpack_o.argtypes = [UP, I32, I32, P, P, P]
+    for name in ("sbsa_ulysses_pack_qkv", "sbsa_ulysses_unpack_qkv", "sbsa_ulysses_pack_o", "sbsa_ulysses_unpack_o"):
+        getattr(lib, name).restype = ctypes.c_int
     for name in ("sbsa_pool_qk", "sbsa_select_blocks", "sbsa_attention_fwd", "sbsa_forward", "sbsa_check",
                  "sbsa_validate_csr", "sbsa_forward_noalloc", "sbsa_rope_table_init", "sbsa_rope_pool_qk",
                  "sbsa_key_mean", "sbsa_quantize_qk_fp8", "sbsa_attention_fwd_fp8", "sbsa_nvfp4_amax",
@@ -227,6 +244,57 @@ def sbsa_attention_fwd_fp8(shape: Shape, q8, k8, v, q_scale, k_scale, row_ptr, c
                                             _dev(k_scale, torch.float32, "k_scale"),
                                             _dev(row_ptr, torch.int32, "row_ptr"), _dev(col_idx, torch.int32, "col_idx"),
                                             float(scale), _dev(o, torch.bfloat16, "o"), _stream(stream)))
+
+
+def make_ulysses_shape(world: int, tokens: int, tokens_padded: int, heads: int, head_dim: int = 128) -> UlyssesShape:
+    return UlyssesShape(world, tokens, tokens_padded, heads, head_dim)
+
+
+def sbsa_ulysses_qkv_bytes(shape: UlyssesShape, head_chunk: int) -> int:
+    return int(load().sbsa_ulysses_qkv_bytes(ctypes.byref(shape), head_chunk))
+
+
+def sbsa_ulysses_o_bytes(shape: UlyssesShape, head_chunk: int) -> int:
+    return int(load().sbsa_ulysses_o_bytes(ctypes.byref(shape), head_chunk))
+
+
+def _uly_sizes(shape: UlyssesShape):
+    lr, hg = shape.tokens // max(shape.world, 1), shape.heads // max(shape.world, 1)
+    return lr, hg
+
+
+def sbsa_ulysses_pack_qkv(shape: UlyssesShape, head0: int, head_chunk: int, x, send, stream=None):
+    lr, _ = _uly_sizes(shape)
+    _check_numel(x, lr * 3 * shape.heads * shape.head_dim, "x")
+    _check_numel(send, sbsa_ulysses_qkv_bytes(shape, head_chunk), "send")
+    _raise_on(load().sbsa_ulysses_pack_qkv(ctypes.byref(shape), head0, head_chunk, _dev(x, torch.bfloat16, "x"),
+                                           _dev(send, torch.uint8, "send"), _stream(stream)))
+
+
+def sbsa_ulysses_unpack_qkv(shape: UlyssesShape, head0: int, head_chunk: int, recv, q, k, v, stream=None):
+    _, hg = _uly_sizes(shape)
+    _check_numel(recv, sbsa_ulysses_qkv_bytes(shape, head_chunk), "recv")
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        _check_numel(t, hg * shape.tokens_padded * shape.head_dim, nm)
+    _raise_on(load().sbsa_ulysses_unpack_qkv(ctypes.byref(shape), head0, head_chunk, _dev(recv, torch.uint8, "recv"),
+                                             _dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"),
+                                             _dev(v, torch.bfloat16, "v"), _stream(stream)))
+
+
+def sbsa_ulysses_pack_o(shape: UlyssesShape, head0: int, head_chunk: int, o, send, stream=None):
+    _, hg = _uly_sizes(shape)
+    _check_numel(o, hg * shape.tokens_padded * shape.head_dim, "o")
+    _check_numel(send, sbsa_ulysses_o_bytes(shape, head_chunk), "send")
+    _raise_on(load().sbsa_ulysses_pack_o(ctypes.byref(shape), head0, head_chunk, _dev(o, torch.bfloat16, "o"),
+                                         _dev(send, torch.uint8, "send"), _stream(stream)))
+
+
+def sbsa_ulysses_unpack_o(shape: UlyssesShape, head0: int, head_chunk: int, recv, y, stream=None):
+    lr, _ = _uly_sizes(shape)
+    _check_numel(recv, sbsa_ulysses_o_bytes(shape, head_chunk), "recv")
+    _check_numel(y, lr * shape.heads * shape.head_dim, "y")
+    _raise_on(load().sbsa_ulysses_unpack_o(ctypes.byref(shape), head0, head_chunk, _dev(recv, torch.uint8, "recv"),
+                                           _dev(y, torch.bfloat16, "y"), _stream(stream)))
 
 
 def sbsa_nvfp4_scale_bytes(rows: int, cols: int) -> int:
