@@ -51,6 +51,7 @@ def parse():
     ap.add_argument("--no-rope", action="store_true", help="skip timing the fused RoPE + pooling kernel")
     ap.add_argument("--no-fp8", action="store_true", help="skip timing the FP8 path")
     ap.add_argument("--no-nvfp4", action="store_true", help="skip timing the NVFP4 linear layer")
+    ap.add_argument("--no-ulysses", action="store_true", help="skip timing the Light-Ulysses kernels")
     ap.add_argument("--cpu-units", type=int, default=16, help="attention units in the CPU sample")
     return ap.parse_args()
 
@@ -505,6 +506,43 @@ def run_gpu(args, wl):
                "gemm_flop": 2.0 * fm * fn * fk}
         del xa, wb, bias4, a_codes, b_codes, a_sf, b_sf, c4
 
+    # Light-Ulysses pre/post-processing of the same layer: the four kernels around the two
+    # all-to-alls, over the whole layer (what G ranks do together, 1/G each)
+    uly = None
+    if not args.no_ulysses and wl.head_dim == 128:
+        ushape = sbsa.make_ulysses_shape(1, wl.seq_len, wl.seq_len_padded, wl.heads, wl.head_dim)
+        g5 = torch.Generator(device=dev).manual_seed(200 + rank)
+        xq = torch.randn(wl.seq_len, 3, wl.heads, wl.head_dim, generator=g5, device=dev).to(torch.bfloat16)
+        ub = sbsa.sbsa_ulysses_qkv_bytes(ushape, wl.heads)
+        ob = sbsa.sbsa_ulysses_o_bytes(ushape, wl.heads)
+        usend = torch.empty(ub, dtype=torch.uint8, device=dev)
+        uq, uk, uv = (torch.empty_like(q) for _ in range(3))
+        uy = torch.empty(wl.seq_len, wl.heads, wl.head_dim, dtype=torch.bfloat16, device=dev)
+        osend = torch.empty(ob, dtype=torch.uint8, device=dev)
+        calls = [
+            ("pack_qkv", lambda: sbsa.sbsa_ulysses_pack_qkv(ushape, 0, wl.heads, xq, usend, stream=stream),
+             xq.numel() * 2 + ub),
+            ("unpack_qkv", lambda: sbsa.sbsa_ulysses_unpack_qkv(ushape, 0, wl.heads, usend, uq, uk, uv, stream=stream),
+             ub + 3 * uq.numel() * 2),
+            ("pack_o", lambda: sbsa.sbsa_ulysses_pack_o(ushape, 0, wl.heads, uq, osend, stream=stream),
+             uy.numel() * 2 + ob),
+            ("unpack_o", lambda: sbsa.sbsa_ulysses_unpack_o(ushape, 0, wl.heads, osend, uy, stream=stream),
+             ob + uy.numel() * 2),
+        ]
+        uly = {}
+        for uname, ucall, nbytes in calls:
+            for _ in range(2):
+                ucall()
+            u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            u0.record(stream)
+            for _ in range(5):
+                ucall()
+            u1.record(stream)
+            torch.cuda.synchronize(dev)
+            uly[uname] = {"ms": u0.elapsed_time(u1) / 5, "algorithmic_bytes": nbytes}
+        sbsa.sbsa_check(stream)
+        del xq, usend, uq, uk, uv, uy, osend
+
     # end to end through the public API from pinned host buffers
     e2e = None
     if not args.no_e2e:
@@ -533,7 +571,8 @@ def run_gpu(args, wl):
                                  "fp8_quant": fp8["quant_ms"] if fp8 is not None else 0.0,
                                  "fp8_att": fp8["att_ms"] if fp8 is not None else 0.0,
                                  "fp4_quant": fp4["quant_ms"] if fp4 is not None else 0.0,
-                                 "fp4_gemm": fp4["gemm_ms"] if fp4 is not None else 0.0})
+                                 "fp4_gemm": fp4["gemm_ms"] if fp4 is not None else 0.0,
+                                 **({f"uly_{k}": v["ms"] for k, v in uly.items()} if uly is not None else {})})
     elapsed_ms, att_avg, pool_avg, sel_avg, forward_ms = (t[n] for n in ("elapsed", "att", "pool", "sel", "forward"))
     if e2e is not None:
         e2e["ms"] = t["e2e"]
@@ -543,6 +582,9 @@ def run_gpu(args, wl):
         fp8["quant_ms"], fp8["att_ms"] = t["fp8_quant"], t["fp8_att"]
     if fp4 is not None:
         fp4["quant_ms"], fp4["gemm_ms"] = t["fp4_quant"], t["fp4_gemm"]
+    if uly is not None:
+        for uname in uly:
+            uly[uname]["ms"] = t[f"uly_{uname}"]
     ms_step = elapsed_ms / args.steps
     value = job_tflops(flops, ws_n, ms_step)
 
@@ -580,6 +622,9 @@ def run_gpu(args, wl):
                    if rope is not None else {}),
                 **({"fp8": fp8_summary(fp8, flops, pool_avg + sel_avg, peaks)} if fp8 is not None else {}),
                 **({"nvfp4_linear": fp4_summary(fp4, peaks)} if fp4 is not None else {}),
+                **({"ulysses": {k: {**v, "GB/s": v["algorithmic_bytes"] / (v["ms"] / 1e3) / 1e9,
+                                    "hbm_frac": v["algorithmic_bytes"] / (v["ms"] / 1e3) / 1e9 / peaks["hbm_gbs"]}
+                                for k, v in uly.items()}} if uly is not None else {}),
             },
             "peaks": {"source": peak_src, **peaks},
         }

@@ -235,7 +235,7 @@ sbsa_status sbsa_nvfp4_gemm(int32_t m, int32_t n, int32_t k, const void *a, cons
  * codes 0); the receiver restores bf16(code * scale).
  *
  * Buffers: `send`/`recv` hold `world` equal slices in rank order, each slice its codes then
- * its scales.  QKV slice for peer j: codes [L/world][3][head_chunk][128], scales
+ * its scales, padded to a multiple of 16 bytes.  QKV slice for peer j: codes [L/world][3][head_chunk][128], scales
  * [L/world][3][head_chunk] (fp32); O slice: codes [L/world][head_chunk][128], scales
  * [L/world][head_chunk].  The all-to-all sends slice j of `send` to rank j and writes the
  * slice from rank i at slice i of `recv`.

@@ -187,6 +187,9 @@ sbsa_status ulysses_dims(const sbsa_ulysses_shape* s, int32_t head0, int32_t hea
     u->Hg = hg;
     u->h0 = head0;
     u->hc = head_chunk;
+    // the kernels index rows in 32 bits
+    const long long rows = static_cast<long long>(u->G) * u->Lr * 3 * u->hc + 3LL * u->hc * (u->Lp - u->L);
+    if (rows >= (1LL << 31)) return fail(SBSA_ERR_UNSUPPORTED, "head chunk of 2^31 rows or more");
     return SBSA_OK;
 }
 
@@ -594,7 +597,7 @@ sbsa_status sbsa_ulysses_pack_qkv(const sbsa_ulysses_shape* shape, int32_t head0
     if (!x || !send) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
     if (!aligned16(x) || !aligned16(send)) return fail(SBSA_ERR_INVALID_ARG, "x and send must be 16-byte aligned");
     const long long warps = static_cast<long long>(u.G) * u.Lr * 3 * u.hc;
-    const long long grid = (warps + kUlyWarps - 1) / kUlyWarps;
+    const long long grid = (warps + kUlyRowsPerCta - 1) / kUlyRowsPerCta;
     ulysses_pack_qkv_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const __nv_bfloat16*>(x), static_cast<uint8_t*>(send), u);
     cudaError_t e = cudaGetLastError();
@@ -610,7 +613,7 @@ sbsa_status sbsa_ulysses_unpack_qkv(const sbsa_ulysses_shape* shape, int32_t hea
     if (!aligned16(recv) || !aligned16(q) || !aligned16(k) || !aligned16(v))
         return fail(SBSA_ERR_INVALID_ARG, "recv, q, k, v must be 16-byte aligned");
     const long long warps = static_cast<long long>(u.G) * u.Lr * 3 * u.hc + 3LL * u.hc * (u.Lp - u.L);
-    const long long grid = (warps + kUlyWarps - 1) / kUlyWarps;
+    const long long grid = (warps + kUlyRowsPerCta - 1) / kUlyRowsPerCta;
     ulysses_unpack_qkv_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const uint8_t*>(recv), static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k),
         static_cast<__nv_bfloat16*>(v), u);
@@ -626,7 +629,7 @@ sbsa_status sbsa_ulysses_pack_o(const sbsa_ulysses_shape* shape, int32_t head0, 
     if (!o || !send) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
     if (!aligned16(o) || !aligned16(send)) return fail(SBSA_ERR_INVALID_ARG, "o and send must be 16-byte aligned");
     const long long warps = static_cast<long long>(u.G) * u.Lr * u.hc;
-    const long long grid = (warps + kUlyWarps - 1) / kUlyWarps;
+    const long long grid = (warps + kUlyRowsPerCta - 1) / kUlyRowsPerCta;
     ulysses_pack_o_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<uint8_t*>(send), u);
     cudaError_t e = cudaGetLastError();
@@ -641,7 +644,7 @@ sbsa_status sbsa_ulysses_unpack_o(const sbsa_ulysses_shape* shape, int32_t head0
     if (!recv || !y) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
     if (!aligned16(recv) || !aligned16(y)) return fail(SBSA_ERR_INVALID_ARG, "recv and y must be 16-byte aligned");
     const long long warps = static_cast<long long>(u.G) * u.Lr * u.hc;
-    const long long grid = (warps + kUlyWarps - 1) / kUlyWarps;
+    const long long grid = (warps + kUlyRowsPerCta - 1) / kUlyRowsPerCta;
     ulysses_unpack_o_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const uint8_t*>(recv), static_cast<__nv_bfloat16*>(y), u);
     cudaError_t e = cudaGetLastError();

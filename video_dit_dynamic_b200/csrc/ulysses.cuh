@@ -12,7 +12,7 @@
 //   an all-zero row has scale 1 and codes 0;  restored value = bf16(code * scale).
 //
 // Buffers (one chunk, bytes), one slice per peer, slices in rank order, each slice its
-// codes followed by its scales:
+// codes followed by its scales and padded to a multiple of 16 bytes:
 //   QKV slice for peer j: codes [L/G][3][hc][d], scales [L/G][3][hc]
 //   O   slice for peer j: codes [L/G][hc][d],    scales [L/G][hc]
 // Layouts around them:
@@ -22,6 +22,7 @@
 //   y  (all heads of this rank's tokens)             [L/G][H][d] bf16
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "fp8.cuh"
@@ -33,143 +34,217 @@ struct UlyssesDims {
     int G, Lr, L, Lp, H, Hg, h0, hc;
 };
 
-// e4m3 code -> exact fp32 value (sign, bias 7, three mantissa bits, subnormals m 2^-9)
-__device__ __forceinline__ float e4m3_signed_value(uint32_t code) {
-    const uint32_t e = (code >> 3) & 15u, m = code & 7u;
-    const float v = e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : static_cast<float>(m) * 0.001953125f;
-    return (code & 0x80u) ? -v : v;
-}
-
-// One warp quantizes one row of 128 bf16 values (4 per lane) into 128 codes (4 bytes per
-// lane) and one scale (lane 0).
-__device__ __forceinline__ void quantize_row_warp(const uint2* __restrict__ src, uint32_t* __restrict__ codes,
-                                                  float* __restrict__ scale, int lane) {
-    const uint2 w = src[lane];
-    float v[4] = {__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u), __uint_as_float(w.y << 16),
-                  __uint_as_float(w.y & 0xFFFF0000u)};
-    float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-    const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
-    const uint32_t lo = cvt_e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv));
-    const uint32_t hi = cvt_e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv));
-    codes[lane] = lo | (hi << 16);
-    if (lane == 0) *scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-}
-
-// One warp restores one row: 4 codes per lane -> 4 bf16 values.
-__device__ __forceinline__ void dequantize_row_warp(const uint32_t* __restrict__ codes, const float* __restrict__ scale,
-                                                    uint2* __restrict__ dst, int lane) {
-    const uint32_t c = codes[lane];
-    const float s = *scale;
-    const float v0 = __fmul_rn(e4m3_signed_value(c & 0xFFu), s);
-    const float v1 = __fmul_rn(e4m3_signed_value((c >> 8) & 0xFFu), s);
-    const float v2 = __fmul_rn(e4m3_signed_value((c >> 16) & 0xFFu), s);
-    const float v3 = __fmul_rn(e4m3_signed_value(c >> 24), s);
-    dst[lane] = make_uint2(pack_bf16x2(v0, v1), pack_bf16x2(v2, v3));
+// Two e4m3 codes (low byte first) -> their exact values as fp32 (e4m3 is a subset of
+// f16, so the hardware conversion to f16 is exact).
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two_codes) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(two_codes & 0xFFFFu)));
+    return __half22float2(*reinterpret_cast<const __half2*>(&h2));
 }
 
 constexpr int kUlyD = 128;          // head_dim handled by these kernels
-constexpr int kUlyWarps = 8;        // rows per 256-thread CTA
+constexpr int kUlyRowsPerWarp = 8;  // 16 lanes per row (8 values each), 4 row pairs per warp
+constexpr int kUlyRowsPerCta = 8 * kUlyRowsPerWarp;
 
+// slices are padded to 16 bytes, so every slice's codes start 16-byte aligned
 __host__ __device__ constexpr size_t ulysses_qkv_slice_bytes(const UlyssesDims& u) {
-    return static_cast<size_t>(u.Lr) * 3 * u.hc * (kUlyD + 4);
+    return (static_cast<size_t>(u.Lr) * 3 * u.hc * (kUlyD + 4) + 15) & ~size_t(15);
 }
 __host__ __device__ constexpr size_t ulysses_o_slice_bytes(const UlyssesDims& u) {
-    return static_cast<size_t>(u.Lr) * u.hc * (kUlyD + 4);
+    return (static_cast<size_t>(u.Lr) * u.hc * (kUlyD + 4) + 15) & ~size_t(15);
+}
+
+// Where row `row` of a pack goes and comes from.
+struct RowPtrs {
+    const uint4* src;  // 8 bf16 per lane (pack) or 8 codes per lane (unpack, as uint2)
+    void* dst;
+    float* scale;
+    bool zero;         // unpack only: a padded token, written as zeros
+};
+
+// Row decompositions use 32-bit unsigned arithmetic: the host refuses chunks of 2^31
+// rows or more.  Offsets are formed in 64 bits.
+__device__ __forceinline__ RowPtrs qkv_pack_row(uint32_t w, const __nv_bfloat16* x, uint8_t* send,
+                                                const UlyssesDims& u) {
+    const uint32_t per_peer = static_cast<uint32_t>(u.Lr) * 3u * static_cast<uint32_t>(u.hc);
+    const uint32_t j = w / per_peer;
+    const uint32_t row = w - j * per_peer;  // (t * 3 + c) * hc + hh
+    const uint32_t tc = row / static_cast<uint32_t>(u.hc);
+    const uint32_t hh = row - tc * static_cast<uint32_t>(u.hc);
+    uint8_t* slice = send + static_cast<size_t>(j) * ulysses_qkv_slice_bytes(u);
+    const size_t src = (static_cast<size_t>(tc) * u.H + j * u.Hg + u.h0 + hh) * kUlyD;
+    return {reinterpret_cast<const uint4*>(x + src), slice + static_cast<size_t>(row) * kUlyD,
+            reinterpret_cast<float*>(slice + static_cast<size_t>(per_peer) * kUlyD) + row, false};
+}
+
+__device__ __forceinline__ RowPtrs o_pack_row(uint32_t w, const __nv_bfloat16* o, uint8_t* send,
+                                              const UlyssesDims& u) {
+    const uint32_t per_peer = static_cast<uint32_t>(u.Lr) * static_cast<uint32_t>(u.hc);
+    const uint32_t j = w / per_peer;
+    const uint32_t row = w - j * per_peer;  // t * hc + hh
+    const uint32_t t = row / static_cast<uint32_t>(u.hc);
+    const uint32_t hh = row - t * static_cast<uint32_t>(u.hc);
+    const size_t token = static_cast<size_t>(j) * u.Lr + t;
+    uint8_t* slice = send + static_cast<size_t>(j) * ulysses_o_slice_bytes(u);
+    return {reinterpret_cast<const uint4*>(o + (static_cast<size_t>(u.h0 + hh) * u.Lp + token) * kUlyD),
+            slice + static_cast<size_t>(row) * kUlyD,
+            reinterpret_cast<float*>(slice + static_cast<size_t>(per_peer) * kUlyD) + row, false};
+}
+
+__device__ __forceinline__ RowPtrs qkv_unpack_row(uint32_t w, const uint8_t* recv, __nv_bfloat16* q,
+                                                  __nv_bfloat16* k, __nv_bfloat16* v, const UlyssesDims& u) {
+    const uint32_t per_peer = static_cast<uint32_t>(u.Lr) * 3u * static_cast<uint32_t>(u.hc);
+    const uint32_t n_rows = per_peer * static_cast<uint32_t>(u.G);
+    if (w < n_rows) {
+        const uint32_t i = w / per_peer;
+        const uint32_t row = w - i * per_peer;
+        const uint32_t tc = row / static_cast<uint32_t>(u.hc);
+        const uint32_t hh = row - tc * static_cast<uint32_t>(u.hc);
+        const uint32_t t3 = tc / 3u;
+        const uint32_t c = tc - 3u * t3;
+        __nv_bfloat16* t = c == 0 ? q : (c == 1 ? k : v);
+        const size_t token = static_cast<size_t>(i) * u.Lr + t3;
+        const uint8_t* slice = recv + static_cast<size_t>(i) * ulysses_qkv_slice_bytes(u);
+        return {reinterpret_cast<const uint4*>(slice + static_cast<size_t>(row) * kUlyD),
+                t + (static_cast<size_t>(u.h0 + hh) * u.Lp + token) * kUlyD,
+                const_cast<float*>(reinterpret_cast<const float*>(slice + static_cast<size_t>(per_peer) * kUlyD)) + row,
+                false};
+    }
+    const uint32_t z = w - n_rows;  // padded rows (c, hh, token - L)
+    const uint32_t pad = static_cast<uint32_t>(u.Lp - u.L);
+    const uint32_t per_c = static_cast<uint32_t>(u.hc) * pad;
+    const uint32_t c = z / per_c;
+    const uint32_t rem = z - c * per_c;
+    const uint32_t hh = rem / pad;
+    __nv_bfloat16* t = c == 0 ? q : (c == 1 ? k : v);
+    return {nullptr, t + (static_cast<size_t>(u.h0 + hh) * u.Lp + u.L + (rem - hh * pad)) * kUlyD, nullptr, true};
+}
+
+__device__ __forceinline__ RowPtrs o_unpack_row(uint32_t w, const uint8_t* recv, __nv_bfloat16* y,
+                                                const UlyssesDims& u) {
+    const uint32_t per_peer = static_cast<uint32_t>(u.Lr) * static_cast<uint32_t>(u.hc);
+    const uint32_t i = w / per_peer;
+    const uint32_t row = w - i * per_peer;
+    const uint32_t t = row / static_cast<uint32_t>(u.hc);
+    const uint32_t hh = row - t * static_cast<uint32_t>(u.hc);
+    const uint8_t* slice = recv + static_cast<size_t>(i) * ulysses_o_slice_bytes(u);
+    return {reinterpret_cast<const uint4*>(slice + static_cast<size_t>(row) * kUlyD),
+            y + (static_cast<size_t>(t) * u.H + i * u.Hg + u.h0 + hh) * kUlyD,
+            const_cast<float*>(reinterpret_cast<const float*>(slice + static_cast<size_t>(per_peer) * kUlyD)) + row,
+            false};
+}
+
+// Quantize rows [first, first + 8) of a pack (rows >= n_rows skipped): half-warp h takes
+// rows first + 2 s + h, lane l % 16 the 8 values 8 (l % 16) .. + 7; all loads are issued
+// before any is used.
+template <typename RowFn>
+__device__ __forceinline__ void pack_rows(uint32_t first, uint32_t n_rows, RowFn row_of) {
+    const int lane = threadIdx.x % 32, h = lane / 16, l = lane % 16;
+    uint4 in[4];
+    RowPtrs rp[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        const uint32_t w = first + 2u * s + h;
+        in[s] = make_uint4(0u, 0u, 0u, 0u);
+        if (w < n_rows) {
+            rp[s] = row_of(w);
+            in[s] = __ldg(rp[s].src + l);
+        }
+    }
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        const uint32_t w = first + 2u * s + h;
+        const uint32_t wd[4] = {in[s].x, in[s].y, in[s].z, in[s].w};
+        float vals[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            vals[2 * e] = __uint_as_float(wd[e] << 16);
+            vals[2 * e + 1] = __uint_as_float(wd[e] & 0xFFFF0000u);
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(vals[e]));
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+        if (w >= n_rows) continue;  // (after the shuffles, which every lane takes part in)
+        const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
+        uint32_t c2[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c2[e] = cvt_e4m3x2(__fmul_rn(vals[2 * e], inv), __fmul_rn(vals[2 * e + 1], inv));
+        reinterpret_cast<uint2*>(rp[s].dst)[l] = make_uint2(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16));
+        if (l == 0) *rp[s].scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    }
+}
+
+// Restore rows [first, first + 8) (rows >= n_rows skipped), same thread layout.
+template <typename RowFn>
+__device__ __forceinline__ void unpack_rows(uint32_t first, uint32_t n_rows, RowFn row_of) {
+    const int lane = threadIdx.x % 32, h = lane / 16, l = lane % 16;
+    uint2 in[4];
+    float sc[4];
+    RowPtrs rp[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        const uint32_t w = first + 2u * s + h;
+        if (w < n_rows) {
+            rp[s] = row_of(w);
+            if (!rp[s].zero) {
+                in[s] = __ldg(reinterpret_cast<const uint2*>(rp[s].src) + l);
+                sc[s] = __ldg(rp[s].scale);
+            }
+        }
+    }
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        const uint32_t w = first + 2u * s + h;
+        if (w >= n_rows) continue;
+        uint4 out = make_uint4(0u, 0u, 0u, 0u);
+        if (!rp[s].zero) {
+            const float2 a = e4m3x2_to_float2(in[s].x), b = e4m3x2_to_float2(in[s].x >> 16);
+            const float2 c = e4m3x2_to_float2(in[s].y), d = e4m3x2_to_float2(in[s].y >> 16);
+            const float k = sc[s];
+            out = make_uint4(pack_bf16x2(__fmul_rn(a.x, k), __fmul_rn(a.y, k)), pack_bf16x2(__fmul_rn(b.x, k), __fmul_rn(b.y, k)),
+                             pack_bf16x2(__fmul_rn(c.x, k), __fmul_rn(c.y, k)), pack_bf16x2(__fmul_rn(d.x, k), __fmul_rn(d.y, k)));
+        }
+        reinterpret_cast<uint4*>(rp[s].dst)[l] = out;
+    }
 }
 
 // x [Lr][3][H][d] -> send: slice j holds rows (t, c, hh) of head j Hg + h0 + hh.
 __global__ void __launch_bounds__(256) ulysses_pack_qkv_kernel(const __nv_bfloat16* __restrict__ x,
                                                                uint8_t* __restrict__ send, UlyssesDims u) {
-    const int lane = threadIdx.x % 32;
-    const long long w = blockIdx.x * static_cast<long long>(kUlyWarps) + threadIdx.x / 32;
-    const long long per_peer = static_cast<long long>(u.Lr) * 3 * u.hc;
-    if (w >= per_peer * u.G) return;
-    const int j = static_cast<int>(w / per_peer);
-    const long long row = w % per_peer;  // (t * 3 + c) * hc + hh
-    const int hh = static_cast<int>(row % u.hc);
-    const long long tc = row / u.hc;     // t * 3 + c
-    const int h = j * u.Hg + u.h0 + hh;
-    const uint2* src = reinterpret_cast<const uint2*>(x + (tc * u.H + h) * kUlyD);
-    uint8_t* slice = send + static_cast<size_t>(j) * ulysses_qkv_slice_bytes(u);
-    quantize_row_warp(src, reinterpret_cast<uint32_t*>(slice + row * kUlyD),
-                      reinterpret_cast<float*>(slice + per_peer * kUlyD) + row, lane);
+    const uint32_t first = blockIdx.x * kUlyRowsPerCta + (threadIdx.x / 32) * kUlyRowsPerWarp;
+    const uint32_t n_rows = static_cast<uint32_t>(u.G) * u.Lr * 3u * u.hc;
+    pack_rows(first, n_rows, [&](uint32_t w) { return qkv_pack_row(w, x, send, u); });
 }
 
 // recv (slice i from rank i) -> q, k, v [Hg][Lp][d]: row (t, c, hh) is token i Lr + t of
-// head h0 + hh of tensor c.  Warps past the received rows zero the padded tokens
-// [L, Lp) of the chunk's heads.
+// head h0 + hh of tensor c; after those rows come the padded tokens [L, Lp) of the
+// chunk's heads, written as zeros.
 __global__ void __launch_bounds__(256) ulysses_unpack_qkv_kernel(const uint8_t* __restrict__ recv,
                                                                  __nv_bfloat16* __restrict__ q,
                                                                  __nv_bfloat16* __restrict__ k,
                                                                  __nv_bfloat16* __restrict__ v, UlyssesDims u) {
-    const int lane = threadIdx.x % 32;
-    const long long w = blockIdx.x * static_cast<long long>(kUlyWarps) + threadIdx.x / 32;
-    const long long per_peer = static_cast<long long>(u.Lr) * 3 * u.hc;
-    const long long n_rows = per_peer * u.G;
-    if (w < n_rows) {
-        const int i = static_cast<int>(w / per_peer);
-        const long long row = w % per_peer;
-        const int hh = static_cast<int>(row % u.hc);
-        const long long tc = row / u.hc;
-        const int c = static_cast<int>(tc % 3);
-        const long long t = tc / 3;
-        __nv_bfloat16* dst_t = c == 0 ? q : (c == 1 ? k : v);
-        const long long token = static_cast<long long>(i) * u.Lr + t;
-        const uint8_t* slice = recv + static_cast<size_t>(i) * ulysses_qkv_slice_bytes(u);
-        dequantize_row_warp(reinterpret_cast<const uint32_t*>(slice + row * kUlyD),
-                            reinterpret_cast<const float*>(slice + per_peer * kUlyD) + row,
-                            reinterpret_cast<uint2*>(dst_t + (static_cast<long long>(u.h0 + hh) * u.Lp + token) * kUlyD),
-                            lane);
-        return;
-    }
-    const long long z = w - n_rows;  // padded rows: (c, hh, t - L)
-    const long long pad = u.Lp - u.L;
-    if (z >= 3 * u.hc * pad) return;
-    const int c = static_cast<int>(z / (u.hc * pad));
-    const long long rem = z % (u.hc * pad);
-    const int hh = static_cast<int>(rem / pad);
-    const long long token = u.L + rem % pad;
-    __nv_bfloat16* dst_t = c == 0 ? q : (c == 1 ? k : v);
-    reinterpret_cast<uint2*>(dst_t + (static_cast<long long>(u.h0 + hh) * u.Lp + token) * kUlyD)[lane] =
-        make_uint2(0u, 0u);
+    const uint32_t first = blockIdx.x * kUlyRowsPerCta + (threadIdx.x / 32) * kUlyRowsPerWarp;
+    const uint32_t n_rows = static_cast<uint32_t>(u.G) * u.Lr * 3u * u.hc + 3u * u.hc * (u.Lp - u.L);
+    unpack_rows(first, n_rows, [&](uint32_t w) { return qkv_unpack_row(w, recv, q, k, v, u); });
 }
 
 // o [Hg][Lp][d] -> send: slice j holds rows (t, hh) of token j Lr + t, head h0 + hh.
 __global__ void __launch_bounds__(256) ulysses_pack_o_kernel(const __nv_bfloat16* __restrict__ o,
                                                              uint8_t* __restrict__ send, UlyssesDims u) {
-    const int lane = threadIdx.x % 32;
-    const long long w = blockIdx.x * static_cast<long long>(kUlyWarps) + threadIdx.x / 32;
-    const long long per_peer = static_cast<long long>(u.Lr) * u.hc;
-    if (w >= per_peer * u.G) return;
-    const int j = static_cast<int>(w / per_peer);
-    const long long row = w % per_peer;  // t * hc + hh
-    const int hh = static_cast<int>(row % u.hc);
-    const long long t = row / u.hc;
-    const long long token = static_cast<long long>(j) * u.Lr + t;
-    const uint2* src = reinterpret_cast<const uint2*>(o + (static_cast<long long>(u.h0 + hh) * u.Lp + token) * kUlyD);
-    uint8_t* slice = send + static_cast<size_t>(j) * ulysses_o_slice_bytes(u);
-    quantize_row_warp(src, reinterpret_cast<uint32_t*>(slice + row * kUlyD),
-                      reinterpret_cast<float*>(slice + per_peer * kUlyD) + row, lane);
+    const uint32_t first = blockIdx.x * kUlyRowsPerCta + (threadIdx.x / 32) * kUlyRowsPerWarp;
+    const uint32_t n_rows = static_cast<uint32_t>(u.G) * u.Lr * u.hc;
+    pack_rows(first, n_rows, [&](uint32_t w) { return o_pack_row(w, o, send, u); });
 }
 
 // recv (slice i from rank i) -> y [Lr][H][d]: row (t, hh) is head i Hg + h0 + hh of
 // token t.
 __global__ void __launch_bounds__(256) ulysses_unpack_o_kernel(const uint8_t* __restrict__ recv,
                                                                __nv_bfloat16* __restrict__ y, UlyssesDims u) {
-    const int lane = threadIdx.x % 32;
-    const long long w = blockIdx.x * static_cast<long long>(kUlyWarps) + threadIdx.x / 32;
-    const long long per_peer = static_cast<long long>(u.Lr) * u.hc;
-    if (w >= per_peer * u.G) return;
-    const int i = static_cast<int>(w / per_peer);
-    const long long row = w % per_peer;
-    const int hh = static_cast<int>(row % u.hc);
-    const long long t = row / u.hc;
-    const uint8_t* slice = recv + static_cast<size_t>(i) * ulysses_o_slice_bytes(u);
-    dequantize_row_warp(reinterpret_cast<const uint32_t*>(slice + row * kUlyD),
-                        reinterpret_cast<const float*>(slice + per_peer * kUlyD) + row,
-                        reinterpret_cast<uint2*>(y + (t * u.H + i * u.Hg + u.h0 + hh) * kUlyD), lane);
+    const uint32_t first = blockIdx.x * kUlyRowsPerCta + (threadIdx.x / 32) * kUlyRowsPerWarp;
+    const uint32_t n_rows = static_cast<uint32_t>(u.G) * u.Lr * u.hc;
+    unpack_rows(first, n_rows, [&](uint32_t w) { return o_unpack_row(w, recv, y, u); });
 }
 
 }  // namespace sbsa

@@ -67,10 +67,11 @@ class UlyssesPlan:
         return [(h0, min(self.head_chunk, hg - h0)) for h0 in range(0, hg, self.head_chunk)]
 
     def qkv_slice_bytes(self, count: int) -> int:
-        return self.tokens_local * 3 * count * (self.head_dim + 4)
+        # codes then scales, padded to 16 bytes (the library's slice layout)
+        return (self.tokens_local * 3 * count * (self.head_dim + 4) + 15) // 16 * 16
 
     def o_slice_bytes(self, count: int) -> int:
-        return self.tokens_local * count * (self.head_dim + 4)
+        return (self.tokens_local * count * (self.head_dim + 4) + 15) // 16 * 16
 
 
 class CudaOps:
