@@ -412,4 +412,270 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
     }
 }
 
+// ---------------------------------------------------------------- GEMM on CTA pairs
+// The same product on pairs of CTAs (clusters of two) with tcgen05's two-CTA MMA: a
+// pair owns a 256 x 256 output tile.  CTA r of the pair loads rows 128 r .. + 127 of the
+// tile's A and of its B, the scales of its A rows and the scales of all 256 B rows; the
+// leader (r = 0) issues, for both CTAs, the scale copies into TMEM
+// (tcgen05.cp.cta_group::2) and the MMAs (tcgen05.mma.cta_group::2, M = 256, N = 256,
+// K = 64), which read A from each CTA's own shared memory and B from both, and leave
+// rows 128 r .. + 127 x 256 columns of the accumulator in CTA r's TMEM.  Each CTA moves
+// 38 KB per K-tile instead of the 54 KB of a 128 x 256 tile on one CTA, for the same
+// number of MMA cycles per SM.  Built when SBSA_NVFP4_PAIR is 1: parity-tested, but
+// measured slower than the one-CTA kernel above, whose bound is the scale copies into
+// TMEM (each SM still makes three per 128-cycle MMA), not the loads.
+//   Both CTAs' copies complete on the leader's stage barrier (two-CTA TMA), whose
+//   expected bytes the leader sets for both; the leader's commits arrive on the stage's
+//   free barrier and, at the end of a tile, the accumulator barrier of both CTAs; each
+//   CTA's epilogue hands the accumulator back by arriving on the leader's barrier.
+struct Nvfp4Gemm2Params {
+    const float* amax_a;
+    const float* amax_b;
+    const float* bias;  // [N] or null
+    __nv_bfloat16* c;   // [M][N]
+    int M, N, K;
+    int tiles_m, tiles_n;   // 256 x 256 tiles
+    int groups_a, groups_b; // 128-row scale groups of A and B
+    unsigned int epoch;
+};
+
+constexpr int kF2Stages = 5;
+constexpr int kF2Half = 128 * 128;                   // 128 rows x 128 bytes of codes
+constexpr int kF2SfaBytes = 4 * 512;                 // this CTA's A rows, one K-tile
+constexpr int kF2SfbBytes = 2 * 4 * 512;             // all 256 B rows of the tile, one K-tile
+constexpr int kF2StageBytes = 2 * kF2Half + kF2SfaBytes + kF2SfbBytes;
+constexpr int kF2BarOff = kF2Stages * kF2StageBytes;
+constexpr int kF2NumBars = 2 * kF2Stages + 3;  // full[S] (leader's counts both CTAs), empty[S], acc_full, acc_empty, drain
+constexpr int kF2SmemBytes = kF2BarOff + kF2NumBars * 8 + 16 + 1024;
+static_assert(kF2StageBytes % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
+static_assert(kF2SmemBytes <= 232448, "shared memory");
+
+__device__ __forceinline__ void umma_nvfp4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_cp_pair_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// Arrive on the barrier at this shared offset in both CTAs of the pair once the
+// tensor-core work issued so far has completed.
+__device__ __forceinline__ void umma_commit_pair_both(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(static_cast<uint16_t>(0x3))
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair_own(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+// Two-CTA tiled load into this CTA's shared memory whose bytes complete on the barrier
+// at `bar_cluster` (a shared::cluster address, here the leader's).
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
+                                                 int y, uint64_t cache_policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y), "l"(cache_policy)
+        : "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4Threads, 1)
+    nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                           const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
+                           const Nvfp4Gemm2Params p) {
+    extern __shared__ __align__(1024) uint8_t fp4p_smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fp4p_smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kF2BarOff);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + kF2Stages;
+    uint64_t* acc_full = bars + 2 * kF2Stages;
+    uint64_t* acc_empty = acc_full + 1;
+    uint64_t* drain = acc_full + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kF2NumBars);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x / 2;
+    const int n_pairs = gridDim.x / 2;
+    const int num_tiles = p.tiles_m * p.tiles_n;
+    const int k_tiles = p.K / kFp4TileK;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int s = 0; s < kF2Stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 16);  // eight epilogue warps in each CTA
+        mbar_init(drain, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&map_a);
+        tma_prefetch_desc(&map_b);
+        tma_prefetch_desc(&map_sfa);
+        tma_prefetch_desc(&map_sfb);
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(512)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync_all();  // both CTAs' barriers exist before either uses the other's
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    auto give_up = [&]() {
+        *abort_flag = 1;
+        abort_launch(p.epoch);
+    };
+    auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+        if (mbar_wait_bounded_cluster(bar, parity, abort_flag, kWaitLimitNs)) return true;
+        if (!*abort_flag) give_up();
+        return false;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0 && !launch_aborted(p.epoch)) {
+            const uint64_t pol_a = policy_evict_normal();
+            const uint64_t pol_b = policy_evict_last();
+            const int k_atoms = p.K / 64;
+            int it = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < num_tiles; tile += n_pairs) {
+                const int tm = tile / p.tiles_n;
+                const int tn = tile % p.tiles_n;
+                // scale groups that do not exist (past the padded rows) are replaced by the
+                // last one: they only feed rows and columns that are never stored
+                const int ga = min(tm * 2 + static_cast<int>(rank), p.groups_a - 1);
+                const int gb0 = min(tn * 2, p.groups_b - 1);
+                const int gb1 = min(tn * 2 + 1, p.groups_b - 1);
+                for (int kt = 0; kt < k_tiles; ++kt, ++it) {
+                    const int s = it % kF2Stages;
+                    if (!(ok = wait(&empty[s], ((it / kF2Stages) & 1) ^ 1))) break;
+                    uint8_t* st = smem + s * kF2StageBytes;
+                    const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * kF2StageBytes);
+                    tma_load_2d_pair(st, &map_a, bar, kt * 128, tm * 256 + static_cast<int>(rank) * 128, pol_a);
+                    tma_load_2d_pair(st + kF2Half, &map_b, bar, kt * 128, tn * 256 + static_cast<int>(rank) * 128, pol_b);
+                    tma_load_2d_pair(st + 2 * kF2Half, &map_sfa, bar, 0, ga * k_atoms + 4 * kt, pol_a);
+                    tma_load_2d_pair(st + 2 * kF2Half + kF2SfaBytes, &map_sfb, bar, 0, gb0 * k_atoms + 4 * kt, pol_b);
+                    tma_load_2d_pair(st + 2 * kF2Half + kF2SfaBytes + 2048, &map_sfb, bar, 0, gb1 * k_atoms + 4 * kt, pol_b);
+                }
+            }
+            if (!ok && leader) {
+                // every copy issued for the stages still pending must land before the pair exits
+                volatile int never = 0;
+                for (int q = it - kF2Stages < 0 ? 0 : it - kF2Stages; q < it; ++q)
+                    mbar_wait_bounded_cluster(&full[q % kF2Stages], (q / kF2Stages) & 1, &never, kWaitLimitNs);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ tensor-pipe issuer (leader)
+        if (lane == 0 && leader && !launch_aborted(p.epoch)) {
+            constexpr uint32_t idesc = idesc_nvfp4(256, 256);
+            int it = 0, tcount = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < num_tiles; tile += n_pairs, ++tcount) {
+                // both CTAs' epilogues must have read the previous tile's accumulator
+                if (tcount > 0 && !(ok = wait(acc_empty, (tcount - 1) & 1))) break;
+                tc_fence_after();
+                for (int kt = 0; kt < k_tiles; ++kt, ++it) {
+                    const int s = it % kF2Stages;
+                    if (!(ok = wait(&full[s], (it / kF2Stages) & 1))) break;
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(smem + s * kF2StageBytes);
+                    const uint32_t sfa = st + 2 * kF2Half;
+                    const uint32_t sfb = sfa + kF2SfaBytes;
+                    const uint32_t t_sfa = tmem + kFp4ColSf + (it & 1) * kFp4SfRegion;
+                    const uint32_t t_sfb = t_sfa + 16;
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb) {
+                        tmem_cp_pair_32x128b_warpx4(t_sfa + 4 * kb, sdesc_atom(sfa + kb * 512));
+                        tmem_cp_pair_32x128b_warpx4(t_sfb + 8 * kb, sdesc_atom(sfb + kb * 512));
+                        tmem_cp_pair_32x128b_warpx4(t_sfb + 8 * kb + 4, sdesc_atom(sfb + 2048 + kb * 512));
+                    }
+                    const uint64_t a0 = sdesc_sw128(st, 16, 1024);
+                    const uint64_t b0 = sdesc_sw128(st + kF2Half, 16, 1024);
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb)
+                        umma_nvfp4_pair(tmem, a0 + static_cast<uint64_t>((kb * 32) >> 4),
+                                        b0 + static_cast<uint64_t>((kb * 32) >> 4), idesc, t_sfa + 4 * kb, t_sfb + 8 * kb,
+                                        (kt | kb) ? 1u : 0u);
+                    umma_commit_pair_both(&empty[s]);
+                }
+                if (ok) umma_commit_pair_both(acc_full);
+            }
+            if (!ok) {
+                umma_commit_pair_own(drain);  // wait for every MMA this thread issued
+                volatile int never = 0;
+                mbar_wait_bounded_cluster(drain, 0, &never, kWaitLimitNs);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int quarter = warp & 3;
+        const int half = (warp - 2) >> 2;
+        const uint32_t t_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(half * 128);
+        const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+        const float alpha = __frcp_rn(__fmul_rn(nvfp4_tensor_scale(__ldg(p.amax_a)), nvfp4_tensor_scale(__ldg(p.amax_b))));
+        int tcount = 0;
+        for (int tile = pair; tile < num_tiles && !launch_aborted(p.epoch); tile += n_pairs, ++tcount) {
+            const int tm = tile / p.tiles_n;
+            const int tn = tile % p.tiles_n;
+            const bool ok = __all_sync(0xFFFFFFFFu, wait(acc_full, tcount & 1));
+            if (!ok) break;
+            tc_fence_after();
+            const int n0 = tn * 256 + half * 128;
+            uint32_t packed[64];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t raw[64];
+                tmem_ld64(t_row + c * 64, raw);
+#pragma unroll
+                for (int e = 0; e < 64; e += 2) {
+                    const int n = n0 + c * 64 + e;
+                    const float b0 = (p.bias && n < p.N) ? __ldg(p.bias + n) : 0.f;
+                    const float b1 = (p.bias && n + 1 < p.N) ? __ldg(p.bias + n + 1) : 0.f;
+                    packed[c * 32 + e / 2] = pack_bf16x2(fmaf(__uint_as_float(raw[e]), alpha, b0),
+                                                         fmaf(__uint_as_float(raw[e + 1]), alpha, b1));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+            const long long m = static_cast<long long>(tm) * 256 + static_cast<int>(rank) * 128 + quarter * 32 + lane;
+            if (m < p.M) {
+                uint4* dst = reinterpret_cast<uint4*>(p.c + m * p.N + n0);
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    if (n0 + 8 * j < p.N)
+                        dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+            }
+        }
+    }
+
+    // neither CTA releases its shared memory or TMEM while the pair's copies, MMAs or
+    // epilogue may still use them
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
+    }
+}
+
 }  // namespace sbsa

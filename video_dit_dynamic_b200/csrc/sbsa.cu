@@ -25,6 +25,13 @@
 #include "select.cuh"
 #include "ulysses.cuh"
 
+// 1: the NVFP4 GEMM on CTA pairs (256 x 256 tiles).  Parity-tested, but measured slower
+// than one CTA per 128 x 256 tile (1.80 vs 1.67 ms on 32,768 x 15,360 x 5,120): the scale
+// copies into TMEM, not the loads, bound both, and the pair adds cross-CTA hand-overs.
+#ifndef SBSA_NVFP4_PAIR
+#define SBSA_NVFP4_PAIR 0
+#endif
+
 namespace sbsa {
 namespace {
 
@@ -154,6 +161,22 @@ sbsa_status make_map_fp4(CUtensorMap* m, const void* base, long long rows, int K
     cuuint32_t es[2] = {1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SBSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return SBSA_OK;
+}
+
+// NVFP4 scale array viewed as 512-byte atoms ([atoms][128] uint32); a box is the 4 atoms
+// of one K-tile of one 128-row group (2 KB), no swizzle.
+sbsa_status make_map_scales(CUtensorMap* m, const void* base, long long atoms) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(SBSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(atoms)};
+    cuuint64_t strides[1] = {512};
+    cuuint32_t box[2] = {128, 4};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(SBSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
     return SBSA_OK;
@@ -702,6 +725,41 @@ sbsa_status sbsa_nvfp4_gemm(int32_t m, int32_t n, int32_t k, const void* a, cons
     if ((reinterpret_cast<uintptr_t>(a_amax) | reinterpret_cast<uintptr_t>(b_amax) |
          reinterpret_cast<uintptr_t>(bias)) & 3u)
         return fail(SBSA_ERR_INVALID_ARG, "amax and bias must be 4-byte aligned");
+#if SBSA_NVFP4_PAIR
+    {
+        // pairs of CTAs, 256 x 256 tiles
+        CUtensorMap ma, mb, msa, msb;
+        sbsa_status r;
+        Nvfp4Gemm2Params q;
+        q.amax_a = a_amax;
+        q.amax_b = b_amax;
+        q.bias = bias;
+        q.c = static_cast<__nv_bfloat16*>(c);
+        q.M = m;
+        q.N = n;
+        q.K = k;
+        q.tiles_m = (m + 255) / 256;
+        q.tiles_n = (n + 255) / 256;
+        q.groups_a = (m + 127) / 128;
+        q.groups_b = (n + 127) / 128;
+        q.epoch = g_epoch.fetch_add(1);
+        if ((r = make_map_fp4(&ma, a, m, k, 128)) != SBSA_OK) return r;
+        if ((r = make_map_fp4(&mb, b, n, k, 128)) != SBSA_OK) return r;
+        if ((r = make_map_scales(&msa, a_scales, static_cast<long long>(q.groups_a) * (k / 64))) != SBSA_OK) return r;
+        if ((r = make_map_scales(&msb, b_scales, static_cast<long long>(q.groups_b) * (k / 64))) != SBSA_OK) return r;
+        const long long tiles = static_cast<long long>(q.tiles_m) * q.tiles_n;
+        if (tiles > 0x3FFFFFFFLL) return fail(SBSA_ERR_UNSUPPORTED, "too many tiles");
+        const int pairs = static_cast<int>(tiles < sm_count() / 2 ? tiles : sm_count() / 2);
+        cudaError_t e = cudaFuncSetAttribute(nvfp4_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kF2SmemBytes);
+        if (e != cudaSuccess) return cuda_fail(e, "nvfp4 gemm smem attribute");
+        nvfp4_gemm_pair_kernel<<<2 * pairs, kFp4Threads, kF2SmemBytes, static_cast<cudaStream_t>(stream)>>>(ma, mb, msa,
+                                                                                                       msb, q);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "nvfp4 gemm launch");
+        return ok();
+    }
+#endif
     CUtensorMap ma, mb;
     sbsa_status r;
     if ((r = make_map_fp4(&ma, a, m, k, kFp4TileM)) != SBSA_OK) return r;
