@@ -274,3 +274,24 @@ def test_forward_from_host_matches_device_path():
     torch.cuda.synchronize()
     assert torch.equal(oh, od.cpu())
     assert math.isfinite(float(oh.float().abs().max()))
+
+
+@pytest.mark.parametrize("head_chunk", [None, 1, 3, 10])
+def test_forward_from_host_chunked_pipeline(head_chunk):
+    """The copy/compute/copy pipeline over head chunks gives the one-call result bit for
+    bit, also when the chunks do not divide the heads, and when called back to back."""
+    B, H, L, d, blk = 2, 5, 700, 128, 128
+    s = sbsa.make_shape(B, H, L, d, blk)
+    q, k, v = inputs.random_qkv(B, H, s.seq_len_padded, d, L=L, seed=21)
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    kk = sbsa.sbsa_keep_blocks(s.num_blocks, 0.5)
+    od = torch.empty_like(q, device="cuda")
+    sbsa.sbsa_forward(s, q.cuda(), k.cuda(), v.cuda(), kk, 0.0, od, None, sbsa.alloc_workspace(s, kk))
+    bufs = (torch.empty_like(od), torch.empty_like(od), torch.empty_like(od), torch.empty_like(od),
+            sbsa.alloc_workspace(s, kk))
+    outs = [sbsa.forward_from_host(s, qh, kh, vh, kk, device_buffers=bufs, head_chunk=head_chunk) for _ in range(2)]
+    torch.cuda.synchronize()
+    sbsa.sbsa_check()
+    ref = od.cpu()
+    for oh in outs:
+        assert torch.equal(oh, ref)

@@ -417,11 +417,28 @@ def alloc_workspace(shape: Shape, k_keep: int, device="cuda") -> torch.Tensor:
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
+_copy_streams = {}
+
+
+def _side_streams(device):
+    """Two streams per device, one for host-to-device and one for device-to-host copies."""
+    key = torch.device(device).index if torch.device(device).index is not None else torch.cuda.current_device()
+    if key not in _copy_streams:
+        _copy_streams[key] = (torch.cuda.Stream(device=key), torch.cuda.Stream(device=key))
+    return _copy_streams[key]
+
+
 def forward_from_host(shape: Shape, q_host, k_host, v_host, k_keep: int, scale: float = 0.0, *, o_host=None,
-                      device_buffers=None, stream=None):
+                      device_buffers=None, stream=None, head_chunk: int | None = None):
     """End-to-end call from host tensors: copy Q/K/V (pinned host memory) to the device,
     run sbsa_forward, copy O back.  ``device_buffers`` (q, k, v, o, workspace) may be
-    passed to reuse device memory across calls.  Returns the host output tensor."""
+    passed to reuse device memory across calls.  Returns the host output tensor.
+
+    The layer is processed in chunks of ``head_chunk`` (batch, head) pairs (every pair is
+    independent, so the result is the same as one call): the copy-in of a chunk, the
+    attention of the previous one and the copy-out of the one before overlap on three
+    streams.  Default: about eight chunks.  Asynchronous with respect to the host; the
+    work is complete once ``stream`` (default: the current stream) is."""
     s = stream or torch.cuda.current_stream()
     if device_buffers is None:
         dq = torch.empty(q_host.shape, dtype=torch.bfloat16, device="cuda")
@@ -429,12 +446,28 @@ def forward_from_host(shape: Shape, q_host, k_host, v_host, k_keep: int, scale: 
         ws = alloc_workspace(shape, k_keep)
     else:
         dq, dk, dv, do, ws = device_buffers
-    with torch.cuda.stream(s):
-        dq.copy_(q_host, non_blocking=True)
-        dk.copy_(k_host, non_blocking=True)
-        dv.copy_(v_host, non_blocking=True)
-        sbsa_forward(shape, dq, dk, dv, k_keep, scale, do, None, ws, stream=s)
-        if o_host is None:
-            o_host = torch.empty(do.shape, dtype=do.dtype, pin_memory=True)
-        o_host.copy_(do, non_blocking=True)
+    if o_host is None:
+        o_host = torch.empty(do.shape, dtype=do.dtype, pin_memory=True)
+    pairs = shape.batch * shape.heads
+    n = head_chunk or max(1, -(-pairs // 8))
+    rows = shape.seq_len_padded * shape.head_dim  # elements per (batch, head)
+    flat = [t.reshape(pairs, rows) for t in (q_host, k_host, v_host, o_host, dq, dk, dv, do)]
+    qh, kh, vh, oh, fq, fk, fv, fo = flat
+    h2d, d2h = _side_streams(dq.device)
+    # this call's copies must not overwrite buffers that earlier work on `s` or on the
+    # copy streams still uses
+    h2d.wait_stream(s)
+    s.wait_stream(d2h)
+    for c0 in range(0, pairs, n):
+        c1 = min(pairs, c0 + n)
+        with torch.cuda.stream(h2d):
+            for dst, src in ((fq, qh), (fk, kh), (fv, vh)):
+                dst[c0:c1].copy_(src[c0:c1], non_blocking=True)
+        s.wait_stream(h2d)
+        cs = make_shape(1, c1 - c0, shape.seq_len, shape.head_dim, shape.block_size, shape.seq_len_padded)
+        sbsa_forward(cs, fq[c0:c1], fk[c0:c1], fv[c0:c1], k_keep, scale, fo[c0:c1], None, ws, stream=s)
+        d2h.wait_stream(s)
+        with torch.cuda.stream(d2h):
+            oh[c0:c1].copy_(fo[c0:c1], non_blocking=True)
+    s.wait_stream(d2h)
     return o_host
