@@ -182,7 +182,14 @@ constexpr int kFp4SfaBytes = (kFp4TileM / 128) * 4 * 512;
 constexpr int kFp4SfbBytes = (kFp4TileN / 128) * 4 * 512;
 constexpr int kFp4StageBytes = kFp4ABytes + kFp4BBytes + kFp4SfaBytes + kFp4SfbBytes;
 constexpr int kFp4BarOff = kFp4Stages * kFp4StageBytes;
-constexpr int kFp4NumBars = 2 * kFp4Stages + 3;  // full[S], empty[S], acc_full, acc_empty, drain
+// 1: the scale atoms go into TMEM by tcgen05.st from four epilogue warps (one TMEM region
+// per stage), so the MMA thread issues only MMAs; 0: the MMA thread copies them with
+// tcgen05.cp ahead of its MMAs.
+#ifndef SBSA_NVFP4_SF_STORE
+#define SBSA_NVFP4_SF_STORE 1
+#endif
+constexpr uint32_t kFp4SfStageCols = 48;  // A scales (16 columns) then B scales (32) of one K-tile
+constexpr int kFp4NumBars = 3 * kFp4Stages + 3;  // full[S], empty[S], sf_full[S], acc_full, acc_empty, drain
 constexpr int kFp4SmemBytes = kFp4BarOff + kFp4NumBars * 8 + 16 + 1024;  // + tmem slot, flag, alignment slack
 constexpr int kFp4Threads = 320;
 constexpr uint32_t kFp4ColSf = 256;     // two scale regions of 48 columns, by K-tile parity
@@ -237,7 +244,8 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kFp4BarOff);
     uint64_t* full = bars;
     uint64_t* empty = bars + kFp4Stages;
-    uint64_t* acc_full = bars + 2 * kFp4Stages;
+    uint64_t* sf_full = bars + 2 * kFp4Stages;  // a stage's scales are in TMEM
+    uint64_t* acc_full = bars + 3 * kFp4Stages;
     uint64_t* acc_empty = acc_full + 1;
     uint64_t* drain = acc_full + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kFp4NumBars);
@@ -254,6 +262,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
         for (int s = 0; s < kFp4Stages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&sf_full[s], 4);  // one arrival per scale-storing warp
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 8);
@@ -331,6 +340,13 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
                     if (!(ok = wait(&full[s], (it / kFp4Stages) & 1))) break;
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + s * kFp4StageBytes);
+#if SBSA_NVFP4_SF_STORE
+                    // the stage's scales were stored into its TMEM region by warps 2-5
+                    if (!(ok = wait(&sf_full[s], (it / kFp4Stages) & 1))) break;
+                    tc_fence_after();
+                    const uint32_t t_sfa = tmem + kFp4ColSf + static_cast<uint32_t>(s) * kFp4SfStageCols;
+                    const uint32_t t_sfb = t_sfa + 16;
+#else
                     const uint32_t sfa = st + kFp4ABytes + kFp4BBytes;
                     const uint32_t sfb = sfa + kFp4SfaBytes;
                     // consecutive K-tiles use different TMEM scale regions
@@ -342,6 +358,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
                         tmem_cp_32x128b_warpx4(t_sfb + 8 * kb, sdesc_atom(sfb + kb * 512));
                         tmem_cp_32x128b_warpx4(t_sfb + 8 * kb + 4, sdesc_atom(sfb + 2048 + kb * 512));
                     }
+#endif
                     const uint64_t a0 = sdesc_sw128(st, 16, 1024);
                     const uint64_t b0 = sdesc_sw128(st + kFp4ABytes, 16, 1024);
 #pragma unroll
@@ -362,16 +379,18 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // (warps 2-5 also store every stage's scales into TMEM; see sf_stage)
         const int quarter = warp & 3;
         const int half = (warp - 2) >> 2;
         const uint32_t t_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(half * 128);
         const float alpha = __frcp_rn(__fmul_rn(nvfp4_tensor_scale(__ldg(p.amax_a)), nvfp4_tensor_scale(__ldg(p.amax_b))));
-        int tcount = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
+        // one output tile: read this warp's rows and columns out of TMEM, hand the
+        // accumulator back, store
+        auto epilogue = [&](int tile, int tcount) -> bool {
             const int tm = tile / p.tiles_n;
             const int tn = tile % p.tiles_n;
             const bool ok = __all_sync(0xFFFFFFFFu, wait(acc_full, tcount & 1));
-            if (!ok) break;
+            if (!ok) return false;
             tc_fence_after();
             const int n0 = tn * kFp4TileN + half * 128;
             // this warp's 128 columns in two 64-column TMEM loads
@@ -401,6 +420,55 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
                     if (n0 + 8 * j < p.N)
                         dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
             }
+            return true;
+        };
+#if SBSA_NVFP4_SF_STORE
+        if (half == 0) {
+            // K-tile i's scales into TMEM region i % S: lane L of quarter q holds, for rows
+            // 32 q + L % 32 of A (4 columns per K step) and of B's two 128-row groups
+            // (8 columns per K step), the 16 bytes of row L % 32 of each 512-byte atom --
+            // the layout tcgen05.cp.32x128b.warpx4 would leave there
+            auto sf_stage = [&](int i) -> bool {
+                const int s = i % kFp4Stages;
+                if (!__all_sync(0xFFFFFFFFu, wait(&full[s], (i / kFp4Stages) & 1))) return false;
+                const uint32_t base = smem_u32(smem + s * kFp4StageBytes + kFp4ABytes + kFp4BBytes) + lane * 16;
+                uint32_t va[16], vb[32];
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb) {
+                    ld_shared_v4(base + kb * 512, va[4 * kb], va[4 * kb + 1], va[4 * kb + 2], va[4 * kb + 3]);
+#pragma unroll
+                    for (int g = 0; g < 2; ++g)
+                        ld_shared_v4(base + kFp4SfaBytes + g * 2048 + kb * 512, vb[8 * kb + 4 * g], vb[8 * kb + 4 * g + 1],
+                                     vb[8 * kb + 4 * g + 2], vb[8 * kb + 4 * g + 3]);
+                }
+                const uint32_t t = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kFp4ColSf +
+                                   static_cast<uint32_t>(s) * kFp4SfStageCols;
+                tmem_st16(t, va);
+                tmem_st32(t + 16, vb);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_full[s]);
+                return true;
+            };
+            // scales of every K-tile in order; a tile's epilogue after the next tile's
+            // first scales, so the MMAs of that tile need not wait for them
+            int it = 0, tcount = 0, prev = -1;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++tcount) {
+                for (int kt = 0; ok && kt < k_tiles; ++kt, ++it) {
+                    ok = sf_stage(it);
+                    if (ok && kt == 0 && prev >= 0) ok = epilogue(prev, tcount - 1);
+                }
+                prev = tile;
+            }
+            if (ok && prev >= 0) epilogue(prev, tcount - 1);
+        } else
+#endif
+        {
+            int tcount = 0;
+            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount)
+                if (!epilogue(tile, tcount)) break;
         }
     }
 
