@@ -147,19 +147,18 @@ __global__ void __launch_bounds__(256) nvfp4_quantize_kernel(const uint4* __rest
 //              128 bytes), B (256 x 128 bytes), their scale atoms (2 KB and 4 KB,
 //              contiguous in global memory, one bulk copy per 128-row group) through a
 //              four-stage ring;
-//   warp 1     TMEM allocation and the one thread that issues everything on the
-//              tensor pipe: per K-tile, twelve tcgen05.cp of scale atoms into TMEM and
-//              four block-scaled MMAs (M = 128, N = 256, K = 64).  tcgen05.cp and
-//              tcgen05.mma from one thread execute in issue order, so a TMEM scale
-//              region can be refilled right after the MMAs that read it were issued
-//              (issuing the next K-tile's copies ahead of the current MMAs was measured
-//              slower: it makes the MMAs wait for one more stage to land);
+//   warp 1     TMEM allocation and the one thread that issues the block-scaled MMAs
+//              (M = 128, N = 256, K = 64; four per K-tile) and nothing else;
 //   warps 2-9  epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 and output columns
-//              128 ((w - 2) / 4) .. + 127 of the tile, applies alpha and the bias in
-//              fp32, rounds to bf16, hands the accumulator back, then stores its rows.
-// TMEM: accumulator in columns 0-255; two scale regions of 48 columns at 256 and 304,
-// used by alternate K-tiles, each with the A scales (four columns per K step) and then
-// the B scales (eight per K step).
+//              128 ((w - 2) / 4) .. + 127 of the tile, applies alpha and the bias in fp32,
+//              rounds to bf16, hands the accumulator back, then stores its rows.  Warps 2-5
+//              also store every stage's 12 scale atoms into that stage's TMEM region
+//              (tcgen05.st, in the layout tcgen05.cp.32x128b.warpx4 would leave) and arrive
+//              on its sf_full barrier; a tile's epilogue comes after the next tile's first
+//              scales.  (Measured: copying the scales with tcgen05.cp from the MMA thread,
+//              in order with its MMAs, was 13% slower.)
+// TMEM: accumulator in columns 0-255; one scale region of 48 columns per stage from
+// column 256 (A scales: four columns per K step, then B scales: eight per K step).
 struct Nvfp4GemmParams {
     const uint8_t* sfa;
     const uint8_t* sfb;
@@ -182,12 +181,6 @@ constexpr int kFp4SfaBytes = (kFp4TileM / 128) * 4 * 512;
 constexpr int kFp4SfbBytes = (kFp4TileN / 128) * 4 * 512;
 constexpr int kFp4StageBytes = kFp4ABytes + kFp4BBytes + kFp4SfaBytes + kFp4SfbBytes;
 constexpr int kFp4BarOff = kFp4Stages * kFp4StageBytes;
-// 1: the scale atoms go into TMEM by tcgen05.st from four epilogue warps (one TMEM region
-// per stage), so the MMA thread issues only MMAs; 0: the MMA thread copies them with
-// tcgen05.cp ahead of its MMAs.
-#ifndef SBSA_NVFP4_SF_STORE
-#define SBSA_NVFP4_SF_STORE 1
-#endif
 constexpr uint32_t kFp4SfStageCols = 48;  // A scales (16 columns) then B scales (32) of one K-tile
 constexpr int kFp4NumBars = 3 * kFp4Stages + 3;  // full[S], empty[S], sf_full[S], acc_full, acc_empty, drain
 constexpr int kFp4SmemBytes = kFp4BarOff + kFp4NumBars * 8 + 16 + 1024;  // + tmem slot, flag, alignment slack
@@ -213,11 +206,6 @@ __device__ __forceinline__ void umma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uin
         : "memory");
 }
 
-// 32 rows x 16 bytes of shared memory into TMEM columns taddr .. taddr + 3 of every lane
-// quarter (row i of the source goes to lane i of each quarter).
-__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
 
 // Descriptor of a 512-byte scale atom: no swizzle, 8-row x 16-byte core matrices 128
 // bytes apart (both offsets 128: the atom is one core matrix wide).
@@ -340,25 +328,11 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
                     if (!(ok = wait(&full[s], (it / kFp4Stages) & 1))) break;
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + s * kFp4StageBytes);
-#if SBSA_NVFP4_SF_STORE
                     // the stage's scales were stored into its TMEM region by warps 2-5
                     if (!(ok = wait(&sf_full[s], (it / kFp4Stages) & 1))) break;
                     tc_fence_after();
                     const uint32_t t_sfa = tmem + kFp4ColSf + static_cast<uint32_t>(s) * kFp4SfStageCols;
                     const uint32_t t_sfb = t_sfa + 16;
-#else
-                    const uint32_t sfa = st + kFp4ABytes + kFp4BBytes;
-                    const uint32_t sfb = sfa + kFp4SfaBytes;
-                    // consecutive K-tiles use different TMEM scale regions
-                    const uint32_t t_sfa = tmem + kFp4ColSf + (it & 1) * kFp4SfRegion;
-                    const uint32_t t_sfb = t_sfa + 16;
-#pragma unroll
-                    for (int kb = 0; kb < 4; ++kb) {
-                        tmem_cp_32x128b_warpx4(t_sfa + 4 * kb, sdesc_atom(sfa + kb * 512));
-                        tmem_cp_32x128b_warpx4(t_sfb + 8 * kb, sdesc_atom(sfb + kb * 512));
-                        tmem_cp_32x128b_warpx4(t_sfb + 8 * kb + 4, sdesc_atom(sfb + 2048 + kb * 512));
-                    }
-#endif
                     const uint64_t a0 = sdesc_sw128(st, 16, 1024);
                     const uint64_t b0 = sdesc_sw128(st + kFp4ABytes, 16, 1024);
 #pragma unroll
@@ -422,7 +396,6 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
             }
             return true;
         };
-#if SBSA_NVFP4_SF_STORE
         if (half == 0) {
             // K-tile i's scales into TMEM region i % S: lane L of quarter q holds, for rows
             // 32 q + L % 32 of A (4 columns per K step) and of B's two 128-row groups
@@ -463,9 +436,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
                 prev = tile;
             }
             if (ok && prev >= 0) epilogue(prev, tcount - 1);
-        } else
-#endif
-        {
+        } else {
             int tcount = 0;
             for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount)
                 if (!epilogue(tile, tcount)) break;
