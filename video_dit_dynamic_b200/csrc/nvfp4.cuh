@@ -142,21 +142,24 @@ __global__ void __launch_bounds__(256) nvfp4_quantize_kernel(const uint4* __rest
 //
 // Persistent: one CTA per SM walks output tiles of 128 x 256 (tile index t -> row
 // tile t / tiles_n, column tile t % tiles_n, so the CTAs running at one time share a
-// few A row tiles and all of B in L2).  320 threads:
-//   warp 0     TMA producer: per K-tile of 256 elements one stage of A (128 rows x
-//              128 bytes), B (256 x 128 bytes), their scale atoms (2 KB and 4 KB,
-//              contiguous in global memory, one bulk copy per 128-row group) through a
-//              four-stage ring;
-//   warp 1     TMEM allocation and the one thread that issues the block-scaled MMAs
-//              (M = 128, N = 256, K = 64; four per K-tile) and nothing else;
-//   warps 2-9  epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 and output columns
-//              128 ((w - 2) / 4) .. + 127 of the tile, applies alpha and the bias in fp32,
-//              rounds to bf16, hands the accumulator back, then stores its rows.  Warps 2-5
-//              also store every stage's 12 scale atoms into that stage's TMEM region
-//              (tcgen05.st, in the layout tcgen05.cp.32x128b.warpx4 would leave) and arrive
-//              on its sf_full barrier; a tile's epilogue comes after the next tile's first
-//              scales.  (Measured: copying the scales with tcgen05.cp from the MMA thread,
-//              in order with its MMAs, was 13% slower.)
+// few A row tiles and all of B in L2).  448 threads:
+//   warp 0      TMA producer: per K-tile of 256 elements one stage of A (128 rows x
+//               128 bytes), B (256 x 128 bytes), their scale atoms (2 KB and 4 KB,
+//               contiguous in global memory, one bulk copy per 128-row group) through a
+//               four-stage ring;
+//   warp 1      TMEM allocation and the one thread that issues the block-scaled MMAs
+//               (M = 128, N = 256, K = 64; four per K-tile) and nothing else;
+//   warps 2-9   epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 and output columns
+//               128 ((w - 2) / 4) .. + 127 of the tile, applies alpha and the bias (staged
+//               in shared memory while the tile is computed) in one fp32 FMA, rounds to
+//               bf16, hands the accumulator back, then stores its rows;
+//   warps 10-13 scales: each stage's 12 scale atoms into that stage's TMEM region
+//               (tcgen05.st, in the layout tcgen05.cp.32x128b.warpx4 would leave), then
+//               its sf_full barrier.
+// Measured on the way: scale copies issued with tcgen05.cp by the MMA thread, in order
+// with its MMAs, bounded the kernel; stored by warps that also ran the epilogue, they
+// queued behind its stores; a bias read from global memory per element made the
+// accumulator's hand-back slow.
 // TMEM: accumulator in columns 0-255; one scale region of 48 columns per stage from
 // column 256 (A scales: four columns per K step, then B scales: eight per K step).
 struct Nvfp4GemmParams {
@@ -180,11 +183,13 @@ constexpr int kFp4BBytes = kFp4TileN * 128;
 constexpr int kFp4SfaBytes = (kFp4TileM / 128) * 4 * 512;
 constexpr int kFp4SfbBytes = (kFp4TileN / 128) * 4 * 512;
 constexpr int kFp4StageBytes = kFp4ABytes + kFp4BBytes + kFp4SfaBytes + kFp4SfbBytes;
-constexpr int kFp4BarOff = kFp4Stages * kFp4StageBytes;
+constexpr int kFp4BiasOff = kFp4Stages * kFp4StageBytes;  // each epilogue warp's 128 bias values of the tile
+constexpr int kFp4BarOff = kFp4BiasOff + 8 * 128 * 4;
 constexpr uint32_t kFp4SfStageCols = 48;  // A scales (16 columns) then B scales (32) of one K-tile
 constexpr int kFp4NumBars = 3 * kFp4Stages + 3;  // full[S], empty[S], sf_full[S], acc_full, acc_empty, drain
 constexpr int kFp4SmemBytes = kFp4BarOff + kFp4NumBars * 8 + 16 + 1024;  // + tmem slot, flag, alignment slack
-constexpr int kFp4Threads = 320;
+constexpr int kFp4Threads = 448;      // 14 warps: producer, MMA, eight epilogue, four scale warps
+constexpr int kFp4PairThreads = 320;
 constexpr uint32_t kFp4ColSf = 256;     // two scale regions of 48 columns, by K-tile parity
 constexpr uint32_t kFp4SfRegion = 48;   // A scales at +0 (16 columns), B scales at +16 (32 columns)
 static_assert(kFp4StageBytes % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
@@ -253,7 +258,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
             mbar_init(&sf_full[s], 4);  // one arrival per scale-storing warp
         }
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 8);
+        mbar_init(acc_empty, 8);  // the eight epilogue warps
         mbar_init(drain, 1);
         fence_mbar_init();
         tma_prefetch_desc(&map_a);
@@ -328,7 +333,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
                     if (!(ok = wait(&full[s], (it / kFp4Stages) & 1))) break;
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + s * kFp4StageBytes);
-                    // the stage's scales were stored into its TMEM region by warps 2-5
+                    // the stage's scales were stored into its TMEM region by warps 10-13
                     if (!(ok = wait(&sf_full[s], (it / kFp4Stages) & 1))) break;
                     tc_fence_after();
                     const uint32_t t_sfa = tmem + kFp4ColSf + static_cast<uint32_t>(s) * kFp4SfStageCols;
@@ -352,58 +357,78 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
             }
         }
     } else {
-        // ------------------------------------------------------------ epilogue
-        // (warps 2-5 also store every stage's scales into TMEM; see sf_stage)
-        const int quarter = warp & 3;
-        const int half = (warp - 2) >> 2;
-        const uint32_t t_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(half * 128);
-        const float alpha = __frcp_rn(__fmul_rn(nvfp4_tensor_scale(__ldg(p.amax_a)), nvfp4_tensor_scale(__ldg(p.amax_b))));
-        // one output tile: read this warp's rows and columns out of TMEM, hand the
-        // accumulator back, store
-        auto epilogue = [&](int tile, int tcount) -> bool {
-            const int tm = tile / p.tiles_n;
-            const int tn = tile % p.tiles_n;
-            const bool ok = __all_sync(0xFFFFFFFFu, wait(acc_full, tcount & 1));
-            if (!ok) return false;
-            tc_fence_after();
-            const int n0 = tn * kFp4TileN + half * 128;
-            // this warp's 128 columns in two 64-column TMEM loads
-            uint32_t packed[64];
+        const int quarter = warp & 3;  // the TMEM lane quarter this warp may access
+        if (warp < 10) {
+            // ------------------------------------------------------------ epilogue (warps 2-9)
+            const int half = (warp - 2) >> 2;
+            const uint32_t t_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(half * 128);
+            const float alpha =
+                __frcp_rn(__fmul_rn(nvfp4_tensor_scale(__ldg(p.amax_a)), nvfp4_tensor_scale(__ldg(p.amax_b))));
+            // this warp's copy of the tile's 128 bias values (read back as broadcasts)
+            const uint32_t bias_w = smem_u32(smem + kFp4BiasOff) + static_cast<uint32_t>((warp - 2) * 128 * 4);
+            int tcount = 0;
+            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
+                const int tm = tile / p.tiles_n;
+                const int tn = tile % p.tiles_n;
+                const int n0 = tn * kFp4TileN + half * 128;
+                // the bias goes to shared memory while the tile is still being computed
+                {
+                    float b[4];
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t raw[64];
-                tmem_ld64(t_row + c * 64, raw);
-#pragma unroll
-                for (int e = 0; e < 64; e += 2) {
-                    const int n = n0 + c * 64 + e;
-                    const float b0 = (p.bias && n < p.N) ? __ldg(p.bias + n) : 0.f;
-                    const float b1 = (p.bias && n + 1 < p.N) ? __ldg(p.bias + n + 1) : 0.f;
-                    packed[c * 32 + e / 2] = pack_bf16x2(fmaf(__uint_as_float(raw[e]), alpha, b0),
-                                                         fmaf(__uint_as_float(raw[e + 1]), alpha, b1));
+                    for (int e = 0; e < 4; ++e) {
+                        const int n = n0 + 4 * lane + e;
+                        b[e] = (p.bias && n < p.N) ? __ldg(p.bias + n) : 0.f;
+                    }
+                    st_shared_v4(bias_w + lane * 16, __float_as_uint(b[0]), __float_as_uint(b[1]), __float_as_uint(b[2]),
+                                 __float_as_uint(b[3]));
+                    __syncwarp();
                 }
-            }
-            // the accumulator is in registers: the next tile's MMAs may overwrite it
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
-            const long long m = static_cast<long long>(tm) * kFp4TileM + quarter * 32 + lane;
-            if (m < p.M) {
-                uint4* dst = reinterpret_cast<uint4*>(p.c + m * p.N + n0);
+                if (!__all_sync(0xFFFFFFFFu, wait(acc_full, tcount & 1))) break;
+                tc_fence_after();
+                // this warp's 128 columns in two 64-column TMEM loads
+                uint32_t packed[64];
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    if (n0 + 8 * j < p.N)
-                        dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t raw[64];
+                    tmem_ld64(t_row + c * 64, raw);
+#pragma unroll
+                    for (int e = 0; e < 64; e += 4) {
+                        uint32_t b0, b1, b2, b3;
+                        ld_shared_v4(bias_w + (c * 64 + e) * 4, b0, b1, b2, b3);
+                        packed[c * 32 + e / 2] = pack_bf16x2(fmaf(__uint_as_float(raw[e]), alpha, __uint_as_float(b0)),
+                                                             fmaf(__uint_as_float(raw[e + 1]), alpha, __uint_as_float(b1)));
+                        packed[c * 32 + e / 2 + 1] =
+                            pack_bf16x2(fmaf(__uint_as_float(raw[e + 2]), alpha, __uint_as_float(b2)),
+                                        fmaf(__uint_as_float(raw[e + 3]), alpha, __uint_as_float(b3)));
+                    }
+                }
+                // the accumulator is in registers: the next tile's MMAs may overwrite it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty);
+                const long long m = static_cast<long long>(tm) * kFp4TileM + quarter * 32 + lane;
+                if (m < p.M) {
+                    uint4* dst = reinterpret_cast<uint4*>(p.c + m * p.N + n0);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (n0 + 8 * j < p.N)
+                            dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+                }
+                __syncwarp();  // every lane has read the bias before the next tile's is written
             }
-            return true;
-        };
-        if (half == 0) {
+        } else {
+            // ------------------------------------------------------------ scales (warps 10-13)
             // K-tile i's scales into TMEM region i % S: lane L of quarter q holds, for rows
             // 32 q + L % 32 of A (4 columns per K step) and of B's two 128-row groups
             // (8 columns per K step), the 16 bytes of row L % 32 of each 512-byte atom --
             // the layout tcgen05.cp.32x128b.warpx4 would leave there
-            auto sf_stage = [&](int i) -> bool {
+            const int my_tiles = static_cast<int>(blockIdx.x) < num_tiles
+                                     ? (num_tiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                                     : 0;
+            const int total = my_tiles * k_tiles;
+            for (int i = 0; i < total; ++i) {
                 const int s = i % kFp4Stages;
-                if (!__all_sync(0xFFFFFFFFu, wait(&full[s], (i / kFp4Stages) & 1))) return false;
+                if (!__all_sync(0xFFFFFFFFu, wait(&full[s], (i / kFp4Stages) & 1))) break;
                 const uint32_t base = smem_u32(smem + s * kFp4StageBytes + kFp4ABytes + kFp4BBytes) + lane * 16;
                 uint32_t va[16], vb[32];
 #pragma unroll
@@ -422,24 +447,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sf_full[s]);
-                return true;
-            };
-            // scales of every K-tile in order; a tile's epilogue after the next tile's
-            // first scales, so the MMAs of that tile need not wait for them
-            int it = 0, tcount = 0, prev = -1;
-            bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++tcount) {
-                for (int kt = 0; ok && kt < k_tiles; ++kt, ++it) {
-                    ok = sf_stage(it);
-                    if (ok && kt == 0 && prev >= 0) ok = epilogue(prev, tcount - 1);
-                }
-                prev = tile;
             }
-            if (ok && prev >= 0) epilogue(prev, tcount - 1);
-        } else {
-            int tcount = 0;
-            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount)
-                if (!epilogue(tile, tcount)) break;
         }
     }
 
@@ -525,7 +533,7 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
         : "memory");
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4Threads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4PairThreads, 1)
     nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                            const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
                            const Nvfp4Gemm2Params p) {

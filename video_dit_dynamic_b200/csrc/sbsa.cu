@@ -753,7 +753,7 @@ sbsa_status sbsa_nvfp4_gemm(int32_t m, int32_t n, int32_t k, const void* a, cons
         cudaError_t e = cudaFuncSetAttribute(nvfp4_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kF2SmemBytes);
         if (e != cudaSuccess) return cuda_fail(e, "nvfp4 gemm smem attribute");
-        nvfp4_gemm_pair_kernel<<<2 * pairs, kFp4Threads, kF2SmemBytes, static_cast<cudaStream_t>(stream)>>>(ma, mb, msa,
+        nvfp4_gemm_pair_kernel<<<2 * pairs, kFp4PairThreads, kF2SmemBytes, static_cast<cudaStream_t>(stream)>>>(ma, mb, msa,
                                                                                                        msb, q);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "nvfp4 gemm launch");
