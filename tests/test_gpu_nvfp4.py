@@ -116,6 +116,26 @@ def test_gemm_matches_oracle_on_oracle_codes(m, n, k, bias):
     _check_gemm(c, ref, oracle.nvfp4_dequantize(ac, asf, a_s), oracle.nvfp4_dequantize(bc, bsf, b_s))
 
 
+def test_gemm_output_only_16_byte_aligned():
+    """C starting 16 bytes past a 32-byte boundary takes the 16-byte store path."""
+    sbsa = _sbsa()
+    m, n, k = 259, 512, 256
+    a = inputs.bf16_bits(_bf16(m, k, seed=41))
+    b = inputs.bf16_bits(_bf16(n, k, seed=42, scale=0.05))
+    ac, asf, a_s = oracle.nvfp4_quantize(a)
+    bc, bsf, b_s = oracle.nvfp4_quantize(b)
+    ref = oracle.nvfp4_gemm(ac, asf, a_s, bc, bsf, b_s, None)
+    dev = lambda arr: torch.from_numpy(np.ascontiguousarray(arr)).cuda()
+    buf = torch.empty(m * n + 32, dtype=torch.bfloat16, device="cuda")
+    base = (-buf.data_ptr() // 2) % 16  # elements to the next 32-byte boundary
+    c = buf[base + 8:base + 8 + m * n].view(m, n)
+    assert c.data_ptr() % 32 == 16
+    sbsa.sbsa_nvfp4_gemm(m, n, k, dev(ac), dev(asf), dev(np.array([_amax_of(a)])), dev(bc), dev(bsf),
+                         dev(np.array([_amax_of(b)])), None, c)
+    sbsa.sbsa_check()
+    _check_gemm(c, ref, oracle.nvfp4_dequantize(ac, asf, a_s), oracle.nvfp4_dequantize(bc, bsf, b_s))
+
+
 def test_gemm_end_to_end_from_bf16():
     sbsa = _sbsa()
     m, n, k = 520, 768, 1024

@@ -188,8 +188,7 @@ constexpr int kFp4BarOff = kFp4BiasOff + 8 * 128 * 4;
 constexpr uint32_t kFp4SfStageCols = 48;  // A scales (16 columns) then B scales (32) of one K-tile
 constexpr int kFp4NumBars = 3 * kFp4Stages + 3;  // full[S], empty[S], sf_full[S], acc_full, acc_empty, drain
 constexpr int kFp4SmemBytes = kFp4BarOff + kFp4NumBars * 8 + 16 + 1024;  // + tmem slot, flag, alignment slack
-constexpr int kFp4Threads = 448;      // 14 warps: producer, MMA, eight epilogue, four scale warps
-constexpr int kFp4PairThreads = 320;
+constexpr int kFp4Threads = 448;  // 14 warps: producer, MMA, eight epilogue, four scale warps
 constexpr uint32_t kFp4ColSf = 256;     // two scale regions of 48 columns, by K-tile parity
 constexpr uint32_t kFp4SfRegion = 48;   // A scales at +0 (16 columns), B scales at +16 (32 columns)
 static_assert(kFp4StageBytes % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
@@ -227,6 +226,25 @@ __device__ __forceinline__ uint64_t policy_evict_normal() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
     return p;
+}
+
+// One thread's 128 bf16 outputs of a row from column n0 (64 packed pairs).  With
+// `wide` (row starts 32-byte aligned, N a multiple of 16) each store is 32 bytes, a
+// whole L2 sector: the 16-byte stores of a warp fill half-sectors of 32 rows and cost
+// the kernel about 9% (measured).
+__device__ __forceinline__ void store_row128(__nv_bfloat16* row, const uint32_t (&v)[64], int n0, int N, bool wide) {
+    if (wide) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (n0 + 16 * j < N)
+                st_global_v8(row + n0 + 16 * j, v[8 * j], v[8 * j + 1], v[8 * j + 2], v[8 * j + 3], v[8 * j + 4],
+                             v[8 * j + 5], v[8 * j + 6], v[8 * j + 7]);
+    } else {
+        uint4* dst = reinterpret_cast<uint4*>(row + n0);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (n0 + 8 * j < N) dst[j] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    }
 }
 
 __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
@@ -364,6 +382,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
             const uint32_t t_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(half * 128);
             const float alpha =
                 __frcp_rn(__fmul_rn(nvfp4_tensor_scale(__ldg(p.amax_a)), nvfp4_tensor_scale(__ldg(p.amax_b))));
+            const bool wide = (reinterpret_cast<uintptr_t>(p.c) & 31u) == 0 && p.N % 16 == 0;
             // this warp's copy of the tile's 128 bias values (read back as broadcasts)
             const uint32_t bias_w = smem_u32(smem + kFp4BiasOff) + static_cast<uint32_t>((warp - 2) * 128 * 4);
             int tcount = 0;
@@ -407,13 +426,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
                 __syncwarp();
                 if (lane == 0) mbar_arrive(acc_empty);
                 const long long m = static_cast<long long>(tm) * kFp4TileM + quarter * 32 + lane;
-                if (m < p.M) {
-                    uint4* dst = reinterpret_cast<uint4*>(p.c + m * p.N + n0);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        if (n0 + 8 * j < p.N)
-                            dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-                }
+                if (m < p.M) store_row128(p.c + m * p.N, packed, n0, p.N, wide);
                 __syncwarp();  // every lane has read the bias before the next tile's is written
             }
         } else {
@@ -461,21 +474,26 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
 
 // ---------------------------------------------------------------- GEMM on CTA pairs
 // The same product on pairs of CTAs (clusters of two) with tcgen05's two-CTA MMA: a
-// pair owns a 256 x 256 output tile.  CTA r of the pair loads rows 128 r .. + 127 of the
-// tile's A and of its B, the scales of its A rows and the scales of all 256 B rows; the
-// leader (r = 0) issues, for both CTAs, the scale copies into TMEM
-// (tcgen05.cp.cta_group::2) and the MMAs (tcgen05.mma.cta_group::2, M = 256, N = 256,
-// K = 64), which read A from each CTA's own shared memory and B from both, and leave
-// rows 128 r .. + 127 x 256 columns of the accumulator in CTA r's TMEM.  Each CTA moves
-// 38 KB per K-tile instead of the 54 KB of a 128 x 256 tile on one CTA, for the same
-// number of MMA cycles per SM.  Built when SBSA_NVFP4_PAIR is 1: parity-tested, but
-// measured slower than the one-CTA kernel above, whose bound is the scale copies into
-// TMEM (each SM still makes three per 128-cycle MMA), not the loads.
-//   Both CTAs' copies complete on the leader's stage barrier (two-CTA TMA), whose
-//   expected bytes the leader sets for both; the leader's commits arrive on the stage's
-//   free barrier and, at the end of a tile, the accumulator barrier of both CTAs; each
-//   CTA's epilogue hands the accumulator back by arriving on the leader's barrier.
+// pair owns a 256 x 256 output tile, so each SM loads 38 KB per K-tile instead of the
+// 54 KB of a 128 x 256 tile on one CTA, for the same number of MMA cycles (the load
+// path, about 61 bytes per clock per SM from L2, bounds the one-CTA kernel).
+//   warp 0      (both CTAs) loads this CTA's 128 rows of the tile's A and of its B with
+//               two-CTA TMA, whose bytes complete on the leader's stage barrier, and the
+//               scales of its A rows and of all 256 B rows with bulk copies on its own
+//               barrier;
+//   warp 1      (leader) issues the MMAs (tcgen05.mma.cta_group::2, M = 256, N = 256,
+//               K = 64), which read A from each CTA's shared memory and B from both and
+//               leave rows 128 r .. + 127 of the accumulator in CTA r's TMEM;
+//   warps 2-9   (both CTAs) epilogue as in the one-CTA kernel;
+//   warps 10-13 (both CTAs) store this CTA's scales into its TMEM.
+// The leader's commits arrive on the stage's free barrier and, at the end of a tile, the
+// accumulator barrier of both CTAs.  The other CTA's hand-overs to the leader (scales
+// stored, accumulator read) are relaxed remote arrivals made after tcgen05.wait::st /
+// ::ld returned: with release semantics each took about 1,400 cycles and the kernel ran
+// at a third of the speed.
 struct Nvfp4Gemm2Params {
+    const uint8_t* sfa;
+    const uint8_t* sfb;
     const float* amax_a;
     const float* amax_b;
     const float* bias;  // [N] or null
@@ -491,11 +509,15 @@ constexpr int kF2Half = 128 * 128;                   // 128 rows x 128 bytes of 
 constexpr int kF2SfaBytes = 4 * 512;                 // this CTA's A rows, one K-tile
 constexpr int kF2SfbBytes = 2 * 4 * 512;             // all 256 B rows of the tile, one K-tile
 constexpr int kF2StageBytes = 2 * kF2Half + kF2SfaBytes + kF2SfbBytes;
-constexpr int kF2BarOff = kF2Stages * kF2StageBytes;
-constexpr int kF2NumBars = 2 * kF2Stages + 3;  // full[S] (leader's counts both CTAs), empty[S], acc_full, acc_empty, drain
+constexpr int kF2BiasOff = kF2Stages * kF2StageBytes;  // each epilogue warp's 128 bias values of the tile
+constexpr int kF2BarOff = kF2BiasOff + 8 * 128 * 4;
+// full[S] (leader: both CTAs' codes), sf_in[S] (this CTA's scales landed), sf_full[S]
+// (leader: both CTAs' scales in TMEM), empty[S], acc_full, acc_empty, drain
+constexpr int kF2NumBars = 4 * kF2Stages + 3;
 constexpr int kF2SmemBytes = kF2BarOff + kF2NumBars * 8 + 16 + 1024;
 static_assert(kF2StageBytes % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
 static_assert(kF2SmemBytes <= 232448, "shared memory");
+static_assert(kFp4ColSf + kF2Stages * kFp4SfStageCols <= 512, "accumulator and scale regions fit in TMEM");
 
 __device__ __forceinline__ void umma_nvfp4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                                 uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
@@ -505,9 +527,6 @@ __device__ __forceinline__ void umma_nvfp4_pair(uint32_t d_tmem, uint64_t a_desc
             d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
         : "memory");
-}
-__device__ __forceinline__ void tmem_cp_pair_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 // Arrive on the barrier at this shared offset in both CTAs of the pair once the
 // tensor-core work issued so far has completed.
@@ -533,16 +552,17 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
         : "memory");
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4PairThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4Threads, 1)
     nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                           const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
                            const Nvfp4Gemm2Params p) {
     extern __shared__ __align__(1024) uint8_t fp4p_smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fp4p_smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kF2BarOff);
     uint64_t* full = bars;
-    uint64_t* empty = bars + kF2Stages;
-    uint64_t* acc_full = bars + 2 * kF2Stages;
+    uint64_t* sf_in = bars + kF2Stages;
+    uint64_t* sf_full = bars + 2 * kF2Stages;
+    uint64_t* empty = bars + 3 * kF2Stages;
+    uint64_t* acc_full = bars + 4 * kF2Stages;
     uint64_t* acc_empty = acc_full + 1;
     uint64_t* drain = acc_full + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kF2NumBars);
@@ -556,11 +576,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4PairThreads, 1)
     const int n_pairs = gridDim.x / 2;
     const int num_tiles = p.tiles_m * p.tiles_n;
     const int k_tiles = p.K / kFp4TileK;
+    const int my_tiles = pair < num_tiles ? (num_tiles - 1 - pair) / n_pairs + 1 : 0;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         for (int s = 0; s < kF2Stages; ++s) {
             mbar_init(&full[s], 1);
+            mbar_init(&sf_in[s], 1);
+            mbar_init(&sf_full[s], 8);  // four scale warps in each CTA
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_full, 1);
@@ -569,8 +592,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4PairThreads, 1)
         fence_mbar_init();
         tma_prefetch_desc(&map_a);
         tma_prefetch_desc(&map_b);
-        tma_prefetch_desc(&map_sfa);
-        tma_prefetch_desc(&map_sfb);
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -592,41 +613,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4PairThreads, 1)
         if (!*abort_flag) give_up();
         return false;
     };
+    // a hand-over to the leader after this thread waited for its TMEM accesses: a plain
+    // arrival in the leader, a relaxed remote one from the other CTA
+    auto arrive_leader = [&](uint64_t* bar) {
+        if (leader) mbar_arrive(bar);
+        else mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(bar), 0));
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0 && !launch_aborted(p.epoch)) {
             const uint64_t pol_a = policy_evict_normal();
             const uint64_t pol_b = policy_evict_last();
-            const int k_atoms = p.K / 64;
+            const size_t k_atoms = static_cast<size_t>(p.K / 64);
             int it = 0;
             bool ok = true;
             for (int tile = pair; ok && tile < num_tiles; tile += n_pairs) {
                 const int tm = tile / p.tiles_n;
                 const int tn = tile % p.tiles_n;
-                // scale groups that do not exist (past the padded rows) are replaced by the
-                // last one: they only feed rows and columns that are never stored
-                const int ga = min(tm * 2 + static_cast<int>(rank), p.groups_a - 1);
-                const int gb0 = min(tn * 2, p.groups_b - 1);
-                const int gb1 = min(tn * 2 + 1, p.groups_b - 1);
+                // this CTA's rows of the tile's A and B, and the tile's scale groups; groups
+                // that do not exist (past the padded rows) are replaced by the last one: they
+                // only feed rows and columns that are never stored
+                const int ra = tm * 256 + static_cast<int>(rank) * 128;
+                const int rb = tn * 256 + static_cast<int>(rank) * 128;
+                const size_t ga = static_cast<size_t>(min(tm * 2 + static_cast<int>(rank), p.groups_a - 1));
+                const size_t gb0 = static_cast<size_t>(min(tn * 2, p.groups_b - 1));
+                const size_t gb1 = static_cast<size_t>(min(tn * 2 + 1, p.groups_b - 1));
                 for (int kt = 0; kt < k_tiles; ++kt, ++it) {
                     const int s = it % kF2Stages;
                     if (!(ok = wait(&empty[s], ((it / kF2Stages) & 1) ^ 1))) break;
                     uint8_t* st = smem + s * kF2StageBytes;
                     const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
-                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * kF2StageBytes);
-                    tma_load_2d_pair(st, &map_a, bar, kt * 128, tm * 256 + static_cast<int>(rank) * 128, pol_a);
-                    tma_load_2d_pair(st + kF2Half, &map_b, bar, kt * 128, tn * 256 + static_cast<int>(rank) * 128, pol_b);
-                    tma_load_2d_pair(st + 2 * kF2Half, &map_sfa, bar, 0, ga * k_atoms + 4 * kt, pol_a);
-                    tma_load_2d_pair(st + 2 * kF2Half + kF2SfaBytes, &map_sfb, bar, 0, gb0 * k_atoms + 4 * kt, pol_b);
-                    tma_load_2d_pair(st + 2 * kF2Half + kF2SfaBytes + 2048, &map_sfb, bar, 0, gb1 * k_atoms + 4 * kt, pol_b);
+                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * 2 * kF2Half);
+                    tma_load_2d_pair(st, &map_a, bar, kt * 128, ra, pol_a);
+                    tma_load_2d_pair(st + kF2Half, &map_b, bar, kt * 128, rb, pol_b);
+                    mbar_arrive_expect_tx(&sf_in[s], kF2SfaBytes + kF2SfbBytes);
+                    bulk_load_g2s(st + 2 * kF2Half, p.sfa + (ga * k_atoms + 4 * kt) * 512, 2048, &sf_in[s]);
+                    bulk_load_g2s(st + 2 * kF2Half + kF2SfaBytes, p.sfb + (gb0 * k_atoms + 4 * kt) * 512, 2048, &sf_in[s]);
+                    bulk_load_g2s(st + 2 * kF2Half + kF2SfaBytes + 2048, p.sfb + (gb1 * k_atoms + 4 * kt) * 512, 2048,
+                                  &sf_in[s]);
                 }
             }
-            if (!ok && leader) {
+            if (!ok) {
                 // every copy issued for the stages still pending must land before the pair exits
                 volatile int never = 0;
-                for (int q = it - kF2Stages < 0 ? 0 : it - kF2Stages; q < it; ++q)
-                    mbar_wait_bounded_cluster(&full[q % kF2Stages], (q / kF2Stages) & 1, &never, kWaitLimitNs);
+                for (int q = it - kF2Stages < 0 ? 0 : it - kF2Stages; q < it; ++q) {
+                    if (leader) mbar_wait_bounded_cluster(&full[q % kF2Stages], (q / kF2Stages) & 1, &never, kWaitLimitNs);
+                    mbar_wait_bounded_cluster(&sf_in[q % kF2Stages], (q / kF2Stages) & 1, &never, kWaitLimitNs);
+                }
             }
         }
     } else if (warp == 1) {
@@ -642,18 +676,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4PairThreads, 1)
                 for (int kt = 0; kt < k_tiles; ++kt, ++it) {
                     const int s = it % kF2Stages;
                     if (!(ok = wait(&full[s], (it / kF2Stages) & 1))) break;
+                    // both CTAs' scales of the stage are in their TMEM regions
+                    if (!(ok = wait(&sf_full[s], (it / kF2Stages) & 1))) break;
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + s * kF2StageBytes);
-                    const uint32_t sfa = st + 2 * kF2Half;
-                    const uint32_t sfb = sfa + kF2SfaBytes;
-                    const uint32_t t_sfa = tmem + kFp4ColSf + (it & 1) * kFp4SfRegion;
+                    const uint32_t t_sfa = tmem + kFp4ColSf + static_cast<uint32_t>(s) * kFp4SfStageCols;
                     const uint32_t t_sfb = t_sfa + 16;
-#pragma unroll
-                    for (int kb = 0; kb < 4; ++kb) {
-                        tmem_cp_pair_32x128b_warpx4(t_sfa + 4 * kb, sdesc_atom(sfa + kb * 512));
-                        tmem_cp_pair_32x128b_warpx4(t_sfb + 8 * kb, sdesc_atom(sfb + kb * 512));
-                        tmem_cp_pair_32x128b_warpx4(t_sfb + 8 * kb + 4, sdesc_atom(sfb + 2048 + kb * 512));
-                    }
                     const uint64_t a0 = sdesc_sw128(st, 16, 1024);
                     const uint64_t b0 = sdesc_sw128(st + kF2Half, 16, 1024);
 #pragma unroll
@@ -671,46 +699,83 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4PairThreads, 1)
                 mbar_wait_bounded_cluster(drain, 0, &never, kWaitLimitNs);
             }
         }
-    } else {
+    } else if (warp < 10) {
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int quarter = warp & 3;
         const int half = (warp - 2) >> 2;
         const uint32_t t_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(half * 128);
-        const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
         const float alpha = __frcp_rn(__fmul_rn(nvfp4_tensor_scale(__ldg(p.amax_a)), nvfp4_tensor_scale(__ldg(p.amax_b))));
+        const bool wide = (reinterpret_cast<uintptr_t>(p.c) & 31u) == 0 && p.N % 16 == 0;
+        const uint32_t bias_w = smem_u32(smem + kF2BiasOff) + static_cast<uint32_t>((warp - 2) * 128 * 4);
         int tcount = 0;
         for (int tile = pair; tile < num_tiles && !launch_aborted(p.epoch); tile += n_pairs, ++tcount) {
             const int tm = tile / p.tiles_n;
             const int tn = tile % p.tiles_n;
-            const bool ok = __all_sync(0xFFFFFFFFu, wait(acc_full, tcount & 1));
-            if (!ok) break;
-            tc_fence_after();
             const int n0 = tn * 256 + half * 128;
+            // the bias goes to shared memory while the tile is still being computed
+            {
+                float b[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int n = n0 + 4 * lane + e;
+                    b[e] = (p.bias && n < p.N) ? __ldg(p.bias + n) : 0.f;
+                }
+                st_shared_v4(bias_w + lane * 16, __float_as_uint(b[0]), __float_as_uint(b[1]), __float_as_uint(b[2]),
+                             __float_as_uint(b[3]));
+                __syncwarp();
+            }
+            if (!__all_sync(0xFFFFFFFFu, wait(acc_full, tcount & 1))) break;
+            tc_fence_after();
             uint32_t packed[64];
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t raw[64];
-                tmem_ld64(t_row + c * 64, raw);
+                tmem_ld64(t_row + c * 64, raw);  // returns after tcgen05.wait::ld
 #pragma unroll
-                for (int e = 0; e < 64; e += 2) {
-                    const int n = n0 + c * 64 + e;
-                    const float b0 = (p.bias && n < p.N) ? __ldg(p.bias + n) : 0.f;
-                    const float b1 = (p.bias && n + 1 < p.N) ? __ldg(p.bias + n + 1) : 0.f;
-                    packed[c * 32 + e / 2] = pack_bf16x2(fmaf(__uint_as_float(raw[e]), alpha, b0),
-                                                         fmaf(__uint_as_float(raw[e + 1]), alpha, b1));
+                for (int e = 0; e < 64; e += 4) {
+                    uint32_t b0, b1, b2, b3;
+                    ld_shared_v4(bias_w + (c * 64 + e) * 4, b0, b1, b2, b3);
+                    packed[c * 32 + e / 2] = pack_bf16x2(fmaf(__uint_as_float(raw[e]), alpha, __uint_as_float(b0)),
+                                                         fmaf(__uint_as_float(raw[e + 1]), alpha, __uint_as_float(b1)));
+                    packed[c * 32 + e / 2 + 1] = pack_bf16x2(fmaf(__uint_as_float(raw[e + 2]), alpha, __uint_as_float(b2)),
+                                                             fmaf(__uint_as_float(raw[e + 3]), alpha, __uint_as_float(b3)));
                 }
             }
+            // the accumulator is in registers: the next tile's MMAs may overwrite it
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+            if (lane == 0) arrive_leader(acc_empty);
             const long long m = static_cast<long long>(tm) * 256 + static_cast<int>(rank) * 128 + quarter * 32 + lane;
-            if (m < p.M) {
-                uint4* dst = reinterpret_cast<uint4*>(p.c + m * p.N + n0);
+            if (m < p.M) store_row128(p.c + m * p.N, packed, n0, p.N, wide);
+            __syncwarp();  // every lane has read the bias before the next tile's is written
+        }
+    } else {
+        // ------------------------------------------------------------ scales (warps 10-13, both CTAs)
+        // this CTA's scales of K-tile i into its TMEM region i % S, in the layout of the
+        // one-CTA kernel (A: its 128 rows; B: all 256 rows of the tile)
+        const int quarter = warp & 3;
+        const int total = my_tiles * k_tiles;
+        for (int i = 0; i < total; ++i) {
+            const int s = i % kF2Stages;
+            if (!__all_sync(0xFFFFFFFFu, wait(&sf_in[s], (i / kF2Stages) & 1))) break;
+            const uint32_t base = smem_u32(smem + s * kF2StageBytes + 2 * kF2Half) + lane * 16;
+            uint32_t va[16], vb[32];
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    if (n0 + 8 * j < p.N)
-                        dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+            for (int kb = 0; kb < 4; ++kb) {
+                ld_shared_v4(base + kb * 512, va[4 * kb], va[4 * kb + 1], va[4 * kb + 2], va[4 * kb + 3]);
+#pragma unroll
+                for (int g = 0; g < 2; ++g)
+                    ld_shared_v4(base + kF2SfaBytes + g * 2048 + kb * 512, vb[8 * kb + 4 * g], vb[8 * kb + 4 * g + 1],
+                                 vb[8 * kb + 4 * g + 2], vb[8 * kb + 4 * g + 3]);
             }
+            const uint32_t t = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kFp4ColSf +
+                               static_cast<uint32_t>(s) * kFp4SfStageCols;
+            tmem_st16(t, va);
+            tmem_st32(t + 16, vb);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive_leader(&sf_full[s]);
         }
     }
 

@@ -29,7 +29,7 @@
 // than one CTA per 128 x 256 tile (1.80 vs 1.67 ms on 32,768 x 15,360 x 5,120): the scale
 // copies into TMEM, not the loads, bound both, and the pair adds cross-CTA hand-overs.
 #ifndef SBSA_NVFP4_PAIR
-#define SBSA_NVFP4_PAIR 0
+#define SBSA_NVFP4_PAIR 1
 #endif
 
 namespace sbsa {
@@ -166,22 +166,6 @@ sbsa_status make_map_fp4(CUtensorMap* m, const void* base, long long rows, int K
     return SBSA_OK;
 }
 
-// NVFP4 scale array viewed as 512-byte atoms ([atoms][128] uint32); a box is the 4 atoms
-// of one K-tile of one 128-row group (2 KB), no swizzle.
-sbsa_status make_map_scales(CUtensorMap* m, const void* base, long long atoms) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return fail(SBSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-    cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(atoms)};
-    cuuint64_t strides[1] = {512};
-    cuuint32_t box[2] = {128, 4};
-    cuuint32_t es[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(SBSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
-    return SBSA_OK;
-}
-
 int sm_count() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -216,7 +200,6 @@ sbsa_status ulysses_dims(const sbsa_ulysses_shape* s, int32_t head0, int32_t hea
     return SBSA_OK;
 }
 
-bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
 
 // ---------------------------------------------------------------- launchers
 sbsa_status launch_pool(const sbsa_shape* s, const void* q, const void* k, float* qm, float* km, cudaStream_t st) {
@@ -728,9 +711,11 @@ sbsa_status sbsa_nvfp4_gemm(int32_t m, int32_t n, int32_t k, const void* a, cons
 #if SBSA_NVFP4_PAIR
     {
         // pairs of CTAs, 256 x 256 tiles
-        CUtensorMap ma, mb, msa, msb;
+        CUtensorMap ma, mb;
         sbsa_status r;
         Nvfp4Gemm2Params q;
+        q.sfa = static_cast<const uint8_t*>(a_scales);
+        q.sfb = static_cast<const uint8_t*>(b_scales);
         q.amax_a = a_amax;
         q.amax_b = b_amax;
         q.bias = bias;
@@ -745,16 +730,13 @@ sbsa_status sbsa_nvfp4_gemm(int32_t m, int32_t n, int32_t k, const void* a, cons
         q.epoch = g_epoch.fetch_add(1);
         if ((r = make_map_fp4(&ma, a, m, k, 128)) != SBSA_OK) return r;
         if ((r = make_map_fp4(&mb, b, n, k, 128)) != SBSA_OK) return r;
-        if ((r = make_map_scales(&msa, a_scales, static_cast<long long>(q.groups_a) * (k / 64))) != SBSA_OK) return r;
-        if ((r = make_map_scales(&msb, b_scales, static_cast<long long>(q.groups_b) * (k / 64))) != SBSA_OK) return r;
         const long long tiles = static_cast<long long>(q.tiles_m) * q.tiles_n;
         if (tiles > 0x3FFFFFFFLL) return fail(SBSA_ERR_UNSUPPORTED, "too many tiles");
         const int pairs = static_cast<int>(tiles < sm_count() / 2 ? tiles : sm_count() / 2);
         cudaError_t e = cudaFuncSetAttribute(nvfp4_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kF2SmemBytes);
         if (e != cudaSuccess) return cuda_fail(e, "nvfp4 gemm smem attribute");
-        nvfp4_gemm_pair_kernel<<<2 * pairs, kFp4PairThreads, kF2SmemBytes, static_cast<cudaStream_t>(stream)>>>(ma, mb, msa,
-                                                                                                       msb, q);
+        nvfp4_gemm_pair_kernel<<<2 * pairs, kFp4Threads, kF2SmemBytes, static_cast<cudaStream_t>(stream)>>>(ma, mb, q);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "nvfp4 gemm launch");
         return ok();
