@@ -554,22 +554,28 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                 if (use1) tmem_ld_cols<HD>(tmem + lane_base + C::kColO0 + 128 + g * HD, o1);
             }
             if (row_in_block) {
-                uint4* dst = reinterpret_cast<uint4*>(p.o + (bh * p.Lp + t) * D + g * HD);
+                __nv_bfloat16* dst = p.o + (bh * p.Lp + t) * D + g * HD;
+                const bool wide = (reinterpret_cast<uintptr_t>(p.o) & 31u) == 0;
 #pragma unroll
-                for (int e = 0; e < HD; e += 8) {
-                    float v[8];
+                for (int e = 0; e < HD; e += 16) {
+                    uint32_t w[8];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        float x = write_o ? __uint_as_float(o0[e + q]) * c0 : 0.f;
-                        if (write_o && use1) x = fmaf(__uint_as_float(o1[e + q]), c1, x);
-                        v[q] = x;
+                    for (int q = 0; q < 16; q += 2) {
+                        float x0 = write_o ? __uint_as_float(o0[e + q]) * c0 : 0.f;
+                        float x1 = write_o ? __uint_as_float(o0[e + q + 1]) * c0 : 0.f;
+                        if (write_o && use1) {
+                            x0 = fmaf(__uint_as_float(o1[e + q]), c1, x0);
+                            x1 = fmaf(__uint_as_float(o1[e + q + 1]), c1, x1);
+                        }
+                        w[q / 2] = pack_bf16x2(x0, x1);
                     }
-                    uint4 w;
-                    w.x = pack_bf16x2(v[0], v[1]);
-                    w.y = pack_bf16x2(v[2], v[3]);
-                    w.z = pack_bf16x2(v[4], v[5]);
-                    w.w = pack_bf16x2(v[6], v[7]);
-                    dst[e / 8] = w;
+                    if (wide) {
+                        st_global_v8(dst + e, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+                    } else {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + e);
+                        d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                    }
                 }
             }
         }

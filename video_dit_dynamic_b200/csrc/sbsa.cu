@@ -197,6 +197,12 @@ sbsa_status ulysses_dims(const sbsa_ulysses_shape* s, int32_t head0, int32_t hea
     // the kernels index rows in 32 bits
     const long long rows = static_cast<long long>(u->G) * u->Lr * 3 * u->hc + 3LL * u->hc * (u->Lp - u->L);
     if (rows >= (1LL << 31)) return fail(SBSA_ERR_UNSUPPORTED, "head chunk of 2^31 rows or more");
+    const uint32_t pad = static_cast<uint32_t>(u->Lp - u->L);
+    u->by_qkv_peer = make_fastdiv(static_cast<uint32_t>(u->Lr) * 3u * static_cast<uint32_t>(u->hc));
+    u->by_o_peer = make_fastdiv(static_cast<uint32_t>(u->Lr) * static_cast<uint32_t>(u->hc));
+    u->by_hc = make_fastdiv(static_cast<uint32_t>(u->hc));
+    u->by_pad = make_fastdiv(pad > 0 ? pad : 1u);  // used only when there are padded tokens
+    u->by_pad_hc = make_fastdiv(pad > 0 ? pad * static_cast<uint32_t>(u->hc) : 1u);
     return SBSA_OK;
 }
 

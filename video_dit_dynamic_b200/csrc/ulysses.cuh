@@ -30,8 +30,29 @@
 
 namespace sbsa {
 
+// Division of n < 2^31 by an invariant d >= 1 with one 64-bit multiply and a shift
+// (Granlund and Montgomery, "Division by invariant integers using multiplication", 1994,
+// theorem 4.2 with N = 31): l = ceil(log2 d), s = 31 + l, m = floor(2^s / d) + 1; then
+// 2^s < m d <= 2^s + 2^l and floor(n / d) = floor(n m / 2^s) for every n < 2^31.
+struct FastDiv {
+    unsigned long long m;
+    unsigned int s;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+    unsigned int l = 0;
+    while ((1ull << l) < d) ++l;
+    const unsigned int s = 31 + l;
+    return {(1ull << s) / d + 1, s};
+}
+__device__ __forceinline__ uint32_t udiv(uint32_t n, const FastDiv& f) {
+    return static_cast<uint32_t>((static_cast<unsigned long long>(n) * f.m) >> f.s);
+}
+
 struct UlyssesDims {
     int G, Lr, L, Lp, H, Hg, h0, hc;
+    // divisors of the row decompositions: rows per peer of a QKV and of an O exchange,
+    // the chunk's heads, the padded tokens, and hc times the padded tokens
+    FastDiv by_qkv_peer, by_o_peer, by_hc, by_pad, by_pad_hc;
 };
 
 // Two e4m3 codes (low byte first) -> their exact values as fp32 (e4m3 is a subset of
@@ -43,7 +64,7 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two_codes) {
 }
 
 constexpr int kUlyD = 128;          // head_dim handled by these kernels
-constexpr int kUlyRowsPerWarp = 8;  // 16 lanes per row (8 values each), 4 row pairs per warp
+constexpr int kUlyRowsPerWarp = 16;  // 8 lanes per row (16 values each), 4 rows per step, 4 steps
 constexpr int kUlyRowsPerCta = 8 * kUlyRowsPerWarp;
 
 // slices are padded to 16 bytes, so every slice's codes start 16-byte aligned
@@ -67,9 +88,9 @@ struct RowPtrs {
 __device__ __forceinline__ RowPtrs qkv_pack_row(uint32_t w, const __nv_bfloat16* x, uint8_t* send,
                                                 const UlyssesDims& u) {
     const uint32_t per_peer = static_cast<uint32_t>(u.Lr) * 3u * static_cast<uint32_t>(u.hc);
-    const uint32_t j = w / per_peer;
+    const uint32_t j = udiv(w, u.by_qkv_peer);
     const uint32_t row = w - j * per_peer;  // (t * 3 + c) * hc + hh
-    const uint32_t tc = row / static_cast<uint32_t>(u.hc);
+    const uint32_t tc = udiv(row, u.by_hc);
     const uint32_t hh = row - tc * static_cast<uint32_t>(u.hc);
     uint8_t* slice = send + static_cast<size_t>(j) * ulysses_qkv_slice_bytes(u);
     const size_t src = (static_cast<size_t>(tc) * u.H + j * u.Hg + u.h0 + hh) * kUlyD;
@@ -80,9 +101,9 @@ __device__ __forceinline__ RowPtrs qkv_pack_row(uint32_t w, const __nv_bfloat16*
 __device__ __forceinline__ RowPtrs o_pack_row(uint32_t w, const __nv_bfloat16* o, uint8_t* send,
                                               const UlyssesDims& u) {
     const uint32_t per_peer = static_cast<uint32_t>(u.Lr) * static_cast<uint32_t>(u.hc);
-    const uint32_t j = w / per_peer;
+    const uint32_t j = udiv(w, u.by_o_peer);
     const uint32_t row = w - j * per_peer;  // t * hc + hh
-    const uint32_t t = row / static_cast<uint32_t>(u.hc);
+    const uint32_t t = udiv(row, u.by_hc);
     const uint32_t hh = row - t * static_cast<uint32_t>(u.hc);
     const size_t token = static_cast<size_t>(j) * u.Lr + t;
     uint8_t* slice = send + static_cast<size_t>(j) * ulysses_o_slice_bytes(u);
@@ -96,9 +117,9 @@ __device__ __forceinline__ RowPtrs qkv_unpack_row(uint32_t w, const uint8_t* rec
     const uint32_t per_peer = static_cast<uint32_t>(u.Lr) * 3u * static_cast<uint32_t>(u.hc);
     const uint32_t n_rows = per_peer * static_cast<uint32_t>(u.G);
     if (w < n_rows) {
-        const uint32_t i = w / per_peer;
+        const uint32_t i = udiv(w, u.by_qkv_peer);
         const uint32_t row = w - i * per_peer;
-        const uint32_t tc = row / static_cast<uint32_t>(u.hc);
+        const uint32_t tc = udiv(row, u.by_hc);
         const uint32_t hh = row - tc * static_cast<uint32_t>(u.hc);
         const uint32_t t3 = tc / 3u;
         const uint32_t c = tc - 3u * t3;
@@ -113,9 +134,9 @@ __device__ __forceinline__ RowPtrs qkv_unpack_row(uint32_t w, const uint8_t* rec
     const uint32_t z = w - n_rows;  // padded rows (c, hh, token - L)
     const uint32_t pad = static_cast<uint32_t>(u.Lp - u.L);
     const uint32_t per_c = static_cast<uint32_t>(u.hc) * pad;
-    const uint32_t c = z / per_c;
+    const uint32_t c = udiv(z, u.by_pad_hc);
     const uint32_t rem = z - c * per_c;
-    const uint32_t hh = rem / pad;
+    const uint32_t hh = udiv(rem, u.by_pad);
     __nv_bfloat16* t = c == 0 ? q : (c == 1 ? k : v);
     return {nullptr, t + (static_cast<size_t>(u.h0 + hh) * u.Lp + u.L + (rem - hh * pad)) * kUlyD, nullptr, true};
 }
@@ -123,9 +144,9 @@ __device__ __forceinline__ RowPtrs qkv_unpack_row(uint32_t w, const uint8_t* rec
 __device__ __forceinline__ RowPtrs o_unpack_row(uint32_t w, const uint8_t* recv, __nv_bfloat16* y,
                                                 const UlyssesDims& u) {
     const uint32_t per_peer = static_cast<uint32_t>(u.Lr) * static_cast<uint32_t>(u.hc);
-    const uint32_t i = w / per_peer;
+    const uint32_t i = udiv(w, u.by_o_peer);
     const uint32_t row = w - i * per_peer;
-    const uint32_t t = row / static_cast<uint32_t>(u.hc);
+    const uint32_t t = udiv(row, u.by_hc);
     const uint32_t hh = row - t * static_cast<uint32_t>(u.hc);
     const uint8_t* slice = recv + static_cast<size_t>(i) * ulysses_o_slice_bytes(u);
     return {reinterpret_cast<const uint4*>(slice + static_cast<size_t>(row) * kUlyD),
@@ -134,79 +155,93 @@ __device__ __forceinline__ RowPtrs o_unpack_row(uint32_t w, const uint8_t* recv,
             false};
 }
 
-// Quantize rows [first, first + 8) of a pack (rows >= n_rows skipped): half-warp h takes
-// rows first + 2 s + h, lane l % 16 the 8 values 8 (l % 16) .. + 7; all loads are issued
-// before any is used.
+// Quantize rows [first, first + 16) of a pack (rows >= n_rows skipped): step s takes
+// rows first + 4 s + lane / 8, and lane l = lane % 8 the values 8 l .. + 7 and
+// 64 + 8 l .. + 7 of its row, so that every load and store of a warp covers whole
+// 32-byte sectors of four rows; all loads are issued before any is used.
 template <typename RowFn>
 __device__ __forceinline__ void pack_rows(uint32_t first, uint32_t n_rows, RowFn row_of) {
-    const int lane = threadIdx.x % 32, h = lane / 16, l = lane % 16;
-    uint4 in[4];
+    const int lane = threadIdx.x % 32, h = lane / 8, l = lane % 8;
+    uint4 in[4][2];
     RowPtrs rp[4];
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-        const uint32_t w = first + 2u * s + h;
-        in[s] = make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t w = first + 4u * s + h;
+        in[s][0] = in[s][1] = make_uint4(0u, 0u, 0u, 0u);
         if (w < n_rows) {
             rp[s] = row_of(w);
-            in[s] = __ldg(rp[s].src + l);
+            in[s][0] = __ldg(rp[s].src + l);
+            in[s][1] = __ldg(rp[s].src + 8 + l);
         }
     }
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-        const uint32_t w = first + 2u * s + h;
-        const uint32_t wd[4] = {in[s].x, in[s].y, in[s].z, in[s].w};
-        float vals[8];
+        const uint32_t w = first + 4u * s + h;
+        const uint32_t wd[8] = {in[s][0].x, in[s][0].y, in[s][0].z, in[s][0].w,
+                                in[s][1].x, in[s][1].y, in[s][1].z, in[s][1].w};
+        float vals[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
+        for (int e = 0; e < 8; ++e) {
             vals[2 * e] = __uint_as_float(wd[e] << 16);
             vals[2 * e + 1] = __uint_as_float(wd[e] & 0xFFFF0000u);
         }
         float amax = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(vals[e]));
+        for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(vals[e]));
 #pragma unroll
-        for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+        for (int off = 4; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
         if (w >= n_rows) continue;  // (after the shuffles, which every lane takes part in)
         const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
-        uint32_t c2[4];
+        uint32_t c2[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) c2[e] = cvt_e4m3x2(__fmul_rn(vals[2 * e], inv), __fmul_rn(vals[2 * e + 1], inv));
-        reinterpret_cast<uint2*>(rp[s].dst)[l] = make_uint2(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16));
+        for (int e = 0; e < 8; ++e) c2[e] = cvt_e4m3x2(__fmul_rn(vals[2 * e], inv), __fmul_rn(vals[2 * e + 1], inv));
+        uint2* dst = reinterpret_cast<uint2*>(rp[s].dst);
+        dst[l] = make_uint2(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16));
+        dst[8 + l] = make_uint2(c2[4] | (c2[5] << 16), c2[6] | (c2[7] << 16));
         if (l == 0) *rp[s].scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
     }
 }
 
-// Restore rows [first, first + 8) (rows >= n_rows skipped), same thread layout.
+// Restore rows [first, first + 16) (rows >= n_rows skipped), same thread layout.
 template <typename RowFn>
 __device__ __forceinline__ void unpack_rows(uint32_t first, uint32_t n_rows, RowFn row_of) {
-    const int lane = threadIdx.x % 32, h = lane / 16, l = lane % 16;
-    uint2 in[4];
+    const int lane = threadIdx.x % 32, h = lane / 8, l = lane % 8;
+    uint2 in[4][2];
     float sc[4];
     RowPtrs rp[4];
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-        const uint32_t w = first + 2u * s + h;
+        const uint32_t w = first + 4u * s + h;
         if (w < n_rows) {
             rp[s] = row_of(w);
             if (!rp[s].zero) {
-                in[s] = __ldg(reinterpret_cast<const uint2*>(rp[s].src) + l);
+                const uint2* src = reinterpret_cast<const uint2*>(rp[s].src);
+                in[s][0] = __ldg(src + l);
+                in[s][1] = __ldg(src + 8 + l);
                 sc[s] = __ldg(rp[s].scale);
             }
         }
     }
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-        const uint32_t w = first + 2u * s + h;
+        const uint32_t w = first + 4u * s + h;
         if (w >= n_rows) continue;
-        uint4 out = make_uint4(0u, 0u, 0u, 0u);
+        uint4 out[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
         if (!rp[s].zero) {
-            const float2 a = e4m3x2_to_float2(in[s].x), b = e4m3x2_to_float2(in[s].x >> 16);
-            const float2 c = e4m3x2_to_float2(in[s].y), d = e4m3x2_to_float2(in[s].y >> 16);
             const float k = sc[s];
-            out = make_uint4(pack_bf16x2(__fmul_rn(a.x, k), __fmul_rn(a.y, k)), pack_bf16x2(__fmul_rn(b.x, k), __fmul_rn(b.y, k)),
-                             pack_bf16x2(__fmul_rn(c.x, k), __fmul_rn(c.y, k)), pack_bf16x2(__fmul_rn(d.x, k), __fmul_rn(d.y, k)));
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                const float2 a = e4m3x2_to_float2(in[s][p].x), b = e4m3x2_to_float2(in[s][p].x >> 16);
+                const float2 c = e4m3x2_to_float2(in[s][p].y), d = e4m3x2_to_float2(in[s][p].y >> 16);
+                out[p] = make_uint4(pack_bf16x2(__fmul_rn(a.x, k), __fmul_rn(a.y, k)),
+                                    pack_bf16x2(__fmul_rn(b.x, k), __fmul_rn(b.y, k)),
+                                    pack_bf16x2(__fmul_rn(c.x, k), __fmul_rn(c.y, k)),
+                                    pack_bf16x2(__fmul_rn(d.x, k), __fmul_rn(d.y, k)));
+            }
         }
-        reinterpret_cast<uint4*>(rp[s].dst)[l] = out;
+        uint4* dst = reinterpret_cast<uint4*>(rp[s].dst);
+        dst[l] = out[0];
+        dst[8 + l] = out[1];
     }
 }
 
