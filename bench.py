@@ -113,7 +113,7 @@ def fp4_summary(fp4: dict, peaks: dict) -> dict:
     qgbs = fp4["quant_bytes"] / (fp4["quant_ms"] / 1e3) / 1e9
     return {"shape": {"m": fp4["m"], "n": fp4["n"], "k": fp4["k"]},
             "gemm": {"ms": fp4["gemm_ms"], "TFLOP/s": tf, "peak": fp4_peak, "frac": tf / fp4_peak,
-                     "kernel": "nvfp4_gemm_kernel", "algorithmic_flop": fp4["gemm_flop"],
+                     "kernel": "nvfp4_gemm_pair_kernel", "algorithmic_flop": fp4["gemm_flop"],
                      "algorithmic_bytes": fp4["gemm_bytes"],
                      "GB/s": fp4["gemm_bytes"] / (fp4["gemm_ms"] / 1e3) / 1e9},
             "amax_plus_quantize": {"ms": fp4["quant_ms"], "GB/s": qgbs, "hbm_frac": qgbs / peaks["hbm_gbs"],
