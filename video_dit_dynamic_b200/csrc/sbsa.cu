@@ -25,9 +25,9 @@
 #include "select.cuh"
 #include "ulysses.cuh"
 
-// 1: the NVFP4 GEMM on CTA pairs (256 x 256 tiles).  Parity-tested, but measured slower
-// than one CTA per 128 x 256 tile (1.80 vs 1.67 ms on 32,768 x 15,360 x 5,120): the scale
-// copies into TMEM, not the loads, bound both, and the pair adds cross-CTA hand-overs.
+// 1 (default): the NVFP4 GEMM on CTA pairs (256 x 256 tiles, 38 KB loaded per SM per K-tile);
+// 0: one CTA per 128 x 256 tile (54 KB).  Both parity-tested; on 32,768 x 15,360 x 5,120 the
+// pair kernel takes 1.15 ms, the one-CTA kernel 1.33 ms (the L2 -> SM load path bounds both).
 #ifndef SBSA_NVFP4_PAIR
 #define SBSA_NVFP4_PAIR 1
 #endif
