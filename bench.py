@@ -122,6 +122,12 @@ def fp4_summary(fp4: dict, peaks: dict) -> dict:
             "note": "QKV projection of the same tokens, timed apart from the step"}
 
 
+def spread(ms_list) -> dict:
+    """Median and best of this rank's per-step kernel times (the mean reported beside them is
+    the maximum over ranks)."""
+    return {"ms_median": statistics.median(ms_list), "ms_best": min(ms_list)}
+
+
 def job_tflops(flops_per_rank: float, world: int, ms: float) -> float:
     """Whole-job throughput: every rank's layer counted, divided by the slowest rank's time."""
     return flops_per_rank * world / (ms / 1e3) / 1e12
@@ -239,7 +245,8 @@ def recorded_traffic(kernel_src: str, workload_name: str):
 
 
 # ------------------------------------------------------------------ CPU oracle sample
-def cpu_oracle_sample(wl: inputs.Workload, k: int, q, kt, v, n_units: int, seed: int = 0):
+def cpu_oracle_sample(wl: inputs.Workload, k: int, q, kt, v, n_units: int, seed: int = 0,
+                      single_core_units: int = 0):
     """Time the oracle on a bounded sample of the layer: pool + select of one full head
     and attention of n_units (head 0, query block) units; extrapolate to the layer."""
     import numpy as np
@@ -265,13 +272,32 @@ def cpu_oracle_sample(wl: inputs.Workload, k: int, q, kt, v, n_units: int, seed:
     heads = wl.heads * wl.batch
     layer_s = t_ps * heads + t_at / len(units) * (nb * heads)
     tflops = layer_flops(wl, k) / layer_s / 1e12
-    return {
+    out = {
         "value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
         "sample": (f"pool+select of 1 of {heads} heads ({t_ps:.2f} s) and attention of {len(units)} of "
                    f"{nb * heads} (head, query-block) units ({t_at:.2f} s), extrapolated to the layer: "
                    f"{layer_s:.1f} s/layer"),
         "layer_seconds_extrapolated": layer_s,
     }
+    if single_core_units > 0:
+        # the same kind of sample on one core (fewer attention units)
+        oracle.set_threads(1)
+        try:
+            t0 = time.perf_counter()
+            col1 = oracle.select(oracle.pool(qb, L, blk), oracle.pool(kb, L, blk), k)
+            t_ps1 = time.perf_counter() - t0
+            units1 = units[:single_core_units]
+            t0 = time.perf_counter()
+            oracle.attention(qb, kb, vb, L, blk, rp, col1, units=units1)
+            t_at1 = time.perf_counter() - t0
+        finally:
+            oracle.set_threads(os.cpu_count() or 1)
+        layer_s1 = t_ps1 * heads + t_at1 / len(units1) * (nb * heads)
+        out["single_core"] = {
+            "value": layer_flops(wl, k) / layer_s1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+            "sample": (f"pool+select of 1 of {heads} heads ({t_ps1:.2f} s) and attention of {len(units1)} units "
+                       f"({t_at1:.2f} s) on one core, extrapolated to the layer: {layer_s1:.1f} s/layer")}
+    return out
 
 
 # ------------------------------------------------------------------ reference arm
@@ -609,11 +635,11 @@ def run_gpu(args, wl):
                          "frac_of_sustained": att_tflops / peaks["bf16_tflops_sustained"],
                          "algorithmic_flop_per_launch": flops, "avg_launch_ms": att_avg},
             "kernels": {
-                "pool": {"ms": pool_avg, "GB/s": pool_gbs, "hbm_frac": pool_gbs / peaks["hbm_gbs"],
+                "pool": {"ms": pool_avg, **spread(pool_ms), "GB/s": pool_gbs, "hbm_frac": pool_gbs / peaks["hbm_gbs"],
                          "algorithmic_bytes": pool_bytes},
-                "select": {"ms": sel_avg, "flop": 2.0 * wl.batch * wl.heads * nb * nb * wl.head_dim},
+                "select": {"ms": sel_avg, **spread(sel_ms), "flop": 2.0 * wl.batch * wl.heads * nb * nb * wl.head_dim},
                 "pool_plus_select_effective_GB/s": pool_bytes / ((pool_avg + sel_avg) / 1e3) / 1e9,
-                "attention": {"ms": att_avg, "TFLOP/s": att_tflops},
+                "attention": {"ms": att_avg, **spread(att_ms), "TFLOP/s": att_tflops},
                 "sbsa_forward_ms": forward_ms,
                 **({"rope_pool": {"ms": rope["ms"], "GB/s": rope["algorithmic_bytes"] / (rope["ms"] / 1e3) / 1e9,
                                   "hbm_frac": rope["algorithmic_bytes"] / (rope["ms"] / 1e3) / 1e9 / peaks["hbm_gbs"],
@@ -633,7 +659,7 @@ def run_gpu(args, wl):
                            "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
                            "d2h_bytes_per_step": e2e["d2h_bytes_per_step"], "ms_per_step": e2e["ms"]}
         if ws_n == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_oracle_sample(wl, k, q, kt, v, args.cpu_units)
+            line["cpu_baseline"] = cpu_oracle_sample(wl, k, q, kt, v, args.cpu_units, single_core_units=4)
             line["cpu_baseline"].pop("layer_seconds_extrapolated", None)
         print(json.dumps(line), flush=True)
     if pg is not None:

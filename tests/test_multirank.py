@@ -91,3 +91,16 @@ def test_job_value_counts_every_rank_over_the_slowest():
     assert bench.job_tflops(1e12, 2, 2.0) == pytest.approx(1000.0)
     assert bench.job_tflops(1e12, 1, 2.0) == pytest.approx(500.0)
     assert bench.max_over_ranks(None, "cpu", {"a": 1.5}) == {"a": 1.5}
+
+
+def test_kernel_spread_and_single_core_oracle_sample():
+    import bench
+    from video_dit_dynamic_b200 import inputs
+    assert bench.spread([3.0, 1.0, 2.0, 5.0]) == {"ms_median": 2.5, "ms_best": 1.0}
+    wl = inputs.WORKLOADS["tiny"]
+    k = bench.keep_count(wl.num_blocks, wl.keep)
+    q, kt, v = inputs.make_qkv(wl, seed=0, device="cpu")
+    r = bench.cpu_oracle_sample(wl, k, q, kt, v, n_units=4, single_core_units=2)
+    assert r["kind"] == "oracle" and r["value"] > 0 and r["cores"] >= 1
+    sc = r["single_core"]
+    assert sc["cores"] == 1 and sc["value"] > 0 and "one core" in sc["sample"]
