@@ -509,8 +509,11 @@ constexpr int kF2Half = 128 * 128;                   // 128 rows x 128 bytes of 
 constexpr int kF2SfaBytes = 4 * 512;                 // this CTA's A rows, one K-tile
 constexpr int kF2SfbBytes = 2 * 4 * 512;             // all 256 B rows of the tile, one K-tile
 constexpr int kF2StageBytes = 2 * kF2Half + kF2SfaBytes + kF2SfbBytes;
-constexpr int kF2BiasOff = kF2Stages * kF2StageBytes;  // each epilogue warp's 128 bias values of the tile
-constexpr int kF2BarOff = kF2BiasOff + 8 * 128 * 4;
+// each epilogue warp's 4 KB: the tile's 128 bias values while it converts, then 32 rows x 64
+// columns of bf16 output at a time for the transposed stores
+constexpr int kF2EpiOff = kF2Stages * kF2StageBytes;
+constexpr int kF2EpiBytes = 4096;
+constexpr int kF2BarOff = kF2EpiOff + 8 * kF2EpiBytes;
 // full[S] (leader: both CTAs' codes), sf_in[S] (this CTA's scales landed), sf_full[S]
 // (leader: both CTAs' scales in TMEM), empty[S], acc_full, acc_empty, drain
 constexpr int kF2NumBars = 4 * kF2Stages + 3;
@@ -706,7 +709,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4Threads, 1)
         const uint32_t t_row = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(half * 128);
         const float alpha = __frcp_rn(__fmul_rn(nvfp4_tensor_scale(__ldg(p.amax_a)), nvfp4_tensor_scale(__ldg(p.amax_b))));
         const bool wide = (reinterpret_cast<uintptr_t>(p.c) & 31u) == 0 && p.N % 16 == 0;
-        const uint32_t bias_w = smem_u32(smem + kF2BiasOff) + static_cast<uint32_t>((warp - 2) * 128 * 4);
+        const uint32_t bias_w = smem_u32(smem + kF2EpiOff) + static_cast<uint32_t>((warp - 2) * kF2EpiBytes);
         int tcount = 0;
         for (int tile = pair; tile < num_tiles && !launch_aborted(p.epoch); tile += n_pairs, ++tcount) {
             const int tm = tile / p.tiles_n;
@@ -745,9 +748,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4Threads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) arrive_leader(acc_empty);
-            const long long m = static_cast<long long>(tm) * 256 + static_cast<int>(rank) * 128 + quarter * 32 + lane;
-            if (m < p.M) store_row128(p.c + m * p.N, packed, n0, p.N, wide);
-            __syncwarp();  // every lane has read the bias before the next tile's is written
+            const long long m0 = static_cast<long long>(tm) * 256 + static_cast<int>(rank) * 128 + quarter * 32;
+            if (wide) {
+                // through the warp's buffer, 64 columns at a time: lane r writes row r (16-byte
+                // chunk c at position c ^ (r % 8), so the eight rows of a read hit distinct
+                // banks), then each store instruction writes 128 bytes of each of 8 rows
+                __syncwarp();  // every lane has read the bias
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        st_shared_v4(bias_w + lane * 128 + ((c ^ (lane & 7)) << 4), packed[32 * hh + 4 * c],
+                                     packed[32 * hh + 4 * c + 1], packed[32 * hh + 4 * c + 2], packed[32 * hh + 4 * c + 3]);
+                    __syncwarp();
+                    const int col = n0 + hh * 64 + (lane & 3) * 16;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = i * 8 + (lane >> 2);
+                        const int c0 = (lane & 3) * 2;
+                        uint32_t w[8];
+                        ld_shared_v4(bias_w + r * 128 + ((c0 ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
+                        ld_shared_v4(bias_w + r * 128 + (((c0 + 1) ^ (r & 7)) << 4), w[4], w[5], w[6], w[7]);
+                        if (m0 + r < p.M && col < p.N)
+                            st_global_v8(p.c + (m0 + r) * p.N + col, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+                    }
+                    __syncwarp();  // the buffer is read before it is written again
+                }
+            } else {
+                if (m0 + lane < p.M) store_row128(p.c + (m0 + lane) * p.N, packed, n0, p.N, false);
+                __syncwarp();  // every lane has read the bias before the next tile's is written
+            }
         }
     } else {
         // ------------------------------------------------------------ scales (warps 10-13, both CTAs)
