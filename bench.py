@@ -42,7 +42,7 @@ def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="long122880",
                     help="tiny | 480p | 720p | long122880 | sweep<keep%%> e.g. sweep100")
     ap.add_argument("--impl", default="sbsa", choices=["sbsa", "reference"])

@@ -734,6 +734,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4Threads, 1)
             for (int c = 0; c < 2; ++c) {
                 uint32_t raw[64];
                 tmem_ld64(t_row + c * 64, raw);  // returns after tcgen05.wait::ld
+                if (c == 1) {
+                    // the whole accumulator is in registers: the next tile's MMAs may
+                    // overwrite it while the second half is converted
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) arrive_leader(acc_empty);
+                }
 #pragma unroll
                 for (int e = 0; e < 64; e += 4) {
                     uint32_t b0, b1, b2, b3;
@@ -744,10 +751,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFp4Threads, 1)
                                                              fmaf(__uint_as_float(raw[e + 3]), alpha, __uint_as_float(b3)));
                 }
             }
-            // the accumulator is in registers: the next tile's MMAs may overwrite it
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) arrive_leader(acc_empty);
             const long long m0 = static_cast<long long>(tm) * 256 + static_cast<int>(rank) * 128 + quarter * 32;
             if (wide) {
                 // through the warp's buffer, 64 columns at a time: lane r writes row r (16-byte
