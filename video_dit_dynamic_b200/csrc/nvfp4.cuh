@@ -189,8 +189,7 @@ constexpr uint32_t kFp4SfStageCols = 48;  // A scales (16 columns) then B scales
 constexpr int kFp4NumBars = 3 * kFp4Stages + 3;  // full[S], empty[S], sf_full[S], acc_full, acc_empty, drain
 constexpr int kFp4SmemBytes = kFp4BarOff + kFp4NumBars * 8 + 16 + 1024;  // + tmem slot, flag, alignment slack
 constexpr int kFp4Threads = 448;  // 14 warps: producer, MMA, eight epilogue, four scale warps
-constexpr uint32_t kFp4ColSf = 256;     // two scale regions of 48 columns, by K-tile parity
-constexpr uint32_t kFp4SfRegion = 48;   // A scales at +0 (16 columns), B scales at +16 (32 columns)
+constexpr uint32_t kFp4ColSf = 256;  // scale regions from here, one of kFp4SfStageCols per pipeline stage
 static_assert(kFp4StageBytes % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
 static_assert(kFp4SmemBytes <= 232448, "shared memory");
 
@@ -210,17 +209,6 @@ __device__ __forceinline__ void umma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uin
         : "memory");
 }
 
-
-// Descriptor of a 512-byte scale atom: no swizzle, 8-row x 16-byte core matrices 128
-// bytes apart (both offsets 128: the atom is one core matrix wide).
-__device__ __forceinline__ uint64_t sdesc_atom(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>(128 >> 4) << 16;
-    d |= static_cast<uint64_t>(128 >> 4) << 32;
-    d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm100; layout type 0 = no swizzle
-    return d;
-}
 
 __device__ __forceinline__ uint64_t policy_evict_normal() {
     uint64_t p;
