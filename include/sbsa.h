@@ -224,7 +224,8 @@ sbsa_status sbsa_nvfp4_gemm(int32_t m, int32_t n, int32_t k, const void *a, cons
  * Light-Ulysses 多卡并行; page "单卡 RTX 5090 跑 Wan2.2-A14B：720p 视频生成只要 3.8 秒",
  * 四步拆解 item 4: Ulysses-style sequence parallelism with an FP8 payload, Q, K and V fused
  * into one all-to-all, fused pre/post-processing kernels and a head-level pipeline.
- * These calls are the pre/post-processing; the all-to-all itself is the caller's (NCCL).
+ * These calls are the pre/post-processing around the caller's all-to-all (NCCL), or, with
+ * the peer-put calls below, the exchange itself.
  *
  * `world` ranks; before the attention rank r holds tokens [r L/world, (r+1) L/world), during
  * it heads [r H/world, (r+1) H/world).  A head chunk (head0, head_chunk) selects heads
@@ -263,6 +264,34 @@ sbsa_status sbsa_ulysses_pack_o(const sbsa_ulysses_shape *shape, int32_t head0, 
                                 void *send, void *stream);
 sbsa_status sbsa_ulysses_unpack_o(const sbsa_ulysses_shape *shape, int32_t head0, int32_t head_chunk,
                                   const void *recv, void *y, void *stream);
+
+/* Peer-put exchange: the same slices, written by the packing kernel straight into every
+ * peer's receive buffer (peer-mapped memory over NVLink) instead of a send buffer and a
+ * collective.  Each rank's exchange allocation (the same layout on every rank) holds the
+ * receive buffers and arrays of uint32 flags.
+ *   peer_bases: device array of `world` uint64 base addresses of the ranks' allocations,
+ *     as mapped in this process (peer_bases[rank] is this rank's own); 16-byte aligned.
+ *   recv_offset: byte offset of the receive buffer inside each allocation (multiple of 16).
+ *     Slice `rank` of peer j's receive buffer gets this rank's rows for peer j.
+ * sbsa_ulysses_put_qkv / sbsa_ulysses_put_o: pack as sbsa_ulysses_pack_qkv / _pack_o, the
+ *   slice for peer j written at peer_bases[j] + recv_offset + rank * slice bytes; the
+ *   stores are visible system-wide when the launch ends.
+ * sbsa_peer_signal: flag word `rank` of the uint32 array at flag_offset (a multiple of 4)
+ *   in every peer's allocation := value, a system-scope release ordered after the
+ *   stream's earlier launches.
+ * sbsa_peer_wait: waits on the device until flags[0 .. world) all equal value
+ *   (system-scope acquire), then the stream's later launches run; after timeout_s seconds
+ *   it gives up and latches SBSA_ERR_TIMEOUT for sbsa_check (no fault, no hang).
+ * Values are the caller's (an epoch per exchange and buffer, so no stale flag matches).
+ * The contents of peer_bases cannot be checked on the host: every entry must map a live
+ * allocation of the layout above. */
+sbsa_status sbsa_ulysses_put_qkv(const sbsa_ulysses_shape *shape, int32_t head0, int32_t head_chunk, const void *x,
+                                 const uint64_t *peer_bases, uint64_t recv_offset, int32_t rank, void *stream);
+sbsa_status sbsa_ulysses_put_o(const sbsa_ulysses_shape *shape, int32_t head0, int32_t head_chunk, const void *o,
+                               const uint64_t *peer_bases, uint64_t recv_offset, int32_t rank, void *stream);
+sbsa_status sbsa_peer_signal(const uint64_t *peer_bases, uint64_t flag_offset, int32_t rank, int32_t world,
+                             uint32_t value, void *stream);
+sbsa_status sbsa_peer_wait(const uint32_t *flags, int32_t world, uint32_t value, double timeout_s, void *stream);
 
 /* Steps 1-3 in one call on one stream: pool -> select -> attend, with the means and
  * the CSR lists carved out of `workspace` (device, 256-byte aligned, at least

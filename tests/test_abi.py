@@ -152,3 +152,23 @@ def test_nvfp4_sizes_and_argument_errors():
     assert st == 1 and b"aligned" in lib.sbsa_last_error_message()
     assert lib.sbsa_nvfp4_quantize(fake, 10, 100, fake, fake, fake, None) == 1
     assert lib.sbsa_nvfp4_amax(fake, 10, 12, fake, None) == 1
+
+
+def test_peer_exchange_argument_errors():
+    from video_dit_dynamic_b200 import sbsa
+    lib = sbsa.load()
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: every call below fails its argument checks
+    shape = sbsa.make_ulysses_shape(2, 256, 256, 4, 128)
+    put = lib.sbsa_ulysses_put_qkv
+    assert put(ctypes.byref(shape), 0, 2, None, fake, 0, 0, None) == 1
+    assert put(ctypes.byref(shape), 0, 2, fake, fake, 0, 2, None) == 1 and b"rank" in lib.sbsa_last_error_message()
+    assert put(ctypes.byref(shape), 0, 2, fake, fake, 8, 0, None) == 1  # recv_offset not a multiple of 16
+    assert put(ctypes.byref(shape), 0, 3, fake, fake, 0, 0, None) == 1  # chunk beyond heads / world
+    assert lib.sbsa_ulysses_put_o(ctypes.byref(shape), 0, 2, fake, ctypes.c_void_p((1 << 20) + 4), 0, 0, None) == 1
+    sig = lib.sbsa_peer_signal
+    assert sig(None, 0, 0, 2, 1, None) == 1
+    assert sig(fake, 0, 2, 2, 1, None) == 1 and sig(fake, 0, 0, 0, 1, None) == 1 and sig(fake, 2, 0, 2, 1, None) == 1
+    wait = lib.sbsa_peer_wait
+    assert wait(None, 2, 1, 1.0, None) == 1
+    assert wait(fake, 0, 1, 1.0, None) == 1 and wait(fake, 2, 1, 0.0, None) == 1 and wait(fake, 2, 1, 61.0, None) == 1
+    assert wait(ctypes.c_void_p((1 << 20) + 2), 2, 1, 1.0, None) == 1

@@ -111,3 +111,61 @@ def test_light_ulysses_single_rank_end_to_end():
     row_max = np.abs(yr).max(axis=2, keepdims=True)
     assert np.all(np.abs(yg - yr) <= 2e-2 + row_max * 2.0 ** -3)
     assert np.mean(np.abs(yg - yr)) < 2e-3
+
+
+@pytest.mark.parametrize("G,L,H,Lp,hc", [(2, 256, 4, 256, 1), (4, 400, 8, 512, 1), (2, 250, 6, 256, 2)])
+def test_peer_put_exchange_emulated_ranks(G, L, H, Lp, hc):
+    """The peer-put exchange with G ranks emulated on one GPU (their allocations are local
+    buffers, every rank's step runs before the next step): q, k, v bit-exact with the
+    oracle's exchange, the layer within the attention tolerance of the oracle's, and a
+    second call (buffers reused, acknowledgements awaited) identical to the first."""
+    from video_dit_dynamic_b200 import ulysses
+    sbsa = _sbsa()
+    d = 128
+    plan = ulysses.UlyssesPlan(world=G, tokens=L, tokens_padded=Lp, heads=H, head_dim=d, head_chunk=hc)
+    exs = ulysses.PeerExchange.emulated(plan, "cuda", timeout_s=5.0)
+    layers = [ulysses.LightUlysses(plan, keep=1.0, exchange=exs[r]) for r in range(G)]
+    shards = _shards(G, L, H, d, seed=G * 7 + L)
+    xs = [s.cuda() for s in shards]
+    ys = [y.clone() for y in ulysses.lockstep_forward(layers, xs)]
+    sbsa.sbsa_check()
+    ref = oracle.ulysses_qkv([inputs.bf16_bits(s) for s in shards], H, L, Lp)
+    for r in range(G):
+        for c, t in enumerate((layers[r].q, layers[r].k, layers[r].v)):
+            np.testing.assert_array_equal(inputs.bf16_bits(t.cpu()), ref[r][c])
+    ys2 = ulysses.lockstep_forward(layers, xs)
+    sbsa.sbsa_check()
+    for r in range(G):
+        assert torch.equal(ys[r], ys2[r])
+    # the oracle's layer: exchange -> dense attention (keep = 1) per rank -> bf16 -> return
+    nb = Lp // 128
+    Hg = H // G
+    rp = oracle.uniform_row_ptr(1, Hg, nb, nb)
+    col = np.broadcast_to(np.arange(nb, dtype=np.int32), (1, Hg, nb, nb)).copy()
+    os_ = [oracle.bf16_round(oracle.attention(ref[r][0][None], ref[r][1][None], ref[r][2][None], L, 128, rp, col)[0])
+           for r in range(G)]
+    y_ref = oracle.ulysses_o(os_, H, L)
+    for r in range(G):
+        yr = (y_ref[r].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        yg = ys[r].float().cpu().double().numpy()
+        row_max = np.abs(yr).max(axis=2, keepdims=True)
+        assert np.all(np.abs(yg - yr) <= 2e-2 + row_max * 2.0 ** -3)
+        assert np.mean(np.abs(yg - yr)) < 2e-3
+
+
+def test_peer_wait_gives_up_without_a_fault():
+    """A wait on a flag nothing sets ends after its limit with SBSA_ERR_TIMEOUT from
+    sbsa_check; the context stays usable."""
+    sbsa = _sbsa()
+    flags = torch.zeros(4, dtype=torch.int32, device="cuda")
+    sbsa.sbsa_peer_wait(flags, 4, 12345, timeout_s=0.05)
+    with pytest.raises(sbsa.SbsaError) as err:
+        sbsa.sbsa_check()
+    assert err.value.status == 5  # SBSA_ERR_TIMEOUT
+    # flags that are set end the wait at once, and the next launches run normally
+    bases = torch.tensor([flags.data_ptr()] * 4, dtype=torch.int64, device="cuda")  # four "peers", one array
+    for i in range(4):
+        sbsa.sbsa_peer_signal(bases, 0, i, 4, 777)
+    sbsa.sbsa_peer_wait(flags, 4, 777, timeout_s=5.0)
+    sbsa.sbsa_check()
+    assert torch.all(flags == 777)

@@ -663,6 +663,66 @@ sbsa_status sbsa_ulysses_unpack_o(const sbsa_ulysses_shape* shape, int32_t head0
     return e == cudaSuccess ? ok() : cuda_fail(e, "ulysses unpack_o launch");
 }
 
+sbsa_status sbsa_ulysses_put_qkv(const sbsa_ulysses_shape* shape, int32_t head0, int32_t head_chunk, const void* x,
+                                 const uint64_t* peer_bases, uint64_t recv_offset, int32_t rank, void* stream) {
+    UlyssesDims u;
+    sbsa_status r = ulysses_dims(shape, head0, head_chunk, &u);
+    if (r != SBSA_OK) return r;
+    if (!x || !peer_bases) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(x) || (reinterpret_cast<uintptr_t>(peer_bases) & 7u) || (recv_offset & 15u))
+        return fail(SBSA_ERR_INVALID_ARG, "x 16-byte aligned, peer_bases 8-byte aligned, recv_offset a multiple of 16");
+    if (rank < 0 || rank >= u.G) return fail(SBSA_ERR_INVALID_ARG, "rank outside [0, world)");
+    const PeerDst pd{reinterpret_cast<const unsigned long long*>(peer_bases), recv_offset, rank};
+    const long long rows = static_cast<long long>(u.G) * u.Lr * 3 * u.hc;
+    const long long grid = (rows + kUlyRowsPerCta - 1) / kUlyRowsPerCta;
+    ulysses_put_qkv_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16*>(x), pd, u);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "ulysses put_qkv launch");
+}
+
+sbsa_status sbsa_ulysses_put_o(const sbsa_ulysses_shape* shape, int32_t head0, int32_t head_chunk, const void* o,
+                               const uint64_t* peer_bases, uint64_t recv_offset, int32_t rank, void* stream) {
+    UlyssesDims u;
+    sbsa_status r = ulysses_dims(shape, head0, head_chunk, &u);
+    if (r != SBSA_OK) return r;
+    if (!o || !peer_bases) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(o) || (reinterpret_cast<uintptr_t>(peer_bases) & 7u) || (recv_offset & 15u))
+        return fail(SBSA_ERR_INVALID_ARG, "o 16-byte aligned, peer_bases 8-byte aligned, recv_offset a multiple of 16");
+    if (rank < 0 || rank >= u.G) return fail(SBSA_ERR_INVALID_ARG, "rank outside [0, world)");
+    const PeerDst pd{reinterpret_cast<const unsigned long long*>(peer_bases), recv_offset, rank};
+    const long long rows = static_cast<long long>(u.G) * u.Lr * u.hc;
+    const long long grid = (rows + kUlyRowsPerCta - 1) / kUlyRowsPerCta;
+    ulysses_put_o_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16*>(o), pd, u);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "ulysses put_o launch");
+}
+
+sbsa_status sbsa_peer_signal(const uint64_t* peer_bases, uint64_t flag_offset, int32_t rank, int32_t world,
+                             uint32_t value, void* stream) {
+    if (!peer_bases) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (world < 1 || world > 1024 || rank < 0 || rank >= world)
+        return fail(SBSA_ERR_INVALID_ARG, "world in [1, 1024] and rank in [0, world) required");
+    if ((reinterpret_cast<uintptr_t>(peer_bases) & 7u) || (flag_offset & 3u))
+        return fail(SBSA_ERR_INVALID_ARG, "peer_bases 8-byte aligned, flag_offset a multiple of 4");
+    peer_signal_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const unsigned long long*>(peer_bases), flag_offset, rank, world, value);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "peer signal launch");
+}
+
+sbsa_status sbsa_peer_wait(const uint32_t* flags, int32_t world, uint32_t value, double timeout_s, void* stream) {
+    if (!flags) return fail(SBSA_ERR_INVALID_ARG, "null pointer");
+    if (world < 1 || world > 1024) return fail(SBSA_ERR_INVALID_ARG, "world in [1, 1024] required");
+    if (reinterpret_cast<uintptr_t>(flags) & 3u) return fail(SBSA_ERR_INVALID_ARG, "flags must be 4-byte aligned");
+    if (!(timeout_s > 0.0) || timeout_s > 60.0) return fail(SBSA_ERR_INVALID_ARG, "timeout_s in (0, 60] required");
+    const unsigned long long limit = static_cast<unsigned long long>(timeout_s * 1e9);
+    peer_wait_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(flags, world, value, limit);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "peer wait launch");
+}
+
 size_t sbsa_nvfp4_scale_bytes(int64_t rows, int32_t cols) {
     if (rows < 1 || cols < 64 || cols % 64) return 0;
     return static_cast<size_t>((rows + 127) / 128 * 128) * static_cast<size_t>(cols / 16);

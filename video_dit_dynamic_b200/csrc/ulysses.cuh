@@ -15,6 +15,11 @@
 // codes followed by its scales and padded to a multiple of 16 bytes:
 //   QKV slice for peer j: codes [L/G][3][hc][d], scales [L/G][3][hc]
 //   O   slice for peer j: codes [L/G][hc][d],    scales [L/G][hc]
+// Two exchanges are supported: the caller's all-to-all of the send buffers (NCCL), or
+// peer puts, where each rank's kernel writes every peer's slice straight into that peer's
+// receive buffer (peer-mapped memory over NVLink) and then raises a flag in each peer
+// (system-scope release); the receiver waits on its flags (system-scope acquire, bounded)
+// before it unpacks.  The receive layout is the same in both.
 // Layouts around them:
 //   x  (fused QKV activation of this rank's tokens)  [L/G][3][H][d] bf16
 //   q, k, v (this rank's heads, attention layout)    [H/G][Lp][d] bf16, tokens >= L zero
@@ -107,6 +112,43 @@ __device__ __forceinline__ RowPtrs o_pack_row(uint32_t w, const __nv_bfloat16* o
     const uint32_t hh = row - t * static_cast<uint32_t>(u.hc);
     const size_t token = static_cast<size_t>(j) * u.Lr + t;
     uint8_t* slice = send + static_cast<size_t>(j) * ulysses_o_slice_bytes(u);
+    return {reinterpret_cast<const uint4*>(o + (static_cast<size_t>(u.h0 + hh) * u.Lp + token) * kUlyD),
+            slice + static_cast<size_t>(row) * kUlyD,
+            reinterpret_cast<float*>(slice + static_cast<size_t>(per_peer) * kUlyD) + row, false};
+}
+
+// Peer puts: slice j of this rank goes to peer j's receive buffer, at offset
+// recv_offset + rank * slice bytes of peer j's exchange allocation.
+struct PeerDst {
+    const unsigned long long* bases;  // device array of the world's allocation base addresses
+    unsigned long long recv_offset;   // byte offset of the receive buffer in each allocation
+    int rank;
+};
+
+__device__ __forceinline__ RowPtrs qkv_put_row(uint32_t w, const __nv_bfloat16* x, const PeerDst& pd,
+                                               const UlyssesDims& u) {
+    const uint32_t per_peer = static_cast<uint32_t>(u.Lr) * 3u * static_cast<uint32_t>(u.hc);
+    const uint32_t j = udiv(w, u.by_qkv_peer);
+    const uint32_t row = w - j * per_peer;  // (t * 3 + c) * hc + hh
+    const uint32_t tc = udiv(row, u.by_hc);
+    const uint32_t hh = row - tc * static_cast<uint32_t>(u.hc);
+    uint8_t* slice = reinterpret_cast<uint8_t*>(__ldg(pd.bases + j) + pd.recv_offset) +
+                     static_cast<size_t>(pd.rank) * ulysses_qkv_slice_bytes(u);
+    const size_t src = (static_cast<size_t>(tc) * u.H + j * u.Hg + u.h0 + hh) * kUlyD;
+    return {reinterpret_cast<const uint4*>(x + src), slice + static_cast<size_t>(row) * kUlyD,
+            reinterpret_cast<float*>(slice + static_cast<size_t>(per_peer) * kUlyD) + row, false};
+}
+
+__device__ __forceinline__ RowPtrs o_put_row(uint32_t w, const __nv_bfloat16* o, const PeerDst& pd,
+                                             const UlyssesDims& u) {
+    const uint32_t per_peer = static_cast<uint32_t>(u.Lr) * static_cast<uint32_t>(u.hc);
+    const uint32_t j = udiv(w, u.by_o_peer);
+    const uint32_t row = w - j * per_peer;  // t * hc + hh
+    const uint32_t t = udiv(row, u.by_hc);
+    const uint32_t hh = row - t * static_cast<uint32_t>(u.hc);
+    const size_t token = static_cast<size_t>(j) * u.Lr + t;
+    uint8_t* slice = reinterpret_cast<uint8_t*>(__ldg(pd.bases + j) + pd.recv_offset) +
+                     static_cast<size_t>(pd.rank) * ulysses_o_slice_bytes(u);
     return {reinterpret_cast<const uint4*>(o + (static_cast<size_t>(u.h0 + hh) * u.Lp + token) * kUlyD),
             slice + static_cast<size_t>(row) * kUlyD,
             reinterpret_cast<float*>(slice + static_cast<size_t>(per_peer) * kUlyD) + row, false};
@@ -280,6 +322,54 @@ __global__ void __launch_bounds__(256) ulysses_unpack_o_kernel(const uint8_t* __
     const uint32_t first = blockIdx.x * kUlyRowsPerCta + (threadIdx.x / 32) * kUlyRowsPerWarp;
     const uint32_t n_rows = static_cast<uint32_t>(u.G) * u.Lr * u.hc;
     unpack_rows(first, n_rows, [&](uint32_t w) { return o_unpack_row(w, recv, y, u); });
+}
+
+// x -> every peer's receive buffer (peer puts); each thread's remote stores are made
+// visible system-wide before its CTA ends, so a later signal launch may publish them.
+__global__ void __launch_bounds__(256) ulysses_put_qkv_kernel(const __nv_bfloat16* __restrict__ x, PeerDst pd,
+                                                              UlyssesDims u) {
+    const uint32_t first = blockIdx.x * kUlyRowsPerCta + (threadIdx.x / 32) * kUlyRowsPerWarp;
+    const uint32_t n_rows = static_cast<uint32_t>(u.G) * u.Lr * 3u * u.hc;
+    pack_rows(first, n_rows, [&](uint32_t w) { return qkv_put_row(w, x, pd, u); });
+    __threadfence_system();
+}
+
+__global__ void __launch_bounds__(256) ulysses_put_o_kernel(const __nv_bfloat16* __restrict__ o, PeerDst pd,
+                                                            UlyssesDims u) {
+    const uint32_t first = blockIdx.x * kUlyRowsPerCta + (threadIdx.x / 32) * kUlyRowsPerWarp;
+    const uint32_t n_rows = static_cast<uint32_t>(u.G) * u.Lr * u.hc;
+    pack_rows(first, n_rows, [&](uint32_t w) { return o_put_row(w, o, pd, u); });
+    __threadfence_system();
+}
+
+// Flag word `rank` of the flag array at flag_offset in every peer's allocation := value
+// (system-scope release, after this thread's earlier writes and the previous launches'
+// on the stream).
+__global__ void peer_signal_kernel(const unsigned long long* __restrict__ bases, unsigned long long flag_offset,
+                                   int rank, int world, uint32_t value) {
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= world) return;
+    uint32_t* f = reinterpret_cast<uint32_t*>(__ldg(bases + j) + flag_offset) + rank;
+    asm volatile("fence.sc.sys;" ::: "memory");
+    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(f), "r"(value) : "memory");
+}
+
+// Wait until flags[0 .. world) all equal value (system-scope acquire), at most limit_ns;
+// on running out the launch latches SBSA_ERR_TIMEOUT and returns.
+__global__ void peer_wait_kernel(const uint32_t* flags, int world, uint32_t value, unsigned long long limit_ns) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= world) return;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        uint32_t v;
+        asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(flags + i) : "memory");
+        if (v == value) return;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            raise_error(kErrTimeout);
+            return;
+        }
+        __nanosleep(256);
+    }
 }
 
 }  // namespace sbsa

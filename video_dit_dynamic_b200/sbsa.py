@@ -27,7 +27,8 @@ EXPORTS = ("sbsa_version", "sbsa_status_string", "sbsa_last_error_message", "sbs
            "sbsa_rope_table_init", "sbsa_rope_pool_qk", "sbsa_key_mean", "sbsa_quantize_qk_fp8",
            "sbsa_attention_fwd_fp8", "sbsa_nvfp4_scale_bytes", "sbsa_nvfp4_amax", "sbsa_nvfp4_quantize",
            "sbsa_nvfp4_gemm", "sbsa_ulysses_qkv_bytes", "sbsa_ulysses_o_bytes", "sbsa_ulysses_pack_qkv",
-           "sbsa_ulysses_unpack_qkv", "sbsa_ulysses_pack_o", "sbsa_ulysses_unpack_o")
+           "sbsa_ulysses_unpack_qkv", "sbsa_ulysses_pack_o", "sbsa_ulysses_unpack_o", "sbsa_ulysses_put_qkv",
+           "sbsa_ulysses_put_o", "sbsa_peer_signal", "sbsa_peer_wait")
 
 
 class SbsaError(RuntimeError):
@@ -114,7 +115,13 @@ def load(path: str | None = None):
     lib.sbsa_ulysses_unpack_qkv.argtypes = [UP, I32, I32, P, P, P, P, P]
     lib.sbsa_ulysses_pack_o.argtypes = [UP, I32, I32, P, P, P]
     lib.sbsa_ulysses_unpack_o.argtypes = [UP, I32, I32, P, P, P]
-    for name in ("sbsa_ulysses_pack_qkv", "sbsa_ulysses_unpack_qkv", "sbsa_ulysses_pack_o", "sbsa_ulysses_unpack_o"):
+    U64 = ctypes.c_uint64
+    lib.sbsa_ulysses_put_qkv.argtypes = [UP, I32, I32, P, P, U64, I32, P]
+    lib.sbsa_ulysses_put_o.argtypes = [UP, I32, I32, P, P, U64, I32, P]
+    lib.sbsa_peer_signal.argtypes = [P, U64, I32, I32, ctypes.c_uint32, P]
+    lib.sbsa_peer_wait.argtypes = [P, I32, ctypes.c_uint32, ctypes.c_double, P]
+    for name in ("sbsa_ulysses_pack_qkv", "sbsa_ulysses_unpack_qkv", "sbsa_ulysses_pack_o", "sbsa_ulysses_unpack_o",
+                 "sbsa_ulysses_put_qkv", "sbsa_ulysses_put_o", "sbsa_peer_signal", "sbsa_peer_wait"):
         getattr(lib, name).restype = ctypes.c_int
     for name in ("sbsa_pool_qk", "sbsa_select_blocks", "sbsa_attention_fwd", "sbsa_forward", "sbsa_check",
                  "sbsa_validate_csr", "sbsa_forward_noalloc", "sbsa_rope_table_init", "sbsa_rope_pool_qk",
@@ -295,6 +302,42 @@ def sbsa_ulysses_unpack_o(shape: UlyssesShape, head0: int, head_chunk: int, recv
     _check_numel(y, lr * shape.heads * shape.head_dim, "y")
     _raise_on(load().sbsa_ulysses_unpack_o(ctypes.byref(shape), head0, head_chunk, _dev(recv, torch.uint8, "recv"),
                                            _dev(y, torch.bfloat16, "y"), _stream(stream)))
+
+
+def sbsa_ulysses_put_qkv(shape: UlyssesShape, head0: int, head_chunk: int, x, peer_bases, recv_offset: int,
+                         rank: int, stream=None):
+    """Pack x and write slice j into rank j's receive buffer at peer_bases[j] + recv_offset
+    (peer_bases: int64 CUDA tensor of the world's allocation base addresses)."""
+    lr, _ = _uly_sizes(shape)
+    _check_numel(x, lr * 3 * shape.heads * shape.head_dim, "x")
+    _check_numel(peer_bases, shape.world, "peer_bases")
+    _raise_on(load().sbsa_ulysses_put_qkv(ctypes.byref(shape), head0, head_chunk, _dev(x, torch.bfloat16, "x"),
+                                          _dev(peer_bases, torch.int64, "peer_bases"), recv_offset, rank,
+                                          _stream(stream)))
+
+
+def sbsa_ulysses_put_o(shape: UlyssesShape, head0: int, head_chunk: int, o, peer_bases, recv_offset: int, rank: int,
+                       stream=None):
+    _, hg = _uly_sizes(shape)
+    _check_numel(o, hg * shape.tokens_padded * shape.head_dim, "o")
+    _check_numel(peer_bases, shape.world, "peer_bases")
+    _raise_on(load().sbsa_ulysses_put_o(ctypes.byref(shape), head0, head_chunk, _dev(o, torch.bfloat16, "o"),
+                                        _dev(peer_bases, torch.int64, "peer_bases"), recv_offset, rank,
+                                        _stream(stream)))
+
+
+def sbsa_peer_signal(peer_bases, flag_offset: int, rank: int, world: int, value: int, stream=None):
+    _check_numel(peer_bases, world, "peer_bases")
+    _raise_on(load().sbsa_peer_signal(_dev(peer_bases, torch.int64, "peer_bases"), flag_offset, rank, world,
+                                      value & 0xFFFFFFFF, _stream(stream)))
+
+
+def sbsa_peer_wait(flags, world: int, value: int, timeout_s: float = 10.0, stream=None):
+    """Device-side wait until the `world` uint32 words at `flags` (an int32 CUDA tensor or a
+    view of one) all equal `value`; a wait that runs out latches SBSA_ERR_TIMEOUT."""
+    _check_numel(flags, world, "flags")
+    _raise_on(load().sbsa_peer_wait(_dev(flags, torch.int32, "flags"), world, value & 0xFFFFFFFF, timeout_s,
+                                    _stream(stream)))
 
 
 def sbsa_nvfp4_scale_bytes(rows: int, cols: int) -> int:
