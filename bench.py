@@ -545,6 +545,8 @@ def run_gpu(args, wl):
         uq, uk, uv = (torch.empty_like(q) for _ in range(3))
         uy = torch.empty(wl.seq_len, wl.heads, wl.head_dim, dtype=torch.bfloat16, device=dev)
         osend = torch.empty(ob, dtype=torch.uint8, device=dev)
+        ubase = torch.tensor([usend.data_ptr()], dtype=torch.int64, device=dev)
+        obase = torch.tensor([osend.data_ptr()], dtype=torch.int64, device=dev)
         calls = [
             ("pack_qkv", lambda: sbsa.sbsa_ulysses_pack_qkv(ushape, 0, wl.heads, xq, usend, stream=stream),
              xq.numel() * 2 + ub),
@@ -554,6 +556,11 @@ def run_gpu(args, wl):
              uy.numel() * 2 + ob),
             ("unpack_o", lambda: sbsa.sbsa_ulysses_unpack_o(ushape, 0, wl.heads, osend, uy, stream=stream),
              ob + uy.numel() * 2),
+            # the peer-put packs, world 1: the "peer" receive buffer is this GPU's own
+            ("put_qkv", lambda: sbsa.sbsa_ulysses_put_qkv(ushape, 0, wl.heads, xq, ubase, 0, 0, stream=stream),
+             xq.numel() * 2 + ub),
+            ("put_o", lambda: sbsa.sbsa_ulysses_put_o(ushape, 0, wl.heads, uq, obase, 0, 0, stream=stream),
+             uy.numel() * 2 + ob),
         ]
         uly = {}
         for uname, ucall, nbytes in calls:
@@ -567,7 +574,7 @@ def run_gpu(args, wl):
             torch.cuda.synchronize(dev)
             uly[uname] = {"ms": u0.elapsed_time(u1) / 5, "algorithmic_bytes": nbytes}
         sbsa.sbsa_check(stream)
-        del xq, usend, uq, uk, uv, uy, osend
+        del xq, usend, uq, uk, uv, uy, osend, ubase, obase
 
     # end to end through the public API from pinned host buffers
     e2e = None
