@@ -674,7 +674,8 @@ sbsa_status sbsa_ulysses_put_qkv(const sbsa_ulysses_shape* shape, int32_t head0,
     if (rank < 0 || rank >= u.G) return fail(SBSA_ERR_INVALID_ARG, "rank outside [0, world)");
     const PeerDst pd{reinterpret_cast<const unsigned long long*>(peer_bases), recv_offset, rank};
     const long long rows = static_cast<long long>(u.G) * u.Lr * 3 * u.hc;
-    const long long grid = (rows + kUlyRowsPerCta - 1) / kUlyRowsPerCta;
+    const long long tiles = (rows + kUlyRowsPerCta - 1) / kUlyRowsPerCta;
+    const long long grid = tiles < 8LL * sm_count() ? tiles : 8LL * sm_count();  // one fence per CTA: few CTAs
     ulysses_put_qkv_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const __nv_bfloat16*>(x), pd, u);
     cudaError_t e = cudaGetLastError();
@@ -692,7 +693,8 @@ sbsa_status sbsa_ulysses_put_o(const sbsa_ulysses_shape* shape, int32_t head0, i
     if (rank < 0 || rank >= u.G) return fail(SBSA_ERR_INVALID_ARG, "rank outside [0, world)");
     const PeerDst pd{reinterpret_cast<const unsigned long long*>(peer_bases), recv_offset, rank};
     const long long rows = static_cast<long long>(u.G) * u.Lr * u.hc;
-    const long long grid = (rows + kUlyRowsPerCta - 1) / kUlyRowsPerCta;
+    const long long tiles = (rows + kUlyRowsPerCta - 1) / kUlyRowsPerCta;
+    const long long grid = tiles < 8LL * sm_count() ? tiles : 8LL * sm_count();  // one fence per CTA: few CTAs
     ulysses_put_o_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const __nv_bfloat16*>(o), pd, u);
     cudaError_t e = cudaGetLastError();
