@@ -65,7 +65,8 @@ class FakeDevice:
             assert self.slots[(rank, exchange, buf, writer)] == (want, head0, n)
 
 
-@pytest.mark.parametrize("world,heads,head_chunk,calls", [(2, 4, 1, 2), (4, 8, 1, 1), (2, 6, 2, 3), (3, 3, 1, 2)])
+@pytest.mark.parametrize("world,heads,head_chunk,calls", [(2, 4, 1, 2), (4, 8, 1, 1), (2, 6, 2, 3), (3, 3, 1, 2),
+                                                             (2, 12, 1, 2), (3, 12, 1, 1)])
 def test_lockstep_schedule_satisfies_every_wait_and_never_overwrites_unread_data(monkeypatch, world, heads,
                                                                                    head_chunk, calls):
     tokens = 8 * world
