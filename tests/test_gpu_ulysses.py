@@ -113,7 +113,8 @@ def test_light_ulysses_single_rank_end_to_end():
     assert np.mean(np.abs(yg - yr)) < 2e-3
 
 
-@pytest.mark.parametrize("G,L,H,Lp,hc", [(2, 256, 4, 256, 1), (4, 400, 8, 512, 1), (2, 250, 6, 256, 2)])
+@pytest.mark.parametrize("G,L,H,Lp,hc", [(2, 256, 4, 256, 1), (4, 400, 8, 512, 1), (2, 250, 6, 256, 2),
+                                         (2, 256, 8, 256, 1)])  # 4 chunks: buffers reused within a call
 def test_peer_put_exchange_emulated_ranks(G, L, H, Lp, hc):
     """The peer-put exchange with G ranks emulated on one GPU (their allocations are local
     buffers, every rank's step runs before the next step): q, k, v bit-exact with the
