@@ -135,3 +135,30 @@ def test_steps_cover_every_chunk_in_order():
         assert pos[("send_qkv", c)] < pos[("recv_qkv", c)] < pos[("attend", c)] < pos[("send_o", c)] < pos[("recv_o", c)]
         if c + 1 < n:
             assert pos[("send_qkv", c + 1)] < pos[("attend", c)]  # the next exchange overlaps this attention
+
+
+def test_layers_sharing_an_exchange_get_distinct_epochs(monkeypatch):
+    """Two layers over one allocation: the second layer's chunks must not match the first
+    layer's flags (the call counter lives in the exchange)."""
+    plan = ulysses.UlyssesPlan(1, 8, 8, 2, 128, 1)
+    size = ulysses.PeerExchange.layout(plan)["total"]
+    ex = ulysses.PeerExchange(plan, torch.zeros(size, dtype=torch.uint8), torch.zeros(1, dtype=torch.int64), 0)
+    seen = []
+    monkeypatch.setattr(ulysses.PeerExchange, "send", lambda self, e, c, h0, n, src, epoch: seen.append((e, epoch)))
+    monkeypatch.setattr(ulysses.PeerExchange, "recv", lambda self, e, c, h0, n, dst, epoch: None)
+
+    class Ops:
+        def attend(self, *a):
+            pass
+
+    a = ulysses.LightUlysses(plan, device="cpu", ops=Ops(), exchange=ex)
+    b = ulysses.LightUlysses(plan, device="cpu", ops=Ops(), exchange=ex)
+    x = torch.zeros(8, 3, 2, 128, dtype=torch.bfloat16)
+    a.forward(x)
+    b.forward(x)
+    a.forward(x)
+    # the two exchanges keep separate flags; within each, every epoch is new
+    assert len(seen) == len(set(seen)) == 3 * 2 * 2  # 3 calls x 2 chunks x (qkv, o)
+    other = ulysses.UlyssesPlan(1, 8, 8, 2, 128, 2)
+    with pytest.raises(ValueError):
+        ulysses.LightUlysses(other, device="cpu", ops=Ops(), exchange=ex)

@@ -106,6 +106,13 @@ class PeerExchange:
         self.qkv_off, self.o_off, self.flag_off = lay["qkv"], lay["o"], lay["flags"]
         self.full = sbsa.make_ulysses_shape(plan.world, plan.tokens, plan.tokens_padded, plan.heads, plan.head_dim)
         self.last_epoch = {}  # (exchange, buffer) -> epoch of the buffer's last write
+        self.calls = 0        # forwards through this allocation, by every layer that uses it
+
+    def new_call(self) -> int:
+        """The number of the next forward through this allocation: epochs stay distinct when
+        several layers share it (every rank counts the same calls in the same order)."""
+        self.calls += 1
+        return self.calls
 
     @staticmethod
     def layout(plan: UlyssesPlan) -> dict:
@@ -159,6 +166,9 @@ class PeerExchange:
         """The allocation in torch's symmetric memory (peer-mapped over NVLink), one per rank
         of `group`; collective: every rank of the group calls it."""
         import torch.distributed._symmetric_memory as symm_mem
+        group = group if group is not None else dist.group.WORLD
+        if hasattr(symm_mem, "enable_symm_mem_for_group"):
+            symm_mem.enable_symm_mem_for_group(group.group_name)
         local = symm_mem.empty(cls.layout(plan)["total"], dtype=torch.uint8, device=device)
         local.zero_()
         handle = symm_mem.rendezvous(local, group)
@@ -224,6 +234,8 @@ class LightUlysses:
         self.group = group
         self.peer = exchange
         self._call = 0
+        if exchange is not None and exchange.plan != plan:
+            raise ValueError("the exchange was laid out for another plan")
         if exchange is None:
             if group is not None and dist.get_world_size(group) != plan.world:
                 raise ValueError("plan.world differs from the group's size")
@@ -269,7 +281,7 @@ class LightUlysses:
         if y is None:
             y = torch.empty((p.tokens_local, p.heads, p.head_dim), dtype=x.dtype, device=x.device)
         self._x, self._y = x, y
-        self._call += 1
+        self._call = self.peer.new_call() if self.peer is not None else self._call + 1
         self._pending = {}
         return y
 
