@@ -12,7 +12,6 @@ import os
 
 import torch
 
-from . import build as _build
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
