@@ -3,7 +3,9 @@
 Each case below plants one mistake in a copy of oracle/sbsa_oracle.c (a text edit,
 compiled with gcc into a temporary library, on the CPU), swaps it in for the real
 oracle, and runs every pin in test_oracle_pins.py.  At least one pin must fail for
-each mutant; the real oracle passes them all.
+each mutant; the real oracle passes them all.  The Python-side oracle functions (the
+Light-Ulysses exchanges) get the same treatment: a mutated copy of one function is
+swapped in for the pins' run.
 """
 import ctypes
 import inspect
@@ -73,6 +75,30 @@ MUTANTS = {
 }
 
 
+# Python-side oracle functions: (function, old text, new text)
+PY_MUTANTS = {
+    # the receiver takes the sender's heads instead of its own
+    "uly_qkv_wrong_heads": ("ulysses_qkv", "x_shards[i][:, :, r * Hg:(r + 1) * Hg, :]",
+                            "x_shards[i][:, :, i * Hg:(i + 1) * Hg, :]"),
+    # each sender's tokens land in the receiver's own token range
+    "uly_qkv_wrong_tokens": ("ulysses_qkv", "dst[:, :, i * Lr:(i + 1) * Lr, :]", "dst[:, :, r * Lr:(r + 1) * Lr, :]"),
+    # q, k, v and heads transposed in the attention layout
+    "uly_qkv_transposed": ("ulysses_qkv", "deq.transpose(1, 2, 0, 3)", "deq.transpose(2, 1, 0, 3)"),
+    # the return exchange puts every sender's heads at the receiver's own head range
+    "uly_o_wrong_heads": ("ulysses_o", "dst[:, i * Hg:(i + 1) * Hg, :] = deq", "dst[:, r * Hg:(r + 1) * Hg, :] = deq"),
+    # the return exchange takes the sender's token range instead of the receiver's
+    "uly_o_wrong_tokens": ("ulysses_o", "o_shards[i][:, r * Lr:(r + 1) * Lr, :]", "o_shards[i][:, i * Lr:(i + 1) * Lr, :]"),
+}
+
+
+def _py_mutant(func_name, old, new):
+    src = inspect.getsource(getattr(oracle, func_name))
+    assert src.count(old) == 1, f"mutation anchor for {func_name} not unique/present"
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), f"<mutant {func_name}>", "exec"), ns)
+    return ns[func_name]
+
+
 def _build_mutant(tmp_path, name, old, new):
     text = open(SRC).read()
     assert text.count(old) == 1, f"mutation anchor for {name} not unique/present"
@@ -123,6 +149,14 @@ def test_pins_catch_mutant(tmp_path, name):
     old, new = MUTANTS[name]
     so = _build_mutant(tmp_path, name, old, new)
     failed = _run_pins_with(so)
+    assert failed, f"mutant {name} passed every pin"
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_pins_catch_python_mutant(monkeypatch, name):
+    func_name, old, new = PY_MUTANTS[name]
+    monkeypatch.setattr(oracle, func_name, _py_mutant(func_name, old, new))
+    failed = _run_pins_with(oracle.build())
     assert failed, f"mutant {name} passed every pin"
 
 
