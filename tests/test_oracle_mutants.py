@@ -88,6 +88,13 @@ PY_MUTANTS = {
     "uly_o_wrong_heads": ("ulysses_o", "dst[:, i * Hg:(i + 1) * Hg, :] = deq", "dst[:, r * Hg:(r + 1) * Hg, :] = deq"),
     # the return exchange takes the sender's token range instead of the receiver's
     "uly_o_wrong_tokens": ("ulysses_o", "o_shards[i][:, r * Lr:(r + 1) * Lr, :]", "o_shards[i][:, i * Lr:(i + 1) * Lr, :]"),
+    # the NVFP4 GEMM without its bias, or against B untransposed
+    "fp4_gemm_no_bias": ("nvfp4_gemm", "        c = c + np.asarray(bias, dtype=np.float64)[None, :]", "        c = c"),
+    "fp4_gemm_bias_per_row": ("nvfp4_gemm", "np.asarray(bias, dtype=np.float64)[None, :]",
+                              "np.asarray(bias, dtype=np.float64)[:c.shape[0], None]"),
+    # the FP8 attention path with K taken from Q's codes
+    "fp8_attention_k_from_q": ("attention_fp8", "kd = dequantize_fp8(k_codes, k_scales, blk)",
+                               "kd = dequantize_fp8(q_codes, q_scales, blk)"),
 }
 
 
