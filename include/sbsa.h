@@ -281,7 +281,8 @@ sbsa_status sbsa_ulysses_unpack_o(const sbsa_ulysses_shape *shape, int32_t head0
  *   stream's earlier launches.
  * sbsa_peer_wait: waits on the device until flags[0 .. world) all equal value
  *   (system-scope acquire), then the stream's later launches run; after timeout_s seconds
- *   it gives up and latches SBSA_ERR_TIMEOUT for sbsa_check (no fault, no hang).
+ *   (0 < timeout_s <= 60) it gives up and latches SBSA_ERR_TIMEOUT for sbsa_check (no
+ *   fault, no hang).  world is at most 1024 here and in sbsa_peer_signal.
  * Values are the caller's (an epoch per exchange and buffer, so no stale flag matches).
  * The contents of peer_bases cannot be checked on the host: every entry must map a live
  * allocation of the layout above. */
