@@ -28,6 +28,7 @@ def _rank_main(rank, world, heads, head_chunk, calls, shm_name, out):
         # flags[r][kind_index][writer], slots[r][exchange][buffer][writer] (epochs)
         flags = np.ndarray((world, N_FLAGS, world), dtype=np.uint32, buffer=shm.buf, offset=0)
         slots = np.ndarray((world, 2, 2, world), dtype=np.uint32, buffer=shm.buf, offset=flags.nbytes)
+        ready = np.ndarray((world,), dtype=np.uint32, buffer=shm.buf, offset=flags.nbytes + slots.nbytes)
         tokens = 8 * world
         plan = ulysses.UlyssesPlan(world, tokens, tokens, heads, 128, head_chunk)
         size = ulysses.PeerExchange.layout(plan)["total"]
@@ -48,7 +49,7 @@ def _rank_main(rank, world, heads, head_chunk, calls, shm_name, out):
             k = index_of(flag_view.data_ptr() - local.data_ptr())
             t0 = time.monotonic()
             while not np.all(flags[rank, k] == value):
-                if time.monotonic() - t0 > 20.0:
+                if time.monotonic() - t0 > 60.0:
                     raise TimeoutError(f"rank {rank} waits on flag set {k} for {value:#x}: {flags[rank, k]}")
                 time.sleep(0.0005)
 
@@ -92,6 +93,13 @@ def _rank_main(rank, world, heads, head_chunk, calls, shm_name, out):
 
         layer = ulysses.LightUlysses(plan, device="cpu", ops=Ops(), exchange=ex)
         x = torch.zeros(plan.tokens_local, 3, heads, 128, dtype=torch.bfloat16)
+        # start together: process start-up (imports) must not count against the waits
+        ready[rank] = 1
+        t0 = time.monotonic()
+        while not np.all(ready == 1):
+            if time.monotonic() - t0 > 300.0:
+                raise TimeoutError("not every rank started")
+            time.sleep(0.001)
         for _ in range(calls):
             layer.forward(x)
         out.put((rank, "ok"))
@@ -106,7 +114,7 @@ def _rank_main(rank, world, heads, head_chunk, calls, shm_name, out):
 @pytest.mark.parametrize("world,heads,head_chunk,calls", [(2, 12, 1, 2), (3, 12, 1, 2), (4, 24, 1, 1)])
 def test_every_rank_runs_its_own_schedule_without_deadlock(world, heads, head_chunk, calls):
     from multiprocessing import shared_memory
-    nbytes = world * N_FLAGS * world * 4 + world * 2 * 2 * world * 4
+    nbytes = world * N_FLAGS * world * 4 + world * 2 * 2 * world * 4 + world * 4
     shm = shared_memory.SharedMemory(create=True, size=nbytes)
     try:
         np.ndarray((nbytes,), dtype=np.uint8, buffer=shm.buf)[:] = 0
@@ -116,7 +124,7 @@ def test_every_rank_runs_its_own_schedule_without_deadlock(world, heads, head_ch
                  for r in range(world)]
         for p in procs:
             p.start()
-        results = dict(out.get(timeout=120) for _ in range(world))
+        results = dict(out.get(timeout=600) for _ in range(world))
         for p in procs:
             p.join(timeout=60)
         assert all(v == "ok" for v in results.values()), results
