@@ -1,0 +1,83 @@
+"""The GPU parity checkers themselves, on the CPU: they must accept exactly what the
+tolerances allow and reject the rest (a checker that accepts everything would make every
+GPU parity result meaningless)."""
+import numpy as np
+import pytest
+import torch
+
+from tests import parity_utils as pu
+
+
+def _means():
+    # one (b, h), four blocks, d = 2; query block 0 scores key blocks 1 and 2 equally
+    qm = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0], [0.5, -1.0]])[None, None]
+    km = np.array([[2.0, 0.0], [1.0, 5.0], [1.0, -3.0], [0.25, 0.0]])[None, None]
+    return qm, km
+
+
+def _oracle_cols(qm, km, k):
+    nb = qm.shape[2]
+    out = np.empty((1, 1, nb, k), dtype=np.int32)
+    for i in range(nb):
+        s = km[0, 0] @ qm[0, 0, i]
+        others = sorted((j for j in range(nb) if j != i), key=lambda j: (-s[j], j))
+        out[0, 0, i] = sorted([i] + others[:k - 1])
+    return out
+
+
+def test_selection_identical_and_tie_swap_accepted():
+    qm, km = _means()
+    ora = _oracle_cols(qm, km, 2)
+    assert pu.assert_selection_ok(ora.copy(), ora, qm, km, 2) == 0
+    # row 0: blocks 1 and 2 both score 1.0; the oracle keeps 1 (lower index), taking 2 is a tie swap
+    assert list(ora[0, 0, 0]) == [0, 1]
+    gpu = ora.copy()
+    gpu[0, 0, 0] = [0, 2]
+    assert pu.assert_selection_ok(gpu, ora, qm, km, 2) == 1
+
+
+def test_selection_rejects_real_differences():
+    qm, km = _means()
+    ora = _oracle_cols(qm, km, 2)
+    bad = ora.copy()
+    bad[0, 0, 0] = [0, 3]  # block 3 scores 0.25, far from the k-th score 1.0
+    with pytest.raises(AssertionError):
+        pu.assert_selection_ok(bad, ora, qm, km, 2)
+    no_diag = ora.copy()
+    no_diag[0, 0, 1] = [0, 2]
+    with pytest.raises(AssertionError):
+        pu.assert_selection_ok(no_diag, ora, qm, km, 2)
+    unsorted = ora.copy()
+    unsorted[0, 0, 0] = [1, 0]
+    with pytest.raises(AssertionError):
+        pu.assert_selection_ok(unsorted, ora, qm, km, 2)
+    out_of_range = ora.copy()
+    out_of_range[0, 0, 3] = [3, 4]
+    with pytest.raises(AssertionError):
+        pu.assert_selection_ok(out_of_range, ora, qm, km, 2)
+
+
+def test_attention_tolerance_bounds():
+    ref = np.random.default_rng(0).standard_normal((2, 3, 64, 8))
+    exact = torch.from_numpy(ref)
+    pu.assert_attention_close(exact, ref)
+    one_big = exact.clone()
+    one_big[0, 0, 0, 0] += 0.03  # max-abs 3e-2 > 2e-2
+    with pytest.raises(AssertionError):
+        pu.assert_attention_close(one_big, ref)
+    shifted = exact + 3e-3  # every element within the max bound, the mean beyond 2e-3
+    with pytest.raises(AssertionError):
+        pu.assert_attention_close(shifted, ref)
+    within = exact + 1.5e-3
+    pu.assert_attention_close(within, ref)
+    nan = exact.clone()
+    nan[1, 2, 3, 4] = float("nan")
+    with pytest.raises(AssertionError):
+        pu.assert_attention_close(nan, ref)
+
+
+def test_mean_tolerance_bounds():
+    ref = np.random.default_rng(1).standard_normal((1, 2, 4, 8))
+    pu.assert_means_close(torch.from_numpy(ref * (1 + 1e-7)), ref)
+    with pytest.raises(AssertionError):
+        pu.assert_means_close(torch.from_numpy(ref * (1 + 1e-4)), ref)
