@@ -81,3 +81,21 @@ def test_mean_tolerance_bounds():
     pu.assert_means_close(torch.from_numpy(ref * (1 + 1e-7)), ref)
     with pytest.raises(AssertionError):
         pu.assert_means_close(torch.from_numpy(ref * (1 + 1e-4)), ref)
+
+
+def test_nvfp4_gemm_bound():
+    """One bf16 rounding of the exact product is accepted; an error of a few bf16 steps is
+    not (a dropped or doubled K-block, a wrong scale, would be far larger)."""
+    from tests.test_gpu_nvfp4 import _check_gemm
+    rng = np.random.default_rng(2)
+    a = rng.standard_normal((32, 64))
+    b = rng.standard_normal((48, 64))
+    ref = a @ b.T
+    rounded = torch.from_numpy(ref).to(torch.bfloat16)  # the kernel's output rounding
+    assert _check_gemm(rounded, ref, a, b) <= 1.0
+    off = torch.from_numpy(ref * (1 + 2.0 ** -5)).to(torch.bfloat16)
+    with pytest.raises(AssertionError):
+        _check_gemm(off, ref, a, b)
+    dropped = torch.from_numpy(a[:, :48] @ b[:, :48].T).to(torch.bfloat16)  # one quarter of K missing
+    with pytest.raises(AssertionError):
+        _check_gemm(dropped, ref, a, b)
