@@ -99,3 +99,43 @@ def test_nvfp4_gemm_bound():
     dropped = torch.from_numpy(a[:, :48] @ b[:, :48].T).to(torch.bfloat16)  # one quarter of K missing
     with pytest.raises(AssertionError):
         _check_gemm(dropped, ref, a, b)
+
+
+def test_rope_checker():
+    """The oracle's own rotation passes; two bf16 steps on one element, one step on 2% of
+    the elements, swapped pair members, or a touched padded token do not."""
+    import oracle
+    from tests.test_gpu_rope import _check_tensor
+    from video_dit_dynamic_b200 import inputs
+    grid, L, blk = (2, 3, 9), 54, 32
+    g = torch.Generator().manual_seed(3)
+    x = torch.randn(1, 2, 64, 32, generator=g)
+    x[:, :, L:] = 0.5  # padded tokens: passed through
+    x = x.to(torch.bfloat16)
+    ref_bits, _ = oracle.rope_pool(inputs.bf16_bits(x), grid, L, blk)
+
+    def as_t(bits):
+        return torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16)
+
+    def run(bits):
+        means = torch.from_numpy(oracle.pool(bits, L, blk))
+        return _check_tensor(x, as_t(bits), means, grid, L, blk)
+
+    assert run(ref_bits.copy()) == 0.0
+    two_steps = ref_bits.copy()
+    two_steps[0, 0, 5, 7] += 2
+    with pytest.raises(AssertionError):
+        run(two_steps)
+    many = ref_bits.copy().reshape(-1)
+    idx = np.arange(0, L * 32, 40)  # about 2.5% of the valid elements of the first head, one step each
+    many[idx] = many[idx] + 1
+    with pytest.raises(AssertionError):
+        run(many.reshape(ref_bits.shape))
+    swapped = ref_bits.copy()
+    swapped[..., 0::2], swapped[..., 1::2] = ref_bits[..., 1::2], ref_bits[..., 0::2]
+    with pytest.raises(AssertionError):
+        run(swapped)
+    padded = ref_bits.copy()
+    padded[0, 1, L + 2, 0] ^= 1
+    with pytest.raises(AssertionError):
+        run(padded)
