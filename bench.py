@@ -52,7 +52,6 @@ def parse():
     ap.add_argument("--no-fp8", action="store_true", help="skip timing the FP8 path")
     ap.add_argument("--no-nvfp4", action="store_true", help="skip timing the NVFP4 linear layer")
     ap.add_argument("--no-ulysses", action="store_true", help="skip timing the Light-Ulysses kernels")
-    ap.add_argument("--cpu-units", type=int, default=16, help="attention units in the CPU sample")
     return ap.parse_args()
 
 
@@ -245,59 +244,76 @@ def recorded_traffic(kernel_src: str, workload_name: str):
 
 
 # ------------------------------------------------------------------ CPU oracle sample
-def cpu_oracle_sample(wl: inputs.Workload, k: int, q, kt, v, n_units: int, seed: int = 0,
-                      single_core_units: int = 0):
-    """Time the oracle on a bounded sample of the layer: pool + select of one full head
-    and attention of n_units (head 0, query block) units; extrapolate to the layer."""
+CPU_SAMPLE_UNITS = 64  # attention units of the CPU sample
+
+
+def cpu_sample_inputs(wl: inputs.Workload, q=None, kt=None, v=None):
+    """Head 0 of the layer as bf16 bits on the host: from the given tensors (the GPU arm's)
+    or freshly generated (the reference arm).  The sample's work does not depend on the
+    values, only on the shapes."""
+    if q is None:
+        one = inputs.Workload(wl.name, 1, 1, wl.grid, wl.head_dim, wl.block, wl.keep, wl.kind)
+        q, kt, v = inputs.make_qkv(one, seed=0, device="cpu")
+    return tuple(inputs.bf16_bits(t[:, 0:1]) for t in (q, kt, v))
+
+
+def cpu_oracle_sample(wl: inputs.Workload, k: int, qb, kb, vb, n_units: int = CPU_SAMPLE_UNITS):
+    """Time the oracle on one bounded sample of the layer: pool + select of one full head
+    and attention of n_units (head 0, query block) units, the same units in every call and
+    in both arms; extrapolated to the layer (40 heads x all query blocks).  Returns
+    (seconds per layer, description)."""
     import numpy as np
     import oracle
-    oracle.set_threads(os.cpu_count() or 1)
-    cores = oracle.threads_used()
-    h = 0
-    qb = inputs.bf16_bits(q[:, h:h + 1])
-    kb = inputs.bf16_bits(kt[:, h:h + 1])
-    vb = inputs.bf16_bits(v[:, h:h + 1])
     L, blk, nb = wl.seq_len, wl.block, wl.num_blocks
     t0 = time.perf_counter()
     qm = oracle.pool(qb, L, blk)
     km = oracle.pool(kb, L, blk)
     col = oracle.select(qm, km, k)
     t_ps = time.perf_counter() - t0
-    rng = np.random.default_rng(seed)
-    units = sorted(rng.choice(nb, size=min(n_units, nb), replace=False).tolist())
+    units = sorted(np.random.default_rng(12345).choice(nb, size=min(n_units, nb), replace=False).tolist())
     rp = oracle.uniform_row_ptr(1, 1, nb, k)
     t0 = time.perf_counter()
     oracle.attention(qb, kb, vb, L, blk, rp, col, units=units)
     t_at = time.perf_counter() - t0
     heads = wl.heads * wl.batch
     layer_s = t_ps * heads + t_at / len(units) * (nb * heads)
-    tflops = layer_flops(wl, k) / layer_s / 1e12
-    out = {
-        "value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-        "sample": (f"pool+select of 1 of {heads} heads ({t_ps:.2f} s) and attention of {len(units)} of "
-                   f"{nb * heads} (head, query-block) units ({t_at:.2f} s), extrapolated to the layer: "
-                   f"{layer_s:.1f} s/layer"),
-        "layer_seconds_extrapolated": layer_s,
-    }
-    if single_core_units > 0:
-        # the same kind of sample on one core (fewer attention units)
-        oracle.set_threads(1)
-        try:
-            t0 = time.perf_counter()
-            col1 = oracle.select(oracle.pool(qb, L, blk), oracle.pool(kb, L, blk), k)
-            t_ps1 = time.perf_counter() - t0
-            units1 = units[:single_core_units]
-            t0 = time.perf_counter()
-            oracle.attention(qb, kb, vb, L, blk, rp, col1, units=units1)
-            t_at1 = time.perf_counter() - t0
-        finally:
-            oracle.set_threads(os.cpu_count() or 1)
-        layer_s1 = t_ps1 * heads + t_at1 / len(units1) * (nb * heads)
-        out["single_core"] = {
-            "value": layer_flops(wl, k) / layer_s1 / 1e12, "unit": "TFLOP/s", "cores": 1,
-            "sample": (f"pool+select of 1 of {heads} heads ({t_ps1:.2f} s) and attention of {len(units1)} units "
-                       f"({t_at1:.2f} s) on one core, extrapolated to the layer: {layer_s1:.1f} s/layer")}
+    desc = (f"pool+select of 1 of {heads} heads ({t_ps:.2f} s) and attention of {len(units)} of "
+            f"{nb * heads} (head, query-block) units ({t_at:.2f} s), extrapolated to the layer")
+    return layer_s, desc
+
+
+def cpu_baseline_line(wl: inputs.Workload, k: int, samples_s: list, desc: str, cores: int, extra=None) -> dict:
+    """The cpu_baseline object: the mean over the timed samples, with their spread."""
+    layer_s = statistics.mean(samples_s)
+    out = {"value": layer_flops(wl, k) / layer_s / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+           "sample": f"{desc}; {len(samples_s)} timed samples after one untimed: {layer_s:.1f} s/layer",
+           "layer_seconds": layer_s,
+           "spread": {"min_TFLOP/s": layer_flops(wl, k) / max(samples_s) / 1e12,
+                      "max_TFLOP/s": layer_flops(wl, k) / min(samples_s) / 1e12,
+                      "samples": len(samples_s)}}
+    if extra:
+        out.update(extra)
     return out
+
+
+def gpu_arm_cpu_baseline(wl: inputs.Workload, k: int, q, kt, v, repeats: int = 3) -> dict:
+    """The GPU arm's cpu_baseline: the reference arm's sample (same heads, units and
+    oracle), one untimed call, then `repeats` timed ones on all host cores; plus the same
+    sample on one core."""
+    import oracle
+    qb, kb, vb = cpu_sample_inputs(wl, q, kt, v)
+    oracle.set_threads(os.cpu_count() or 1)
+    cores = oracle.threads_used()
+    cpu_oracle_sample(wl, k, qb, kb, vb)
+    runs = [cpu_oracle_sample(wl, k, qb, kb, vb) for _ in range(repeats)]
+    oracle.set_threads(1)
+    try:
+        one_s, one_desc = cpu_oracle_sample(wl, k, qb, kb, vb, n_units=4)
+    finally:
+        oracle.set_threads(os.cpu_count() or 1)
+    single = {"value": layer_flops(wl, k) / one_s / 1e12, "unit": "TFLOP/s", "cores": 1,
+              "sample": one_desc.replace(f"{CPU_SAMPLE_UNITS} of", "4 of") + " (one core)"}
+    return cpu_baseline_line(wl, k, [r[0] for r in runs], runs[0][1], cores, {"single_core": single})
 
 
 # ------------------------------------------------------------------ reference arm
@@ -305,29 +321,28 @@ def run_reference(args, wl):
     ws, rank, _ = dist_env()
     if rank != 0:
         return
+    import oracle
     nb = wl.num_blocks
     k = keep_count(nb, wl.keep)
-    q, kt, v = inputs.make_qkv(inputs.Workload(wl.name, 1, 1, wl.grid, wl.head_dim, wl.block, wl.keep),
-                               seed=0, device="cpu")
-    # every step is a bounded sample (one head) of the same layer, extrapolated
-    results = []
+    qb, kb, vb = cpu_sample_inputs(wl)
+    oracle.set_threads(os.cpu_count() or 1)
+    cores = oracle.threads_used()
+    # every step is the same bounded sample of the layer (one head's pool + select and
+    # 64 attention units), extrapolated; the warm-up steps are not timed
+    samples, desc = [], ""
     for i in range(args.warmup + args.steps):
-        r = cpu_oracle_sample(inputs.Workload(wl.name, 1, wl.heads, wl.grid, wl.head_dim, wl.block, wl.keep),
-                              k, q, kt, v, n_units=args.cpu_units, seed=i)
+        layer_s, desc = cpu_oracle_sample(wl, k, qb, kb, vb)
         if i >= args.warmup:
-            results.append(r)
-    layer_s = statistics.mean(r["layer_seconds_extrapolated"] for r in results)
-    value = layer_flops(wl, k) / layer_s / 1e12
-    cb = dict(results[-1])
-    cb["value"] = value
-    cb.pop("layer_seconds_extrapolated", None)
+            samples.append(layer_s)
+    cb = cpu_baseline_line(wl, k, samples, desc, cores)
+    value = cb["value"]
     line = {
         "impl": "reference", "metric": "sparse-attn ms/layer & TFLOP/s (selected blocks) at L=122880, 90% sparse",
         "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": layer_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "ms_per_step": cb["layer_seconds"] * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "config": config_of(wl, k, "oracle on host cores; sample per step, extrapolated"),
-        "cpu_baseline": cb,
+        "config": config_of(wl, k, "oracle on host cores; one bounded sample per step, extrapolated to the layer"),
+        "cpu_baseline": {kk: vv for kk, vv in cb.items() if kk != "layer_seconds"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -666,8 +681,9 @@ def run_gpu(args, wl):
                            "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
                            "d2h_bytes_per_step": e2e["d2h_bytes_per_step"], "ms_per_step": e2e["ms"]}
         if ws_n == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_oracle_sample(wl, k, q, kt, v, args.cpu_units, single_core_units=4)
-            line["cpu_baseline"].pop("layer_seconds_extrapolated", None)
+            cb = gpu_arm_cpu_baseline(wl, k, q, kt, v)
+            cb.pop("layer_seconds", None)
+            line["cpu_baseline"] = cb
         print(json.dumps(line), flush=True)
     if pg is not None:
         pg.barrier()

@@ -302,6 +302,33 @@ sbsa_status sbsa_forward(const sbsa_shape *shape, const void *q, const void *k, 
                          float scale, void *o, int32_t *col_idx_out, void *workspace, size_t workspace_bytes,
                          void *stream);
 
+/* Steps 1-3 end to end from host memory (page "单卡 RTX 5090 跑 Wan2.2-A14B：720p 视频
+ * 生成只要 3.8 秒", section 四步拆解, item 3, computed as sbsa_forward does): copies Q, K, V
+ * from the host into the device buffers q, k, v, runs pool -> select -> attend, and
+ * copies O from the device buffer o back to o_host.
+ *   q_host, k_host, v_host, o_host: HOST memory, [B][H][Lp][d] bf16 (Lp rows per
+ *   (batch, head), padded rows included).  Pinned (page-locked) memory is what lets the
+ *   copies run asynchronously and overlap the kernels; pageable memory gives the same
+ *   result with copies the driver stages.  q, k, v, o: device buffers of the same size,
+ *   16-byte aligned; workspace as for sbsa_forward (the full shape's size).
+ *   The (batch, head) pairs are independent, so the call processes them in chunks of
+ *   pairs_per_chunk pairs (0: about eight chunks): the copy-in of a chunk on h2d_stream,
+ *   its three kernels on `stream` and its copy-out on d2h_stream, with events between the
+ *   streams, so that copies of one chunk overlap the kernels of its neighbours.  One
+ *   cudaMemcpyAsync per tensor and chunk.  The result equals one sbsa_forward call on the
+ *   whole shape bit for bit.  h2d_stream / d2h_stream may be NULL (then `stream` does
+ *   the copies too, without overlap); one stream for both copy directions is correct but
+ *   serializes each copy-out with the next copy-in.
+ *   Asynchronous: the work, copies included, is complete when `stream` is (the call makes
+ *   `stream` wait for the last copy-out, and the first copy-in wait for work already
+ *   queued on `stream`).  Host and device buffers must stay valid until then.  Creates
+ *   and releases three CUDA events per call; allocates no memory.  On an error returned
+ *   part way, the work already queued still runs; the returned status says what failed. */
+sbsa_status sbsa_forward_host(const sbsa_shape *shape, const void *q_host, const void *k_host, const void *v_host,
+                              int32_t k_keep, float scale, void *o_host, void *q, void *k, void *v, void *o,
+                              void *workspace, size_t workspace_bytes, int32_t pairs_per_chunk, void *stream,
+                              void *h2d_stream, void *d2h_stream);
+
 /* sbsa_forward without a workspace, for callers that cannot allocate device memory:
  * for example a plug-in inside another engine that owns every device allocation, or
  * a latency-critical loop where cudaMalloc/cudaFree would synchronize the device.
@@ -312,8 +339,10 @@ sbsa_status sbsa_forward(const sbsa_shape *shape, const void *q, const void *k, 
  *   with sbsa_workspace_bytes(shape, k_keep) > 16 MiB (16,777,216 bytes) are rejected
  *   with SBSA_ERR_WORKSPACE before anything is launched.  Example: the 480p case
  *   (40 heads, 256 blocks of 128, d = 128, k = 51) needs 12.6 MB.
- *   The first call on a device looks up the scratch array's device address, with
- *   that device current; make that first call before any stream capture.
+ *   Every call looks up the scratch array's device address in the current context
+ *   (cudaGetSymbolAddress: a lookup, not an allocation), so the address stays valid
+ *   after a device reset or a context switch.  The first call on a device may load
+ *   the library's device code; make that first call before any stream capture.
  *   All calls share the one array, and it keeps the last call's contents.  Calls
  *   whose work overlaps on the GPU (different streams, or different host threads
  *   without ordering) race on it and must be serialized by the caller.  Every scratch
@@ -322,6 +351,18 @@ sbsa_status sbsa_forward(const sbsa_shape *shape, const void *q, const void *k, 
  *   library routine. */
 sbsa_status sbsa_forward_noalloc(const sbsa_shape *shape, const void *q, const void *k, const void *v,
                                  int32_t k_keep, float scale, void *o, int32_t *col_idx_out, void *stream);
+
+/* Failure handling (a bounded wait in every kernel pipeline, latched as
+ * SBSA_ERR_TIMEOUT; nothing traps): sets, on the current device, the limit of the
+ * pipeline waits of the attention, selection, RoPE + pooling and FP8 quantizer kernels
+ * launched afterwards.  Default 1e9 ns (1 s), far above any legitimate wait.  0 makes a
+ * pipeline wait give up unless its barrier has already completed when first tested: a
+ * test uses it to drive the give-up path (latch the error, make the launch's other CTAs
+ * stop, wait for this CTA's own copies and tensor-core work, release its tensor memory)
+ * without stalling a pipeline.  The waits of that drain keep their own 1 s limit.  The
+ * NVFP4 GEMM keeps its fixed 1 s limit.  Synchronous; not for use while kernels of this
+ * library run on the device. */
+sbsa_status sbsa_set_pipeline_wait_ns(uint64_t limit_ns);
 
 /* Synchronizes `stream`, then reads and clears the calling device's error word.
  * Returns SBSA_OK, SBSA_ERR_TIMEOUT, SBSA_ERR_BAD_INDEX or SBSA_ERR_CUDA (a sticky

@@ -65,9 +65,12 @@ def assert_means_close(gpu, ref):
 
 
 def assert_selection_ok(gpu_col: np.ndarray, ora_col: np.ndarray, qmean: np.ndarray, kmean: np.ndarray, k: int,
-                        rows=None):
+                        rows=None, stats=None):
     """gpu_col / ora_col: [B,H,nb,k]; qmean/kmean: [B,H,nb,d] float64 (the oracle's).
-    Returns the number of rows that differ only by tolerated tie swaps."""
+    Returns the number of rows that differ only by tolerated tie swaps.  If `stats` is a
+    dict it receives "swaps" (that count) and "wide_swaps": the rows among them where a
+    swapped block's score is further than TIE_REL * |s_k| from the k-th score, i.e. rows
+    accepted only through the sum-of-magnitudes term of the bound."""
     B, H, nb, _ = qmean.shape
     g = gpu_col.reshape(B * H, nb, k)
     o = ora_col.reshape(B * H, nb, k)
@@ -80,7 +83,7 @@ def assert_selection_ok(gpu_col: np.ndarray, ora_col: np.ndarray, qmean: np.ndar
     differ = np.nonzero(np.any(g != o, axis=-1))
     qm = qmean.reshape(B * H, nb, -1)
     km = kmean.reshape(B * H, nb, -1)
-    swaps = 0
+    swaps = wide = 0
     for bh, i in zip(*differ):
         if rows is not None and (bh, i) not in rows:
             continue
@@ -88,11 +91,17 @@ def assert_selection_ok(gpu_col: np.ndarray, ora_col: np.ndarray, qmean: np.ndar
         s = km[bh] @ qm[bh, i]
         a = np.abs(km[bh]) @ np.abs(qm[bh, i])
         sk = min(s[j] for j in O if j != i)
+        is_wide = False
         for j in G ^ O:
             bound = TIE_REL * max(abs(sk), a[j])
             assert abs(s[j] - sk) <= bound, (
                 f"row (bh={bh}, i={i}): block {j} score {s[j]!r} vs k-th {sk!r} differs by more than the tie bound")
+            is_wide |= abs(s[j] - sk) > TIE_REL * abs(sk)
         swaps += 1
+        wide += int(is_wide)
+    if stats is not None:
+        stats["swaps"] = swaps
+        stats["wide_swaps"] = wide
     return swaps
 
 

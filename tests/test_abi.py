@@ -104,6 +104,16 @@ def test_argument_errors_return_before_launch(lib):
     assert b"smaller" in lib.sbsa_last_error_message()
     # null shape
     assert lib.sbsa_pool_qk(None, fake, fake, fake, fake, None) == 1
+    # the host entry point: null host or device pointers, a negative chunk, a short workspace
+    f0 = ctypes.c_float(0)
+    assert lib.sbsa_forward_host(ctypes.byref(good), None, fake, fake, 4, f0, fake, fake, fake, fake, fake, fake,
+                                 1 << 30, 0, None, None, None) == 1
+    assert lib.sbsa_forward_host(ctypes.byref(good), fake, fake, fake, 4, f0, fake, fake, None, fake, fake, fake,
+                                 1 << 30, 0, None, None, None) == 1
+    assert lib.sbsa_forward_host(ctypes.byref(good), fake, fake, fake, 4, f0, fake, fake, fake, fake, fake, fake,
+                                 1 << 30, -1, None, None, None) == 1
+    assert lib.sbsa_forward_host(ctypes.byref(good), fake, fake, fake, 4, f0, fake, fake, fake, fake, fake, fake,
+                                 16, 0, None, None, None) == 3
 
 
 def test_binding_rejects_cpu_tensors(lib):

@@ -65,8 +65,14 @@ def _check_forward(wl, n_units, full_head=False):
     pu.assert_means_close(km_gpu, km)
     ref_col = oracle.select(qm, km, kk)
     gcol = col.cpu().numpy().reshape(1, H, nb, kk)
-    swaps = pu.assert_selection_ok(gcol, ref_col, qm, km, kk)
+    st = {}
+    swaps = pu.assert_selection_ok(gcol, ref_col, qm, km, kk, stats=st)
+    # reported in the run's output: rows differing from the oracle by tie swaps, and those
+    # among them that needed the sum-of-magnitudes term beyond 1e-5 * |s_k|
+    print(f"\n[selection] {name}: {rows} rows, {swaps} differ by tie swaps, "
+          f"{st['wide_swaps']} of them beyond 1e-5*|s_k|")
     assert swaps <= rows // 100, f"{swaps} rows differ by tie swaps"
+    assert st["wide_swaps"] == 0, f"{st['wide_swaps']} rows accepted only by the sum-of-magnitudes term"
     units = _sample_units(H, nb, n_units, seed=nb)
     if full_head:
         units = sorted(set(units) | set(range((H - 1) * nb, H * nb)))

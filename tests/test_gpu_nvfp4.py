@@ -9,8 +9,9 @@
   accumulation term of 2^-16 of sum_k |A_k B_k| (fp32 accumulation of K <= 5120 exact
   products is far below it);
 - end to end: GPU amax -> quantize -> GEMM against the oracle's quantize -> GEMM;
-- the full-size layer (122,880 x 5,120 activations, 15,360 x 5,120 weights): sampled rows
-  quantized by the oracle with the tensor's amax, and the outputs they produce.
+- the full-size layer (122,880 x 5,120 activations, 15,360 x 5,120 weights): each tensor's
+  amax taken on the host from the full bf16 bits (and the GPU's amax equal to it), sampled
+  rows quantized by the oracle with that host amax, and the outputs they produce.
 """
 import numpy as np
 import pytest
@@ -37,6 +38,14 @@ def _bf16(rows, cols, seed, scale=1.0):
 
 def _amax_of(x_bits):
     return np.float32(np.abs((x_bits.astype(np.uint32) << 16).view(np.float32)).max())
+
+
+def _amax_host(x: torch.Tensor) -> np.float32:
+    """max |x| of a bf16 tensor from its bits on the host: for non-NaN values the order of
+    the magnitude bits (sign cleared) is the order of |x|."""
+    bits = inputs.bf16_bits(x.cpu())
+    top = np.uint32(np.max(bits & np.uint16(0x7FFF)))
+    return np.array([top << np.uint32(16)], dtype=np.uint32).view(np.float32)[0]
 
 
 def _codes_equal(got, ref):
@@ -173,8 +182,11 @@ def test_gemm_full_size_sampled():
     cols = np.sort(np.concatenate([[0, 255, 256, n - 1], rng.choice(n, 60, replace=False)]))
     a_s = inputs.bf16_bits(a[torch.from_numpy(rows).cuda()].cpu())
     b_s = inputs.bf16_bits(b[torch.from_numpy(cols).cuda()].cpu())
-    qa = oracle.nvfp4_quantize(a_s, amax=aam.item())
-    qb = oracle.nvfp4_quantize(b_s, amax=bam.item())
+    # the tensors' amax from the host copies of their bits, independent of the GPU path
+    a_amax, b_amax = _amax_host(a), _amax_host(b)
+    assert aam.item() == a_amax and bam.item() == b_amax, (aam.item(), a_amax, bam.item(), b_amax)
+    qa = oracle.nvfp4_quantize(a_s, amax=float(a_amax))
+    qb = oracle.nvfp4_quantize(b_s, amax=float(b_amax))
     # the sampled rows' codes are the GPU's rows
     got_a = ac.view(m, k // 2)[torch.from_numpy(rows).cuda()].cpu().numpy()
     assert _codes_equal(got_a, qa[0]).all()

@@ -295,3 +295,27 @@ def test_forward_from_host_chunked_pipeline(head_chunk):
     ref = od.cpu()
     for oh in outs:
         assert torch.equal(oh, ref)
+
+
+@pytest.mark.parametrize("pinned,copy_streams", [(True, True), (False, False)])
+def test_forward_host_entry_point(pinned, copy_streams):
+    """sbsa_forward_host through the C ABI: pinned host memory with separate copy streams,
+    and pageable host memory with every copy on the compute stream; both bit-equal to
+    sbsa_forward, with the selection written nowhere else."""
+    B, H, L, d, blk = 1, 6, 1500, 64, 64
+    s = sbsa.make_shape(B, H, L, d, blk)
+    q, k, v = inputs.random_qkv(B, H, s.seq_len_padded, d, L=L, seed=33)
+    kk = sbsa.sbsa_keep_blocks(s.num_blocks, 0.3)
+    od = torch.empty_like(q, device="cuda")
+    sbsa.sbsa_forward(s, q.cuda(), k.cuda(), v.cuda(), kk, 0.0, od, None, sbsa.alloc_workspace(s, kk))
+    hq, hk, hv = ((t.pin_memory() if pinned else t.clone()) for t in (q, k, v))
+    oh = torch.full(q.shape, 3.0, dtype=torch.bfloat16, pin_memory=pinned)
+    dq, dk, dv, do = (torch.empty_like(od) for _ in range(4))
+    ws = sbsa.alloc_workspace(s, kk)
+    side = (torch.cuda.Stream(), torch.cuda.Stream()) if copy_streams else (None, None)
+    st = torch.cuda.current_stream()
+    sbsa.sbsa_forward_host(s, hq, hk, hv, kk, 0.0, oh, dq, dk, dv, do, ws, pairs_per_chunk=4, stream=st,
+                           h2d_stream=side[0], d2h_stream=side[1])
+    st.synchronize()
+    sbsa.sbsa_check()
+    assert torch.equal(oh, od.cpu())

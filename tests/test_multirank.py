@@ -46,7 +46,7 @@ def _rank_main(rank, world, port, out):
         # the reference arm prints on rank 0 only; other ranks exit without work
         buf = io.StringIO()
         if rank != 0:
-            args = type("A", (), {"gpus": world, "steps": 1, "warmup": 3, "cpu_units": 1})()
+            args = type("A", (), {"gpus": world, "steps": 1, "warmup": 3})()
             with contextlib.redirect_stdout(buf):
                 ret = bench.run_reference(args, wl)
             assert ret is None
@@ -93,14 +93,22 @@ def test_job_value_counts_every_rank_over_the_slowest():
     assert bench.max_over_ranks(None, "cpu", {"a": 1.5}) == {"a": 1.5}
 
 
-def test_kernel_spread_and_single_core_oracle_sample():
+def test_kernel_spread_and_cpu_baseline_sample():
     import bench
     from video_dit_dynamic_b200 import inputs
     assert bench.spread([3.0, 1.0, 2.0, 5.0]) == {"ms_median": 2.5, "ms_best": 1.0}
     wl = inputs.WORKLOADS["tiny"]
     k = bench.keep_count(wl.num_blocks, wl.keep)
     q, kt, v = inputs.make_qkv(wl, seed=0, device="cpu")
-    r = bench.cpu_oracle_sample(wl, k, q, kt, v, n_units=4, single_core_units=2)
+    # the GPU arm's baseline: the reference arm's sample, repeated, with its spread, plus one core
+    r = bench.gpu_arm_cpu_baseline(wl, k, q, kt, v, repeats=2)
     assert r["kind"] == "oracle" and r["value"] > 0 and r["cores"] >= 1
+    assert r["spread"]["samples"] == 2
+    assert r["spread"]["min_TFLOP/s"] <= r["value"] <= r["spread"]["max_TFLOP/s"]
     sc = r["single_core"]
     assert sc["cores"] == 1 and sc["value"] > 0 and "one core" in sc["sample"]
+    # both arms time the same sample: the same heads' bits go in whichever tensors they come from
+    a = bench.cpu_sample_inputs(wl, q, kt, v)
+    b = bench.cpu_sample_inputs(wl)
+    assert all(x.shape == y.shape and x.dtype == y.dtype for x, y in zip(a, b))
+    assert all((x == y).all() for x, y in zip(a, b))  # seed 0 on the host in both

@@ -36,6 +36,29 @@ def test_selection_identical_and_tie_swap_accepted():
     assert pu.assert_selection_ok(gpu, ora, qm, km, 2) == 1
 
 
+def test_selection_counts_swaps_that_need_the_magnitude_term():
+    # row 0: block 2 scores 1.001 and block 1 scores 1.0, each the sum of two large terms of
+    # opposite sign (sum of magnitudes about 2000); taking block 1 instead of 2 is 1e-3 away
+    # from the k-th score: beyond 1e-5 * |s_k| but within 1e-5 * 2000
+    qm = np.array([[1.0, 1.0], [0.0, 1.0], [1.0, 0.0], [0.5, 0.5]])[None, None]
+    km = np.array([[0.0, 0.0], [1000.0, -999.0], [1000.0, -998.999], [0.0, 0.0]])[None, None]
+    ora = _oracle_cols(qm, km, 2)
+    assert list(ora[0, 0, 0]) == [0, 2]
+    gpu = ora.copy()
+    gpu[0, 0, 0] = [0, 1]
+    st = {}
+    assert pu.assert_selection_ok(gpu, ora, qm, km, 2, stats=st) == 1
+    assert st == {"swaps": 1, "wide_swaps": 1}
+    # an exact tie swap is not a wide one
+    qm2, km2 = _means()
+    ora2 = _oracle_cols(qm2, km2, 2)
+    gpu2 = ora2.copy()
+    gpu2[0, 0, 0] = [0, 2]
+    st2 = {}
+    pu.assert_selection_ok(gpu2, ora2, qm2, km2, 2, stats=st2)
+    assert st2 == {"swaps": 1, "wide_swaps": 0}
+
+
 def test_selection_rejects_real_differences():
     qm, km = _means()
     ora = _oracle_cols(qm, km, 2)

@@ -36,9 +36,10 @@
 // 384 (D columns each).  For BLK = 64 the 128-row Q tile also holds the next block's
 // 64 rows; those rows are computed and discarded.
 //
-// Every wait is bounded (kWaitLimitNs); a wait that runs out latches SBSA_ERR_TIMEOUT,
-// makes every CTA of the launch give up, drains this CTA's own copies and MMAs and
-// frees its TMEM before returning.
+// Every wait is bounded (the pipeline limit, 1 s unless a test lowered it); a wait that
+// runs out latches SBSA_ERR_TIMEOUT, makes every CTA of the launch give up, drains this
+// CTA's own copies and MMAs (each drain wait bounded by 1 s) and frees its TMEM before
+// returning.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -233,8 +234,9 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
         *abort_flag = 1;
         abort_launch(p.epoch);
     };
+    const uint64_t pipe_limit = pipe_wait_ns();  // pipeline waits; the drain below keeps kWaitLimitNs
     auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
-        if (mbar_wait_bounded(bar, parity, abort_flag, kWaitLimitNs)) return true;
+        if (mbar_wait_bounded(bar, parity, abort_flag, pipe_limit)) return true;
         if (!*abort_flag) give_up();
         return false;
     };

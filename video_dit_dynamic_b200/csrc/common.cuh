@@ -22,8 +22,21 @@ constexpr unsigned int kErrTimeout = 1u << 5;   // SBSA_ERR_TIMEOUT
 constexpr unsigned int kErrBadIndex = 1u << 6;  // SBSA_ERR_BAD_INDEX
 
 // Upper bound on any single wait inside a kernel.  Every legitimate wait is
-// microseconds long; this only ends a kernel whose pipeline has stalled.
+// microseconds long; this only ends a kernel whose pipeline has stalled.  The waits a
+// CTA makes after giving up, for its own copies and tensor-core work still in flight
+// (the drain), always use this limit.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
+
+// Limit of the pipeline waits (everything but the drain) of the attention, selection,
+// RoPE + pooling and FP8 quantizer kernels, per device; kWaitLimitNs unless
+// sbsa_set_pipeline_wait_ns changed it.  0 makes a pipeline wait give up unless its
+// barrier has already completed at the first test, which lets a test drive the
+// give-up path without a stalled pipeline.
+__device__ unsigned long long g_pipe_wait_ns = kWaitLimitNs;
+
+__device__ __forceinline__ uint64_t pipe_wait_ns() {
+    return *reinterpret_cast<volatile unsigned long long*>(&g_pipe_wait_ns);
+}
 
 __device__ __forceinline__ void raise_error(unsigned int bits) { atomicOr(&g_error_bits, bits); }
 

@@ -64,6 +64,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     constexpr uint32_t kSuspendNs = 20000;
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
+    if (limit_ns == 0) return false;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait_suspend(a, parity, kSuspendNs)) return true;
@@ -90,6 +91,7 @@ __device__ __forceinline__ bool mbar_wait_bounded_cluster(uint64_t* bar, uint32_
     constexpr uint32_t kSuspendNs = 20000;
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait_cluster(a, parity, 0)) return true;
+    if (limit_ns == 0) return false;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait_cluster(a, parity, kSuspendNs)) return true;

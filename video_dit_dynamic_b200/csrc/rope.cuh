@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(256) rope_pool_kernel(const uint4* q_in, const
 
     __syncthreads();  // the barrier is initialised before anyone waits on it
     volatile int never = 0;
-    if (!mbar_wait_bounded(&full, 0, &never, kWaitLimitNs)) {
+    if (!mbar_wait_bounded(&full, 0, &never, pipe_wait_ns())) {
         if (threadIdx.x == 0) abort_launch(epoch);
         // give the copy one more bounded wait to land before the shared memory is released
         mbar_wait_bounded(&full, 0, &never, kWaitLimitNs);

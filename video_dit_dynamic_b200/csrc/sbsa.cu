@@ -426,29 +426,19 @@ __global__ void validate_csr_kernel(const int32_t* row_ptr, const int32_t* col_i
 // fixed module-scope array instead of a caller-provided workspace.  Every GPU that
 // loads the library reserves it for the life of the process.  Host code must never
 // hand the symbol itself to a kernel (on the host it is only a stand-in); its device
-// address is looked up once per device with cudaGetSymbolAddress.
+// address is looked up with cudaGetSymbolAddress in the current context on every call
+// (a lookup, not an allocation), so the address stays right after a device reset or a
+// context switch, which load the module again.
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
-constexpr int kMaxDevices = 256;
-void* g_noalloc_ptr[kMaxDevices];
-std::mutex g_noalloc_mu;
-
-// Device address of the scratch array on the current device (looked up on first use).
+// Device address of the scratch array in the current context.
 sbsa_status noalloc_scratch(void** out) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-    if (dev < 0 || dev >= kMaxDevices) return fail(SBSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
-        g_noalloc_ptr[dev] = p;
-    }
-    *out = g_noalloc_ptr[dev];
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    *out = p;
     return SBSA_OK;
 }
 }  // namespace
@@ -899,6 +889,91 @@ sbsa_status sbsa_forward(const sbsa_shape* shape, const void* q, const void* k, 
     return ok();
 }
 
+sbsa_status sbsa_forward_host(const sbsa_shape* shape, const void* q_host, const void* k_host, const void* v_host,
+                              int32_t k_keep, float scale, void* o_host, void* q, void* k, void* v, void* o,
+                              void* workspace, size_t workspace_bytes, int32_t pairs_per_chunk, void* stream,
+                              void* h2d_stream, void* d2h_stream) {
+    sbsa_status r = check_shape(shape);
+    if (r != SBSA_OK) return r;
+    if ((r = check_k(shape, k_keep)) != SBSA_OK) return r;
+    if (!q_host || !k_host || !v_host || !o_host) return fail(SBSA_ERR_INVALID_ARG, "null host pointer");
+    if (!q || !k || !v || !o) return fail(SBSA_ERR_INVALID_ARG, "null device pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return fail(SBSA_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
+    if (!std::isfinite(scale)) return fail(SBSA_ERR_INVALID_ARG, "scale must be finite");
+    if (pairs_per_chunk < 0) return fail(SBSA_ERR_INVALID_ARG, "pairs_per_chunk must be >= 0");
+    const WsLayout w = ws_layout(shape, k_keep);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return fail(SBSA_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+    if (workspace_bytes < w.total)
+        return fail(SBSA_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes,
+                    w.total);
+    const int pairs = shape->batch * shape->heads;
+    const int n = pairs_per_chunk > 0 ? pairs_per_chunk : (pairs + 7) / 8;  // about eight chunks by default
+    const size_t pair_bytes = static_cast<size_t>(shape->seq_len_padded) * shape->head_dim * 2;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaStream_t s_in = h2d_stream ? static_cast<cudaStream_t>(h2d_stream) : st;
+    cudaStream_t s_out = d2h_stream ? static_cast<cudaStream_t>(d2h_stream) : st;
+    cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};  // start, copy-in done, chunk computed
+    for (auto& e : ev) {
+        cudaError_t ce = cudaEventCreateWithFlags(&e, cudaEventDisableTiming);
+        if (ce != cudaSuccess) {
+            for (auto& x : ev)
+                if (x) cudaEventDestroy(x);
+            return cuda_fail(ce, "event create");
+        }
+    }
+    auto finish = [&](sbsa_status res) {
+        for (auto& x : ev) cudaEventDestroy(x);  // released once their last record completes
+        return res;
+    };
+    cudaError_t e;
+    // the copies into q/k/v must wait for earlier work on `stream` that may still read them
+    if ((e = cudaEventRecord(ev[0], st)) != cudaSuccess) return finish(cuda_fail(e, "event record"));
+    if ((e = cudaStreamWaitEvent(s_in, ev[0], 0)) != cudaSuccess) return finish(cuda_fail(e, "stream wait"));
+    if ((e = cudaStreamWaitEvent(s_out, ev[0], 0)) != cudaSuccess) return finish(cuda_fail(e, "stream wait"));
+    const float sc = resolve_scale(shape, scale);
+    for (int c0 = 0; c0 < pairs; c0 += n) {
+        const int c1 = c0 + n < pairs ? c0 + n : pairs;
+        const size_t off = static_cast<size_t>(c0) * pair_bytes, bytes = static_cast<size_t>(c1 - c0) * pair_bytes;
+        // one copy per tensor and chunk (no batched-copy API)
+        const void* src[3] = {q_host, k_host, v_host};
+        void* dst[3] = {q, k, v};
+        for (int t = 0; t < 3; ++t) {
+            e = cudaMemcpyAsync(static_cast<uint8_t*>(dst[t]) + off, static_cast<const uint8_t*>(src[t]) + off, bytes,
+                                cudaMemcpyHostToDevice, s_in);
+            if (e != cudaSuccess) return finish(cuda_fail(e, "host-to-device copy"));
+        }
+        if ((e = cudaEventRecord(ev[1], s_in)) != cudaSuccess) return finish(cuda_fail(e, "event record"));
+        if ((e = cudaStreamWaitEvent(st, ev[1], 0)) != cudaSuccess) return finish(cuda_fail(e, "stream wait"));
+        // the chunk's (batch, head) pairs are a contiguous slab: one shape of c1 - c0 heads
+        sbsa_shape cs = *shape;
+        cs.batch = 1;
+        cs.heads = c1 - c0;
+        const WsLayout cw = ws_layout(&cs, k_keep);
+        uint8_t* ws = static_cast<uint8_t*>(workspace);
+        float* qm = reinterpret_cast<float*>(ws + cw.q_mean);
+        float* km = reinterpret_cast<float*>(ws + cw.k_mean);
+        int32_t* rp = reinterpret_cast<int32_t*>(ws + cw.row_ptr);
+        int32_t* ci = reinterpret_cast<int32_t*>(ws + cw.col_idx);
+        const uint8_t* cq = static_cast<const uint8_t*>(q) + off;
+        const uint8_t* ck = static_cast<const uint8_t*>(k) + off;
+        const uint8_t* cv = static_cast<const uint8_t*>(v) + off;
+        uint8_t* co = static_cast<uint8_t*>(o) + off;
+        if ((r = launch_pool(&cs, cq, ck, qm, km, st)) != SBSA_OK) return finish(r);
+        if ((r = launch_select(&cs, qm, km, k_keep, rp, ci, st)) != SBSA_OK) return finish(r);
+        if ((r = launch_attn(&cs, cq, ck, cv, rp, ci, sc, co, st)) != SBSA_OK) return finish(r);
+        if ((e = cudaEventRecord(ev[2], st)) != cudaSuccess) return finish(cuda_fail(e, "event record"));
+        if ((e = cudaStreamWaitEvent(s_out, ev[2], 0)) != cudaSuccess) return finish(cuda_fail(e, "stream wait"));
+        e = cudaMemcpyAsync(static_cast<uint8_t*>(o_host) + off, co, bytes, cudaMemcpyDeviceToHost, s_out);
+        if (e != cudaSuccess) return finish(cuda_fail(e, "device-to-host copy"));
+    }
+    // the caller's stream completes only after the last copy-out
+    if ((e = cudaEventRecord(ev[0], s_out)) != cudaSuccess) return finish(cuda_fail(e, "event record"));
+    if ((e = cudaStreamWaitEvent(st, ev[0], 0)) != cudaSuccess) return finish(cuda_fail(e, "stream wait"));
+    return finish(ok());
+}
+
 sbsa_status sbsa_forward_noalloc(const sbsa_shape* shape, const void* q, const void* k, const void* v,
                                  int32_t k_keep, float scale, void* o, int32_t* col_idx_out, void* stream) {
     sbsa_status r = check_shape(shape);
@@ -929,6 +1004,13 @@ sbsa_status sbsa_forward_noalloc(const sbsa_shape* shape, const void* q, const v
     if ((r = launch_pool(shape, q, k, qm, km, st)) != SBSA_OK) return r;
     if ((r = launch_select(shape, qm, km, k_keep, rp, ci, st)) != SBSA_OK) return r;
     if ((r = launch_attn(shape, q, k, v, rp, ci, resolve_scale(shape, scale), o, st)) != SBSA_OK) return r;
+    return ok();
+}
+
+sbsa_status sbsa_set_pipeline_wait_ns(uint64_t limit_ns) {
+    const unsigned long long v = limit_ns;
+    cudaError_t e = cudaMemcpyToSymbol(g_pipe_wait_ns, &v, sizeof v);
+    if (e != cudaSuccess) return cuda_fail(e, "set pipeline wait limit");
     return ok();
 }
 

@@ -206,10 +206,12 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ q
 // the transposed form S^T = Kmean . Qmean^T: M = 128 key blocks per tile (TMEM lane =
 // key block, column = query block), N = 32 query blocks, K = d = 128, kind::tf32.
 // fp32 accuracy from three products per K step: each mean x is split exactly into
-// x_t = x with its 13 low mantissa bits cleared (what the tensor core reads from a raw
-// fp32 operand: it truncates) and x_l = x - x_t; s = k_t.q_t + k_t.q_l + k_l.q_t drops
-// only k_l.q_l and the truncation of the small parts, about 2^-19 of |k||q| per product,
-// below the fp32 rounding of a 128-term sum.
+// x_t = x with its 13 low mantissa bits cleared (a value tf32 holds exactly) and
+// x_l = x - x_t; s = k_t.q_t + k_t.q_l + k_l.q_t drops only k_l.q_l and the tf32
+// rounding of the small parts, about 2^-19 of |k||q| per product, below the fp32
+// rounding of a 128-term sum.  Both parts are written into the operand buffers
+// explicitly (x_t over the raw means in place), so the result does not depend on how
+// the tensor core converts an fp32 operand that is not already a tf32 value.
 //
 // CTA = (b*h, 32 query blocks), 320 threads, two CTAs per SM:
 //   warp 8  : TMA of the raw means (box 32 channels x rows, 128-byte swizzle: the
@@ -218,7 +220,8 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ q
 //   warp 9  : TMEM allocation (256 columns: 8 key tiles x 32 query blocks) and the thread
 //             that issues the MMAs, 12 per chunk ((k_t,q_t), (k_t,q_l), (k_l,q_t) at 4 K
 //             steps).
-//   warps 0-7: write q_l once and k_l of every chunk (two buffers); then read the scores
+//   warps 0-7: split the Q tile once and every K chunk into (x_t in place, x_l in one of
+//             two buffers); then read the scores
 //             out of TMEM into shared memory as order-preserving keys, 16 query rows at a
 //             time, and run the warp-per-row top-k.
 constexpr int kSelTcRows = 32;                  // query blocks per CTA
@@ -248,10 +251,14 @@ __device__ __forceinline__ void umma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, u
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
-// x - (x with its 13 low mantissa bits cleared), for four floats
-__device__ __forceinline__ float4 tf32_low_part(float4 v) {
-    auto lo = [](float x) { return x - __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); };
-    return make_float4(lo(v.x), lo(v.y), lo(v.z), lo(v.w));
+// x with its 13 low mantissa bits cleared (exact in tf32), for four floats
+__device__ __forceinline__ float4 tf32_high_part(float4 v) {
+    auto hi = [](float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); };
+    return make_float4(hi(v.x), hi(v.y), hi(v.z), hi(v.w));
+}
+// x - (x with its 13 low mantissa bits cleared), exact, for four floats
+__device__ __forceinline__ float4 tf32_low_part(float4 v, float4 h) {
+    return make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
 }
 
 struct SelTcParams {
@@ -314,8 +321,9 @@ __global__ void __launch_bounds__(kSelTcThreads, 2) select_tc_kernel(const __gri
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const uint64_t pipe_limit = pipe_wait_ns();  // pipeline waits; the drain keeps kWaitLimitNs
     auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
-        if (mbar_wait_bounded(bar, parity, abort_flag, kWaitLimitNs)) return true;
+        if (mbar_wait_bounded(bar, parity, abort_flag, pipe_limit)) return true;
         if (!*abort_flag) {
             *abort_flag = 1;
             abort_launch(p.epoch);
@@ -384,7 +392,9 @@ __global__ void __launch_bounds__(kSelTcThreads, 2) select_tc_kernel(const __gri
             for (int u = 0; u < kSelTcQBytes / 16 / 256; ++u) {
                 const int f = tid + 256 * u;
                 const float4 v = reinterpret_cast<const float4*>(smem + kSelTcOffQ)[f];
-                reinterpret_cast<float4*>(smem + kSelTcOffQl)[f] = tf32_low_part(v);
+                const float4 h = tf32_high_part(v);
+                reinterpret_cast<float4*>(smem + kSelTcOffQ)[f] = h;
+                reinterpret_cast<float4*>(smem + kSelTcOffQl)[f] = tf32_low_part(v, h);
             }
         }
         fence_proxy_async_smem();
@@ -392,10 +402,17 @@ __global__ void __launch_bounds__(kSelTcThreads, 2) select_tc_kernel(const __gri
         for (int c = 0; ok && c < n_chunks; ++c) {
             const int b = c % S, lb = c & 1;
             if (!(ok = wait(&x_full[b], (c / S) & 1))) break;
+            // the raw chunk in slot b is read by no MMA before l_full[lb] below, so its
+            // high parts can be written over it in place
+            float4* xs = reinterpret_cast<float4*>(smem + kSelTcOffX + b * kSelTcTile);
             float4 v[kSelTcTile / 16 / 256];
 #pragma unroll
-            for (int u = 0; u < kSelTcTile / 16 / 256; ++u)
-                v[u] = tf32_low_part(reinterpret_cast<const float4*>(smem + kSelTcOffX + b * kSelTcTile)[tid + 256 * u]);
+            for (int u = 0; u < kSelTcTile / 16 / 256; ++u) {
+                const float4 x = xs[tid + 256 * u];
+                const float4 h = tf32_high_part(x);
+                xs[tid + 256 * u] = h;
+                v[u] = tf32_low_part(x, h);
+            }
             if (c >= 2 && !(ok = wait(&l_empty[lb], ((c - 2) >> 1) & 1))) break;
 #pragma unroll
             for (int u = 0; u < kSelTcTile / 16 / 256; ++u)

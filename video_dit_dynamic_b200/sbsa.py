@@ -27,7 +27,8 @@ EXPORTS = ("sbsa_version", "sbsa_status_string", "sbsa_last_error_message", "sbs
            "sbsa_attention_fwd_fp8", "sbsa_nvfp4_scale_bytes", "sbsa_nvfp4_amax", "sbsa_nvfp4_quantize",
            "sbsa_nvfp4_gemm", "sbsa_ulysses_qkv_bytes", "sbsa_ulysses_o_bytes", "sbsa_ulysses_pack_qkv",
            "sbsa_ulysses_unpack_qkv", "sbsa_ulysses_pack_o", "sbsa_ulysses_unpack_o", "sbsa_ulysses_put_qkv",
-           "sbsa_ulysses_put_o", "sbsa_peer_signal", "sbsa_peer_wait")
+           "sbsa_ulysses_put_o", "sbsa_peer_signal", "sbsa_peer_wait", "sbsa_forward_host",
+           "sbsa_set_pipeline_wait_ns")
 
 
 class SbsaError(RuntimeError):
@@ -91,6 +92,8 @@ def load(path: str | None = None):
     lib.sbsa_attention_fwd.argtypes = [SP, P, P, P, P, P, ctypes.c_float, P, P]
     lib.sbsa_forward.argtypes = [SP, P, P, P, I32, ctypes.c_float, P, P, P, SZ, P]
     lib.sbsa_forward_noalloc.argtypes = [SP, P, P, P, I32, ctypes.c_float, P, P, P]
+    lib.sbsa_forward_host.argtypes = [SP, P, P, P, I32, ctypes.c_float, P, P, P, P, P, P, SZ, I32, P, P, P]
+    lib.sbsa_set_pipeline_wait_ns.argtypes = [ctypes.c_uint64]
     lib.sbsa_check.argtypes = [P]
     lib.sbsa_validate_csr.argtypes = [SP, P, P, ctypes.c_int64, I32, P]
     lib.sbsa_rope_table_floats.argtypes = [I32, I32, I32, I32]
@@ -123,7 +126,8 @@ def load(path: str | None = None):
                  "sbsa_ulysses_put_qkv", "sbsa_ulysses_put_o", "sbsa_peer_signal", "sbsa_peer_wait"):
         getattr(lib, name).restype = ctypes.c_int
     for name in ("sbsa_pool_qk", "sbsa_select_blocks", "sbsa_attention_fwd", "sbsa_forward", "sbsa_check",
-                 "sbsa_validate_csr", "sbsa_forward_noalloc", "sbsa_rope_table_init", "sbsa_rope_pool_qk",
+                 "sbsa_validate_csr", "sbsa_forward_noalloc", "sbsa_forward_host", "sbsa_set_pipeline_wait_ns",
+                 "sbsa_rope_table_init", "sbsa_rope_pool_qk",
                  "sbsa_key_mean", "sbsa_quantize_qk_fp8", "sbsa_attention_fwd_fp8", "sbsa_nvfp4_amax",
                  "sbsa_nvfp4_quantize", "sbsa_nvfp4_gemm"):
         getattr(lib, name).restype = ctypes.c_int
@@ -470,17 +474,47 @@ def _side_streams(device):
     return _copy_streams[key]
 
 
+def _host(t: torch.Tensor, name: str) -> ctypes.c_void_p:
+    if t.device.type != "cpu" or t.dtype != torch.bfloat16 or not t.is_contiguous():
+        raise SbsaError(1, f"{name} must be a contiguous bf16 host tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def sbsa_forward_host(shape: Shape, q_host, k_host, v_host, k_keep: int, scale: float, o_host, q, k, v, o, workspace,
+                      pairs_per_chunk: int = 0, stream=None, h2d_stream=None, d2h_stream=None):
+    """pool -> select -> attend from host tensors through the device buffers q, k, v, o
+    (copies and kernels chunked over (batch, head) pairs on three streams)."""
+    n = shape.batch * shape.heads * shape.seq_len_padded * shape.head_dim
+    for t, nm in ((q_host, "q_host"), (k_host, "k_host"), (v_host, "v_host"), (o_host, "o_host")):
+        _check_numel(t, n, nm)
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _check_numel(t, n, nm)
+    st = load().sbsa_forward_host(ctypes.byref(shape), _host(q_host, "q_host"), _host(k_host, "k_host"),
+                                  _host(v_host, "v_host"), int(k_keep), float(scale), _host(o_host, "o_host"),
+                                  _dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"),
+                                  _dev(v, torch.bfloat16, "v"), _dev(o, torch.bfloat16, "o"),
+                                  _dev(workspace, torch.uint8, "workspace"), workspace.numel(), int(pairs_per_chunk),
+                                  _stream(stream),
+                                  # NULL copy streams: the copies run on `stream`
+                                  _stream(h2d_stream) if h2d_stream is not None else ctypes.c_void_p(0),
+                                  _stream(d2h_stream) if d2h_stream is not None else ctypes.c_void_p(0))
+    _raise_on(st)
+
+
+def sbsa_set_pipeline_wait_ns(limit_ns: int):
+    """Limit of the kernels' pipeline waits on the current device (1e9 by default; 0 drives
+    the give-up path in tests)."""
+    _raise_on(load().sbsa_set_pipeline_wait_ns(int(limit_ns)))
+
+
 def forward_from_host(shape: Shape, q_host, k_host, v_host, k_keep: int, scale: float = 0.0, *, o_host=None,
                       device_buffers=None, stream=None, head_chunk: int | None = None):
-    """End-to-end call from host tensors: copy Q/K/V (pinned host memory) to the device,
-    run sbsa_forward, copy O back.  ``device_buffers`` (q, k, v, o, workspace) may be
-    passed to reuse device memory across calls.  Returns the host output tensor.
-
-    The layer is processed in chunks of ``head_chunk`` (batch, head) pairs (every pair is
-    independent, so the result is the same as one call): the copy-in of a chunk, the
-    attention of the previous one and the copy-out of the one before overlap on three
-    streams.  Default: about eight chunks.  Asynchronous with respect to the host; the
-    work is complete once ``stream`` (default: the current stream) is."""
+    """End-to-end call from host tensors through sbsa_forward_host: Q/K/V copied in (from
+    pinned host memory), pool -> select -> attend, O copied out, chunked over (batch,
+    head) pairs so that copies and kernels overlap.  ``device_buffers`` (q, k, v, o,
+    workspace) may be passed to reuse device memory across calls.  Returns the host output
+    tensor.  Asynchronous with respect to the host; the work is complete once ``stream``
+    (default: the current stream) is."""
     s = stream or torch.cuda.current_stream()
     if device_buffers is None:
         dq = torch.empty(q_host.shape, dtype=torch.bfloat16, device="cuda")
@@ -490,26 +524,7 @@ def forward_from_host(shape: Shape, q_host, k_host, v_host, k_keep: int, scale: 
         dq, dk, dv, do, ws = device_buffers
     if o_host is None:
         o_host = torch.empty(do.shape, dtype=do.dtype, pin_memory=True)
-    pairs = shape.batch * shape.heads
-    n = head_chunk or max(1, -(-pairs // 8))
-    rows = shape.seq_len_padded * shape.head_dim  # elements per (batch, head)
-    flat = [t.reshape(pairs, rows) for t in (q_host, k_host, v_host, o_host, dq, dk, dv, do)]
-    qh, kh, vh, oh, fq, fk, fv, fo = flat
     h2d, d2h = _side_streams(dq.device)
-    # this call's copies must not overwrite buffers that earlier work on `s` or on the
-    # copy streams still uses
-    h2d.wait_stream(s)
-    s.wait_stream(d2h)
-    for c0 in range(0, pairs, n):
-        c1 = min(pairs, c0 + n)
-        with torch.cuda.stream(h2d):
-            for dst, src in ((fq, qh), (fk, kh), (fv, vh)):
-                dst[c0:c1].copy_(src[c0:c1], non_blocking=True)
-        s.wait_stream(h2d)
-        cs = make_shape(1, c1 - c0, shape.seq_len, shape.head_dim, shape.block_size, shape.seq_len_padded)
-        sbsa_forward(cs, fq[c0:c1], fk[c0:c1], fv[c0:c1], k_keep, scale, fo[c0:c1], None, ws, stream=s)
-        d2h.wait_stream(s)
-        with torch.cuda.stream(d2h):
-            oh[c0:c1].copy_(fo[c0:c1], non_blocking=True)
-    s.wait_stream(d2h)
+    sbsa_forward_host(shape, q_host, k_host, v_host, k_keep, scale, o_host, dq, dk, dv, do, ws,
+                      pairs_per_chunk=head_chunk or 0, stream=s, h2d_stream=h2d, d2h_stream=d2h)
     return o_host
