@@ -74,24 +74,36 @@ def test_attention_and_select_give_up_then_recover(sbsa):
     pu.assert_attention_close(o[:, :, :wl.seq_len], ref[:, :, :wl.seq_len], "after the give-up")
 
 
+def _flush_l2():
+    """Write a buffer larger than the 126 MB L2, so the next kernel reads from HBM."""
+    torch.empty(256 << 20, dtype=torch.uint8, device="cuda").fill_(1)
+    torch.cuda.synchronize()
+
+
 def test_rope_pool_and_fp8_quantizer_give_up_then_recover(sbsa):
-    wl, q, k, _ = _case()
-    s = sbsa.make_shape(1, wl.heads, wl.seq_len, wl.head_dim, wl.block)
-    nb, Lp, d = s.num_blocks, s.seq_len_padded, wl.head_dim
-    grid = (1, 60, 85)  # 5,100 tokens
+    # the 480p workload (40 heads, 21 x 30 x 52 tokens, 335 MB per tensor): with L2 flushed
+    # each CTA's tile comes from HBM, so its first test of the copy barrier finds it
+    # still in flight
+    wl = inputs.WORKLOADS["480p"]
+    q, k, _ = inputs.make_qkv(wl, seed=22, device="cuda")
+    grid, d, blk, H = wl.grid, wl.head_dim, wl.block, wl.heads
+    s = sbsa.make_shape(1, H, wl.seq_len, d, blk)
+    nb = s.num_blocks
     table = torch.empty(sbsa.sbsa_rope_table_floats(d, grid), dtype=torch.float32, device="cuda")
     sbsa.sbsa_rope_table_init(d, grid, 10000.0, table)
     qo, ko = torch.empty_like(q), torch.empty_like(k)
-    qm = torch.empty(wl.heads * nb * d, dtype=torch.float32, device="cuda")
+    qm = torch.empty(H * nb * d, dtype=torch.float32, device="cuda")
     km = torch.empty_like(qm)
     q8 = torch.empty(q.numel(), dtype=torch.uint8, device="cuda")
     k8 = torch.empty_like(q8)
-    qs = torch.empty(wl.heads * nb, dtype=torch.float32, device="cuda")
+    qs = torch.empty(H * nb, dtype=torch.float32, device="cuda")
     ks = torch.empty_like(qs)
     sbsa.sbsa_check()
     sbsa.sbsa_set_pipeline_wait_ns(0)
+    _flush_l2()
     sbsa.sbsa_rope_pool_qk(s, grid, table, q, k, qo, ko, qm, km)
     _expect_timeout(sbsa)
+    _flush_l2()
     sbsa.sbsa_quantize_qk_fp8(s, q, k, None, q8, k8, qs, ks)
     _expect_timeout(sbsa)
     sbsa.sbsa_set_pipeline_wait_ns(DEFAULT_LIMIT_NS)
@@ -99,15 +111,18 @@ def test_rope_pool_and_fp8_quantizer_give_up_then_recover(sbsa):
     sbsa.sbsa_quantize_qk_fp8(s, q, k, None, q8, k8, qs, ks)
     sbsa.sbsa_check()
     # the means are the means of the kernel's own rounded output, the rotation within the
-    # rope parity bound of the oracle's, and the FP8 codes and scales the oracle's
+    # rope parity bound of the oracle's (heads 0 and H-1), and the FP8 codes and scales
+    # the oracle's
     got = pu.bits(qo)
-    np.testing.assert_allclose(qm.cpu().double().numpy().reshape(1, wl.heads, nb, d),
-                               oracle.pool(got, wl.seq_len, wl.block), rtol=2e-6, atol=1e-6)
-    ref_bits, _ = oracle.rope_pool(pu.bits(q), grid, wl.seq_len, wl.block)
+    qin = pu.bits(q)
+    np.testing.assert_allclose(qm.cpu().double().numpy().reshape(1, H, nb, d),
+                               oracle.pool(got, wl.seq_len, blk), rtol=2e-6, atol=1e-6)
     to_f = lambda b: (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    g, r = to_f(got), to_f(ref_bits)
-    assert np.all(np.abs(g - r) <= np.maximum(np.abs(g), np.abs(r)) * 2.0 ** -7 + 1e-5)
-    qc, qsc = oracle.quantize_fp8(pu.bits(q), wl.seq_len, wl.block)
+    for h in (0, H - 1):
+        ref_bits, _ = oracle.rope_pool(qin[:, h:h + 1], grid, wl.seq_len, blk)
+        g, r = to_f(got[:, h:h + 1]), to_f(ref_bits)
+        assert np.all(np.abs(g - r) <= np.maximum(np.abs(g), np.abs(r)) * 2.0 ** -7 + 1e-5)
+    qc, qsc = oracle.quantize_fp8(qin, wl.seq_len, blk)
     np.testing.assert_array_equal(qs.cpu().numpy().reshape(qsc.shape), qsc)
     gc = q8.cpu().numpy().reshape(qc.shape)
     assert np.all((gc == qc) | (((gc & 0x7F) == 0) & ((qc & 0x7F) == 0)))

@@ -54,6 +54,14 @@
 #define SBSA_POLY_EXP2_EIGHTHS 2
 #endif
 
+// Issue order of the two MMA threads: with SBSA_ATTN_QK_AFTER_PV = m > 0 the thread that
+// issues S_j = Q K_j^T waits until O += P_{j-m} V_{j-m} has been issued, so that the
+// tensor pipe alternates between the two kinds and the two softmax warpgroups' blocks
+// are staggered; 0 lets the Q K^T thread run ahead as far as the S buffers allow.
+#ifndef SBSA_ATTN_QK_AFTER_PV
+#define SBSA_ATTN_QK_AFTER_PV 0
+#endif
+
 namespace sbsa {
 
 // Pairs (e, e+1) with e = 2 * (pair index); pair index mod 4 below EIGHTHS/2 use the polynomial.
@@ -114,8 +122,8 @@ struct AttnCfg {
     static constexpr int kVOff = kKOff + kStages * kKTile;
     static constexpr int kBarOff = kVOff + kStages * kVTile;
     // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2],
-    // s_free[2], p_full[2], pv_done[2], drain[2]
-    static constexpr int kNumBars = 1 + 4 * kStages + 2 * 5;
+    // s_free[2], p_full[2], pv_done[2], drain[2], pv_issued[4]
+    static constexpr int kNumBars = 1 + 4 * kStages + 2 * 5 + 4;
     static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // + tmem slot, flag, alignment slack
     static constexpr int kThreads = 352;
     static constexpr uint32_t kColS0 = 0, kColO0 = 256;  // S_b at b*128, O_g at 256 + g*128
@@ -183,12 +191,15 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
     uint64_t* p_full = s_free + 2;
     uint64_t* pv_done = p_full + 2;
     uint64_t* drain = pv_done + 2;
+    uint64_t* pv_issued = drain + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x;
     const int warp = tid / 32;
-    if (launch_aborted(p.epoch)) return;
+    // a CTA that starts after another one of its launch gave up returns at once; every
+    // thread takes the same branch (the barriers below need all of them)
+    if (__syncthreads_or(launch_aborted(p.epoch) ? 1 : 0)) return;
 
     const long long unit = blockIdx.x;
     const long long bh = unit / p.nb;
@@ -215,6 +226,7 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
             mbar_init(&pv_done[b], 1);
             mbar_init(&drain[b], 1);
         }
+        for (int b = 0; b < 4; ++b) mbar_init(&pv_issued[b], 1);
         fence_mbar_init();
         tma_prefetch_desc(&map_q);
         tma_prefetch_desc(&map_k);
@@ -304,6 +316,13 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                 const int b = j & 1;
                 if (!(ok = wait(&k_full[slot], (j / NS) & 1))) break;
                 if (j >= 2 && !(ok = wait(&s_free[b], ((j - 2) >> 1) & 1))) break;
+                if constexpr (SBSA_ATTN_QK_AFTER_PV > 0) {
+                    constexpr int m = SBSA_ATTN_QK_AFTER_PV;
+                    // PV_{j-m+4}, the next arrival on this barrier, needs QK_{j-m+4} (m <= 4):
+                    // the barrier is never a whole phase ahead of this wait
+                    static_assert(m <= 4, "pv_issued has four barriers");
+                    if (j >= m && !(ok = wait(&pv_issued[(j - m) & 3], ((j - m) >> 2) & 1))) break;
+                }
                 tc_fence_after();
                 const uint64_t kdesc0 = sdesc_sw128(k_addr + slot * C::kKTile, 16, 1024);
                 const uint32_t d_s = tmem + C::kColS0 + b * 128;
@@ -349,6 +368,7 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                 }
                 umma_commit(&v_empty[slot]);
                 umma_commit(&pv_done[b]);
+                if constexpr (SBSA_ATTN_QK_AFTER_PV > 0) mbar_arrive(&pv_issued[j & 3]);
             }
             if (!ok) {
                 umma_commit(&drain[1]);

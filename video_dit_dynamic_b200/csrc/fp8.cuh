@@ -83,8 +83,12 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint4* __restrict__
     for (int e = 0; e < 8; ++e) sm[e] = (is_k && k_smooth) ? __ldg(k_smooth + bh * D + 8 * c + e) : 0.f;
     __syncthreads();  // the barrier is initialised before anyone waits on it
     volatile int never = 0;
-    if (!mbar_wait_bounded(&full, 0, &never, pipe_wait_ns())) {
+    // every thread takes the same branch (the later __syncthreads need all of them), so
+    // the CTA gives up if any thread's wait ran out
+    const bool landed = mbar_wait_bounded(&full, 0, &never, pipe_wait_ns());
+    if (__syncthreads_or(landed ? 0 : 1)) {
         if (threadIdx.x == 0) abort_launch(epoch);
+        // the copy gets one more bounded wait to land before the shared memory is released
         mbar_wait_bounded(&full, 0, &never, kWaitLimitNs);
         return;
     }

@@ -252,7 +252,8 @@ __global__ void __launch_bounds__(kFp4Threads, 1) nvfp4_gemm_kernel(const __grid
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    if (launch_aborted(p.epoch)) return;
+    // every thread takes the same branch (the barriers below need all of them)
+    if (__syncthreads_or(launch_aborted(p.epoch) ? 1 : 0)) return;
     const int num_tiles = p.tiles_m * p.tiles_n;
     const int k_tiles = p.K / kFp4TileK;
 

@@ -147,9 +147,12 @@ __global__ void __launch_bounds__(256) rope_pool_kernel(const uint4* q_in, const
 
     __syncthreads();  // the barrier is initialised before anyone waits on it
     volatile int never = 0;
-    if (!mbar_wait_bounded(&full, 0, &never, pipe_wait_ns())) {
+    // every thread takes the same branch (the later __syncthreads need all of them), so
+    // the CTA gives up if any thread's wait ran out
+    const bool landed = mbar_wait_bounded(&full, 0, &never, pipe_wait_ns());
+    if (__syncthreads_or(landed ? 0 : 1)) {
         if (threadIdx.x == 0) abort_launch(epoch);
-        // give the copy one more bounded wait to land before the shared memory is released
+        // the copy gets one more bounded wait to land before the shared memory is released
         mbar_wait_bounded(&full, 0, &never, kWaitLimitNs);
         return;
     }

@@ -292,7 +292,8 @@ __global__ void __launch_bounds__(kSelTcThreads, 2) select_tc_kernel(const __gri
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem);  // [HALF][NBP], after the MMAs
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    if (launch_aborted(p.epoch)) return;
+    // every thread takes the same branch (the barriers below need all of them)
+    if (__syncthreads_or(launch_aborted(p.epoch) ? 1 : 0)) return;
     if (smem_u32(smem) & 1023u) {  // the swizzled operand layouts need 1024-byte alignment
         if (tid == 0) abort_launch(p.epoch);
         return;
