@@ -47,25 +47,43 @@
 #include "ptx.cuh"
 #include "tmem_wide.cuh"
 
-// Fraction of the probabilities (in eighths, even) computed with the FMA-pipe
+#include <type_traits>
+
+// Fraction of the probabilities (in eighths) computed with the FMA-pipe
 // polynomial instead of the MUFU ex2 unit; the two run in parallel, so moving some of
 // the work off the MUFU unit (16 results/clk/SM) shortens the softmax.
 #ifndef SBSA_POLY_EXP2_EIGHTHS
 #define SBSA_POLY_EXP2_EIGHTHS 2
 #endif
 
-// Issue order of the two MMA threads: with SBSA_ATTN_QK_AFTER_PV = m > 0 the thread that
-// issues S_j = Q K_j^T waits until O += P_{j-m} V_{j-m} has been issued, so that the
-// tensor pipe alternates between the two kinds and the two softmax warpgroups' blocks
-// are staggered; 0 lets the Q K^T thread run ahead as far as the S buffers allow.
+// Issue order of the two MMA threads: with m > 0 the thread that issues S_j = Q K_j^T
+// waits until O += P_{j-m} V_{j-m} has been issued, which holds the Q K^T thread back so
+// that the tensor pipe alternates more between the two kinds; 0 lets it run ahead as far
+// as the S buffers allow.  Measured (long-sequence and 480p layers): the bf16 form is
+// fastest with 0 (m = 2 and 3 slower); the FP8 form, whose Q K^T MMAs take half as
+// long, with 3 (12% fewer cycles than 0; m = 2 slower).
 #ifndef SBSA_ATTN_QK_AFTER_PV
 #define SBSA_ATTN_QK_AFTER_PV 0
+#endif
+#ifndef SBSA_ATTN_QK_AFTER_PV_FP8
+#define SBSA_ATTN_QK_AFTER_PV_FP8 3
+#endif
+
+// 1: each softmax warpgroup hands P_j over in two halves of 64 keys (block size 128), so
+// that O += P V over the first half runs while the second half's exponentials are
+// computed; 0: one hand-over per block.
+#ifndef SBSA_ATTN_PSPLIT
+#define SBSA_ATTN_PSPLIT 0
+#endif
+// 1: the block max as a depth-5 tree of three-input maxima; 0: eight chains.
+#ifndef SBSA_ATTN_MAXTREE
+#define SBSA_ATTN_MAXTREE 0
 #endif
 
 namespace sbsa {
 
-// Pairs (e, e+1) with e = 2 * (pair index); pair index mod 4 below EIGHTHS/2 use the polynomial.
-__host__ __device__ constexpr bool kPolyPair(int e) { return ((e >> 1) & 3) < SBSA_POLY_EXP2_EIGHTHS / 2; }
+// Pairs (e, e+1) with e = 2 * (pair index); pair index mod 8 below EIGHTHS use the polynomial.
+__host__ __device__ constexpr bool kPolyPair(int e) { return ((e >> 1) & 7) < SBSA_POLY_EXP2_EIGHTHS; }
 
 // 2^x on the FMA pipe for a pair, x <= 8 (x >= -125 after the clamp; smaller x give
 // ~2^-125).  Cody-Waite style split x = n + f with n = rint(x) (the 1.5*2^23 rounding
@@ -122,8 +140,8 @@ struct AttnCfg {
     static constexpr int kVOff = kKOff + kStages * kKTile;
     static constexpr int kBarOff = kVOff + kStages * kVTile;
     // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2],
-    // s_free[2], p_full[2], pv_done[2], drain[2], pv_issued[4]
-    static constexpr int kNumBars = 1 + 4 * kStages + 2 * 5 + 4;
+    // s_free[2], p_full[2], pv_done[2], drain[2], pv_issued[4], p_half[2]
+    static constexpr int kNumBars = 1 + 4 * kStages + 2 * 5 + 4 + 2;
     static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // + tmem slot, flag, alignment slack
     static constexpr int kThreads = 352;
     static constexpr uint32_t kColS0 = 0, kColO0 = 256;  // S_b at b*128, O_g at 256 + g*128
@@ -173,6 +191,7 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                                                       const AttnParams p) {
     using C = AttnCfg<D, BLK, FP8>;
     constexpr int NS = C::kStages;
+    constexpr int kQkAfterPv = FP8 ? SBSA_ATTN_QK_AFTER_PV_FP8 : SBSA_ATTN_QK_AFTER_PV;
     constexpr int HD = D / 2;    // output columns each warpgroup writes in the merge
     extern __shared__ __align__(1024) uint8_t attn_smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(attn_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -192,6 +211,7 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
     uint64_t* pv_done = p_full + 2;
     uint64_t* drain = pv_done + 2;
     uint64_t* pv_issued = drain + 2;
+    uint64_t* p_half = pv_issued + 4;  // first 64 keys of P_j stored (split hand-over)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -227,6 +247,7 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
             mbar_init(&drain[b], 1);
         }
         for (int b = 0; b < 4; ++b) mbar_init(&pv_issued[b], 1);
+        for (int b = 0; b < 2; ++b) mbar_init(&p_half[b], 128);
         fence_mbar_init();
         tma_prefetch_desc(&map_q);
         tma_prefetch_desc(&map_k);
@@ -316,8 +337,8 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                 const int b = j & 1;
                 if (!(ok = wait(&k_full[slot], (j / NS) & 1))) break;
                 if (j >= 2 && !(ok = wait(&s_free[b], ((j - 2) >> 1) & 1))) break;
-                if constexpr (SBSA_ATTN_QK_AFTER_PV > 0) {
-                    constexpr int m = SBSA_ATTN_QK_AFTER_PV;
+                if constexpr (kQkAfterPv > 0) {
+                    constexpr int m = kQkAfterPv;
                     // PV_{j-m+4}, the next arrival on this barrier, needs QK_{j-m+4} (m <= 4):
                     // the barrier is never a whole phase ahead of this wait
                     static_assert(m <= 4, "pv_issued has four barriers");
@@ -347,6 +368,7 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
     } else if (warp == 10) {
         // ------------------------------------------------------------ PV issuer
         if ((tid & 31) == 0 && n > 0) {
+            constexpr bool kPSplit = SBSA_ATTN_PSPLIT && BLK == 128;
             constexpr uint32_t idO = idesc_bf16_f32(128, D, true);
             const uint32_t v_addr = smem_u32(sV);
             const uint64_t pdesc0 = sdesc_sw128(smem_u32(sP), 16, 1024);
@@ -355,20 +377,26 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                 const int slot = j % NS;
                 const int b = j & 1;
                 if (!(ok = wait(&v_full[slot], (j / NS) & 1))) break;
-                if (!(ok = wait(&p_full[b], (j >> 1) & 1))) break;
+                if (!(ok = wait(kPSplit ? &p_half[b] : &p_full[b], (j >> 1) & 1))) break;
                 tc_fence_after();
                 const uint64_t vdesc0 = sdesc_sw128(v_addr + slot * C::kVTile, BLK * 128, 1024);
                 const uint64_t pdesc = pdesc0 + static_cast<uint64_t>((b * C::kPBytes) >> 4);
                 const uint32_t d_o = tmem + C::kColO0 + b * 128;
 #pragma unroll
                 for (int kk = 0; kk < BLK / 16; ++kk) {
+                    if (kPSplit && kk == BLK / 32) {
+                        // the second half of P_j
+                        if (!(ok = wait(&p_full[b], (j >> 1) & 1))) break;
+                        tc_fence_after();
+                    }
                     const uint64_t da = pdesc + static_cast<uint64_t>(((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4);
                     const uint64_t db = vdesc0 + static_cast<uint64_t>((kk * 16 * 128) >> 4);
                     umma_ss(d_o, da, db, idO, (j > 1 || kk > 0) ? 1u : 0u);
                 }
+                if (!ok) break;
                 umma_commit(&v_empty[slot]);
                 umma_commit(&pv_done[b]);
-                if constexpr (SBSA_ATTN_QK_AFTER_PV > 0) mbar_arrive(&pv_issued[j & 3]);
+                if constexpr (kQkAfterPv > 0) mbar_arrive(&pv_issued[j & 3]);
             }
             if (!ok) {
                 umma_commit(&drain[1]);
@@ -444,16 +472,41 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                 for (int e = 0; e < BLK; ++e)
                     if (e >= nvalid) s[e] = -INFINITY;
             }
-            // block max: eight independent chains of three-input maxima, then a tree
-            float mx8[8];
+            float mx;
+#if SBSA_ATTN_MAXTREE
+            {
+                // block max as a tree of three-input maxima (depth 5)
+                float t1[(BLK + 2) / 3];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) mx8[c] = fmaxf(s[c], s[c + 8]);
+                for (int c = 0; c < BLK / 3; ++c) t1[c] = fmax3(s[3 * c], s[3 * c + 1], s[3 * c + 2]);
+                if constexpr (BLK % 3 == 1) t1[BLK / 3] = s[BLK - 1];
+                if constexpr (BLK % 3 == 2) t1[BLK / 3] = fmaxf(s[BLK - 2], s[BLK - 1]);
+                constexpr int N1 = (BLK + 2) / 3;
+                float t2[(N1 + 2) / 3];
 #pragma unroll
-            for (int e = 16; e < BLK; e += 16)
+                for (int c = 0; c < N1 / 3; ++c) t2[c] = fmax3(t1[3 * c], t1[3 * c + 1], t1[3 * c + 2]);
+                if constexpr (N1 % 3 == 1) t2[N1 / 3] = t1[N1 - 1];
+                if constexpr (N1 % 3 == 2) t2[N1 / 3] = fmaxf(t1[N1 - 2], t1[N1 - 1]);
+                constexpr int N2 = (N1 + 2) / 3;
+                float r = t2[0];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) mx8[c] = fmax3(mx8[c], s[e + c], s[e + 8 + c]);
-            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;
+                for (int c = 1; c < N2; ++c) r = fmaxf(r, t2[c]);
+                mx = r * sl2;
+            }
+#else
+            {
+                // block max: eight independent chains of three-input maxima, then a tree
+                float mx8[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) mx8[c] = fmaxf(s[c], s[c + 8]);
+#pragma unroll
+                for (int e = 16; e < BLK; e += 16)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) mx8[c] = fmax3(mx8[c], s[e + c], s[e + 8 + c]);
+                mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;
+            }
+#endif
             // Lazy rescaling: keep the old reference max unless the block's max exceeds
             // it by more than 8 (values up to 2^8 are safe in bf16 P and fp32 O / l).
             float alpha = 1.f;
@@ -466,62 +519,99 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
             float2 sum4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                               make_float2(0.f, 0.f)};
             uint32_t pk[BLK / 2];
-            if (!masked) {
+            // P for keys [E0, E1): exp2(S * sl2 - m) in fp32, summed, packed to bf16 pairs
+            auto exps = [&](auto e0_tag, auto e1_tag) {
+                constexpr int E0 = decltype(e0_tag)::value, E1 = decltype(e1_tag)::value;
+                if (!masked) {
 #pragma unroll
-                for (int e = 0; e < BLK; e += 2) {
-                    const float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), sl2x2, nm2);
-                    float2 pr;
-                    if (kPolyPair(e)) {
-                        pr = exp2_poly2(x);
-                    } else {
+                    for (int e = E0; e < E1; e += 2) {
+                        const float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), sl2x2, nm2);
+                        float2 pr;
+                        if (kPolyPair(e)) {
+                            pr = exp2_poly2(x);
+                        } else {
+                            pr.x = ex2_approx(x.x);
+                            pr.y = ex2_approx(x.y);
+                        }
+                        sum4[(e >> 1) & 3] = __fadd2_rn(sum4[(e >> 1) & 3], pr);
+                        pk[e / 2] = pack_bf16x2(pr.x, pr.y);
+                    }
+                } else {
+                    // masked entries are -inf: ex2 gives exactly 0 (the polynomial would not)
+#pragma unroll
+                    for (int e = E0; e < E1; e += 2) {
+                        const float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), sl2x2, nm2);
+                        float2 pr;
                         pr.x = ex2_approx(x.x);
                         pr.y = ex2_approx(x.y);
+                        sum4[(e >> 1) & 3] = __fadd2_rn(sum4[(e >> 1) & 3], pr);
+                        pk[e / 2] = pack_bf16x2(pr.x, pr.y);
                     }
-                    sum4[(e >> 1) & 3] = __fadd2_rn(sum4[(e >> 1) & 3], pr);
-                    pk[e / 2] = pack_bf16x2(pr.x, pr.y);
                 }
-            } else {
-                // masked entries are -inf: ex2 gives exactly 0 (the polynomial would not)
+            };
+            // P_j's 16-byte chunks [C0, C1) into P buffer g (128-byte rows, one 16 KB region per 64 keys)
+            auto store_p = [&](auto c0_tag, auto c1_tag) {
+                constexpr int C0 = decltype(c0_tag)::value, C1 = decltype(c1_tag)::value;
 #pragma unroll
-                for (int e = 0; e < BLK; e += 2) {
-                    const float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), sl2x2, nm2);
-                    float2 pr;
-                    pr.x = ex2_approx(x.x);
-                    pr.y = ex2_approx(x.y);
-                    sum4[(e >> 1) & 3] = __fadd2_rn(sum4[(e >> 1) & 3], pr);
-                    pk[e / 2] = pack_bf16x2(pr.x, pr.y);
+                for (int c = C0; c < C1; ++c) {
+                    const uint32_t addr = p_row + (c / 8) * (128 * 128) + ((static_cast<uint32_t>(c & 7) ^ p_swz) << 4);
+                    st_shared_v4(addr, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
                 }
+            };
+            // O_g *= alpha when the reference max moved (PV_{j-2} is done)
+            auto rescale_o = [&]() {
+                if (j > 1 && __any_sync(0xFFFFFFFFu, alpha != 1.f)) {
+                    const float2 a2 = make_float2(alpha, alpha);
+                    // 32 columns at a time: few registers next to the live S and P values
+#pragma unroll 1
+                    for (int h = 0; h < D; h += 32) {
+                        uint32_t ov[32];
+                        tmem_ld_cols<32>(o_col + h, ov);
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const float2 v = __fmul2_rn(make_float2(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1])), a2);
+                            ov[e] = __float_as_uint(v.x);
+                            ov[e + 1] = __float_as_uint(v.y);
+                        }
+                        tmem_st_cols<32>(o_col + h, ov);
+                    }
+                    tmem_st_wait();
+                }
+            };
+            using I0 = std::integral_constant<int, 0>;
+            using IH = std::integral_constant<int, BLK / 2>;
+            using IB = std::integral_constant<int, BLK>;
+            using C0 = std::integral_constant<int, 0>;
+            using CH = std::integral_constant<int, BLK / 16>;
+            using CB = std::integral_constant<int, BLK / 8>;
+            if constexpr (SBSA_ATTN_PSPLIT && BLK == 128) {
+                exps(I0{}, IH{});
+                // PV_{j-2} must be done before P buffer g is overwritten or O_g rescaled
+                if (j >= 2) {
+                    ok = wait_warp(&pv_done[g], ((j - 2) >> 1) & 1);
+                    if (!ok) continue;
+                }
+                rescale_o();
+                store_p(C0{}, CH{});
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&p_half[g]);
+                exps(IH{}, IB{});
+                store_p(CH{}, CB{});
+            } else {
+                exps(I0{}, IB{});
+                // PV_{j-2} must be done before P buffer g is overwritten or O_g rescaled
+                if (j >= 2) {
+                    ok = wait_warp(&pv_done[g], ((j - 2) >> 1) & 1);
+                    if (!ok) continue;
+                }
+                store_p(C0{}, CB{});
+                rescale_o();
             }
             const float2 s01 = __fadd2_rn(sum4[0], sum4[1]);
             const float2 s23 = __fadd2_rn(sum4[2], sum4[3]);
             const float2 sall = __fadd2_rn(s01, s23);
             l = l * alpha + (sall.x + sall.y);
-            // PV_{j-2} must be done before P buffer g is overwritten or O_g rescaled
-            if (j >= 2) {
-                ok = wait_warp(&pv_done[g], ((j - 2) >> 1) & 1);
-                if (!ok) continue;
-            }
-#pragma unroll
-            for (int c = 0; c < BLK / 8; ++c) {
-                const uint32_t addr = p_row + (c / 8) * (128 * 128) + ((static_cast<uint32_t>(c & 7) ^ p_swz) << 4);
-                st_shared_v4(addr, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-            }
-            if (j > 1 && __any_sync(0xFFFFFFFFu, alpha != 1.f)) {
-                const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-                for (int h = 0; h < D; h += 64) {
-                    uint32_t ov[D < 64 ? D : 64];
-                    tmem_ld_cols<(D < 64 ? D : 64)>(o_col + h, ov);
-#pragma unroll
-                    for (int e = 0; e < (D < 64 ? D : 64); e += 2) {
-                        const float2 v = __fmul2_rn(make_float2(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1])), a2);
-                        ov[e] = __float_as_uint(v.x);
-                        ov[e + 1] = __float_as_uint(v.y);
-                    }
-                    tmem_st_cols<(D < 64 ? D : 64)>(o_col + h, ov);
-                }
-                tmem_st_wait();
-            }
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&p_full[g]);

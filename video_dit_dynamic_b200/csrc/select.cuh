@@ -14,10 +14,13 @@
 //     product with the QT query means broadcast from shared memory.
 // Scores go to shared memory as order-preserving uint32 keys.  Top-k: one warp per
 // query row, lane l holding keys j = l + 32 r; the (k-1)-th largest key T comes from a
-// search with warp-wide counts; keys > T are kept, and keys == T in ascending j until
-// k-1 are kept; the output position of each kept j is a ballot prefix count, which
-// yields the ascending order directly.
+// search with warp-wide counts, starting at the threshold of the warp's previous
+// (neighbouring) row; keys > T are kept, and keys == T in ascending j until k-1 are
+// kept; the keep bits are transposed with ballots into one 32-block word per lane, and a
+// prefix sum of the words' counts places every kept j in ascending order.
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -31,12 +34,15 @@ __device__ __forceinline__ uint32_t order_key(float s) {
 
 // Keep, for query block i, the diagonal and the k_keep-1 largest of the other keys
 // (ties: lower j), writing them in ascending j.  One warp; lane l holds keys
-// j = l + 32 s.  keys_row (shared memory, this row only) is reused as staging space
-// for the output list.
+// j = l + 32 s.  `hint` carries the threshold key found for the warp's previous row (0
+// for none): rows handled one after the other by a warp are neighbouring query blocks,
+// whose score rows are alike, so it is tried as the first probe.
 template <int KPL>
-__device__ __forceinline__ void select_row_topk(uint32_t* __restrict__ keys_row, int nb, int i, int k_keep,
+__device__ __forceinline__ void select_row_topk(const uint32_t* __restrict__ keys_row, int nb, int i, int k_keep,
                                                 long long row, int32_t* __restrict__ row_ptr,
-                                                int32_t* __restrict__ col_idx) {
+                                                int32_t* __restrict__ col_idx, uint32_t& hint) {
+    static_assert(KPL <= 64, "at most two output words per lane");
+    using Mask = typename std::conditional<(KPL > 32), unsigned long long, uint32_t>::type;
     const int lane = threadIdx.x % 32;
     const uint32_t lt = lanemask_lt();
     const int kk = k_keep - 1;  // off-diagonal blocks to keep
@@ -50,12 +56,13 @@ __device__ __forceinline__ void select_row_topk(uint32_t* __restrict__ keys_row,
         key[s] = (j < nb && j != i) ? max(keys_row[j], 1u) : 0u;
     }
     // The (k-1)-th largest candidate key T: a search over the key range [lo, hi) with
-    // count(key >= lo) >= k-1 > count(key >= hi).  Each probe is placed where the
-    // counts at the two ends put it if the keys were spread evenly in between
-    // (interpolation), with a halving probe after any interpolation that did not at
-    // least halve the range, so the search never takes more than twice the 33 steps
-    // of plain bisection.  It stops early when exactly k-1 keys are >= the probe
-    // ("exact": then no key needs a tie decision).
+    // count(key >= lo) >= k-1 > count(key >= hi).  The first probe is the hint when it
+    // lies inside the range; then each probe is placed where the counts at the two ends
+    // put it if the keys were spread evenly in between (interpolation), with a halving
+    // probe after any interpolation that did not at least halve the range, so the search
+    // never takes more than twice the 33 steps of plain bisection (plus the hint).  It
+    // stops early when exactly k-1 keys are >= the probe ("exact": then no key needs a
+    // tie decision).
     uint32_t T = 0u;
     bool exact = kk == 0;
     if (kk > 0) {
@@ -76,19 +83,26 @@ __device__ __forceinline__ void select_row_topk(uint32_t* __restrict__ keys_row,
         int c_lo = __reduce_add_sync(0xFFFFFFFFu, nc);  // candidates: count(key >= lo)
         int c_hi = 0;
         bool halve = false;
+        bool use_hint = hint > lo && hint < hi;
         T = lo;
 #pragma unroll 1
-        for (int it = 0; it < 72 && hi - lo > 1u; ++it) {
+        for (int it = 0; it < 73 && hi - lo > 1u; ++it) {
             const uint32_t range = hi - lo;
-            uint32_t off;
-            if (halve) {
-                off = range >> 1;
+            uint32_t cand;
+            if (use_hint) {
+                cand = hint;
+                use_hint = false;
             } else {
-                const float f = __fdividef(static_cast<float>(c_lo - kk), static_cast<float>(c_lo - c_hi));
-                off = static_cast<uint32_t>(f * static_cast<float>(range));
+                uint32_t off;
+                if (halve) {
+                    off = range >> 1;
+                } else {
+                    const float f = __fdividef(static_cast<float>(c_lo - kk), static_cast<float>(c_lo - c_hi));
+                    off = static_cast<uint32_t>(f * static_cast<float>(range));
+                }
+                off = min(max(off, 1u), range - 1u);
+                cand = lo + off;
             }
-            off = min(max(off, 1u), range - 1u);
-            const uint32_t cand = lo + off;
             // four independent partial counts keep the add chains short
             int c4[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -109,44 +123,71 @@ __device__ __forceinline__ void select_row_topk(uint32_t* __restrict__ keys_row,
             T = lo;
             halve = !halve && 2ull * (hi - lo) > range;
         }
+        hint = T;
     }
-    // Keys equal to T are kept lowest j first until k-1 are kept (only needed when the
-    // search ended on a key value with ties possible).
-    int need_eq = 0;
-    if (!exact) {
+    // Keep bits of this lane's slots (bit s: j = s*32 + lane).  Keys equal to T are kept
+    // lowest j first until k-1 are kept (only needed when the search ended on a key value
+    // with ties possible).
+    Mask mask = 0u;
+    if (exact) {
+#pragma unroll
+        for (int s = 0; s < KPL; ++s) {
+            const int j = s * 32 + lane;
+            const bool keep = (j == i) || (kk > 0 && key[s] != 0u && key[s] >= T);
+            mask |= keep ? (Mask(1) << s) : Mask(0);
+        }
+    } else {
         int g4[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int s = 0; s < KPL; ++s) g4[s & 3] += key[s] > T ? 1 : 0;
-        need_eq = kk - __reduce_add_sync(0xFFFFFFFFu, (g4[0] + g4[1]) + (g4[2] + g4[3]));
-    }
-    // The kept j in ascending order: ballot prefix counts give each its position in a
-    // staging list over this row's own key buffer (every lane has read its keys), which
-    // then goes out with coalesced stores.
-    __syncwarp();
-    int32_t* stage = reinterpret_cast<int32_t*>(keys_row);
-    int pos = 0, eq_seen = 0;
+        const int need_eq = kk - __reduce_add_sync(0xFFFFFFFFu, (g4[0] + g4[1]) + (g4[2] + g4[3]));
+        int eq_seen = 0;
 #pragma unroll
-    for (int s = 0; s < KPL; ++s) {
-        const int j = s * 32 + lane;
-        const bool cand = key[s] != 0u;  // j < nb and j != i
-        bool keep;
-        if (exact) {
-            keep = (j == i) || (kk > 0 && cand && key[s] >= T);
-        } else {
+        for (int s = 0; s < KPL; ++s) {
+            const int j = s * 32 + lane;
+            const bool cand = key[s] != 0u;  // j < nb and j != i
             const bool is_eq = cand && key[s] == T;
             const uint32_t eq_mask = __ballot_sync(0xFFFFFFFFu, is_eq);
-            keep = (j == i) || (cand && key[s] > T) || (is_eq && eq_seen + __popc(eq_mask & lt) < need_eq);
+            const bool keep = (j == i) || (cand && key[s] > T) || (is_eq && eq_seen + __popc(eq_mask & lt) < need_eq);
             eq_seen += __popc(eq_mask);
+            mask |= keep ? (Mask(1) << s) : Mask(0);
         }
-        const uint32_t m = __ballot_sync(0xFFFFFFFFu, keep);
-        if (keep) stage[pos + __popc(m & lt)] = j;
-        pos += __popc(m);
     }
-    __syncwarp();
+    // Transpose the keep bits: lane w gathers word w (and w + 32 when KPL > 32), whose bit
+    // l is slot w of lane l, i.e. block j = 32 w + l.  Ascending j is then ascending word,
+    // then ascending bit: a prefix sum of the words' counts gives each lane where its
+    // blocks go.
+    constexpr int NW = (KPL + 31) / 32;
+    uint32_t word[NW];
+#pragma unroll
+    for (int w = 0; w < NW; ++w) word[w] = 0u;
+#pragma unroll
+    for (int s = 0; s < KPL; ++s) {
+        const uint32_t b = __ballot_sync(0xFFFFFFFFu, static_cast<uint32_t>(mask >> s) & 1u);
+        word[s / 32] = lane == (s % 32) ? b : word[s / 32];
+    }
     int32_t* out = col_idx + row * k_keep;
-    for (int e = lane; e < k_keep; e += 32) out[e] = stage[e];
+    int base = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+        const int cnt = __popc(word[w]);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        int pos = base + incl - cnt;
+        uint32_t bits = word[w];
+        while (bits) {
+            const int b = __ffs(static_cast<int>(bits)) - 1;
+            out[pos++] = 32 * (32 * w + lane) + b;
+            bits &= bits - 1u;
+        }
+        base += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
     if (lane == 0) row_ptr[row] = static_cast<int32_t>(row * k_keep);
-    __syncwarp();  // the staging area is reused by the caller
+    __syncwarp();
 }
 
 template <int D, int QT, int KPL>
@@ -194,10 +235,16 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ q
     }
     __syncthreads();
 
-    // ---- top-k per row, one warp per row
+    // ---- top-k per row, one warp per row; each warp takes neighbouring rows
     const int warp = threadIdx.x / 32;
-    for (int r = warp; r < nq; r += blockDim.x / 32)
-        select_row_topk<KPL>(keys + r * NBP, nb, i0 + r, k_keep, bh * nb + i0 + r, row_ptr, col_idx);
+    constexpr int kRowsPerWarp = QT / 8;
+    static_assert(QT % 8 == 0, "eight warps share the rows");
+    uint32_t hint = 0u;
+#pragma unroll 1
+    for (int q = 0; q < kRowsPerWarp; ++q) {
+        const int r = warp * kRowsPerWarp + q;
+        if (r < nq) select_row_topk<KPL>(keys + r * NBP, nb, i0 + r, k_keep, bh * nb + i0 + r, row_ptr, col_idx, hint);
+    }
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) row_ptr[n_rows] = static_cast<int32_t>(n_rows * k_keep);
 }
 
@@ -429,6 +476,7 @@ __global__ void __launch_bounds__(kSelTcThreads, 2) select_tc_kernel(const __gri
     tc_fence_after();
     if (ok && warp < 8) {
         const int q4 = warp & 3;  // TMEM lane quarter of this warp
+        uint32_t hint = 0u;       // threshold key of this warp's previous row
         for (int round = 0; round < 2; ++round) {
             const int r0 = round * HALF;
             if (r0 < nq) {
@@ -444,8 +492,14 @@ __global__ void __launch_bounds__(kSelTcThreads, 2) select_tc_kernel(const __gri
                 }
             }
             asm volatile("bar.sync 1, 256;" ::: "memory");
-            for (int r = r0 + warp; r < min(nq, r0 + HALF); r += 8)
-                select_row_topk<KPL>(keys + (r - r0) * NBP, nb, i0 + r, p.k_keep, bh * nb + i0 + r, row_ptr, col_idx);
+            // each warp takes neighbouring rows (the threshold of one is the first probe of the next)
+#pragma unroll 1
+            for (int q = 0; q < HALF / 8; ++q) {
+                const int r = r0 + warp * (HALF / 8) + q;
+                if (r < nq)
+                    select_row_topk<KPL>(keys + (r - r0) * NBP, nb, i0 + r, p.k_keep, bh * nb + i0 + r, row_ptr,
+                                         col_idx, hint);
+            }
             asm volatile("bar.sync 1, 256;" ::: "memory");
         }
     }
