@@ -69,16 +69,6 @@
 #define SBSA_ATTN_QK_AFTER_PV_FP8 3
 #endif
 
-// 1: each softmax warpgroup hands P_j over in two halves of 64 keys (block size 128), so
-// that O += P V over the first half runs while the second half's exponentials are
-// computed; 0: one hand-over per block.
-#ifndef SBSA_ATTN_PSPLIT
-#define SBSA_ATTN_PSPLIT 0
-#endif
-// 1: the block max as a depth-5 tree of three-input maxima; 0: eight chains.
-#ifndef SBSA_ATTN_MAXTREE
-#define SBSA_ATTN_MAXTREE 0
-#endif
 
 namespace sbsa {
 
@@ -140,8 +130,8 @@ struct AttnCfg {
     static constexpr int kVOff = kKOff + kStages * kKTile;
     static constexpr int kBarOff = kVOff + kStages * kVTile;
     // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2],
-    // s_free[2], p_full[2], pv_done[2], drain[2], pv_issued[4], p_half[2]
-    static constexpr int kNumBars = 1 + 4 * kStages + 2 * 5 + 4 + 2;
+    // s_free[2], p_full[2], pv_done[2], drain[2], pv_issued[4]
+    static constexpr int kNumBars = 1 + 4 * kStages + 2 * 5 + 4;
     static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // + tmem slot, flag, alignment slack
     static constexpr int kThreads = 352;
     static constexpr uint32_t kColS0 = 0, kColO0 = 256;  // S_b at b*128, O_g at 256 + g*128
@@ -211,7 +201,6 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
     uint64_t* pv_done = p_full + 2;
     uint64_t* drain = pv_done + 2;
     uint64_t* pv_issued = drain + 2;
-    uint64_t* p_half = pv_issued + 4;  // first 64 keys of P_j stored (split hand-over)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -247,7 +236,6 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
             mbar_init(&drain[b], 1);
         }
         for (int b = 0; b < 4; ++b) mbar_init(&pv_issued[b], 1);
-        for (int b = 0; b < 2; ++b) mbar_init(&p_half[b], 128);
         fence_mbar_init();
         tma_prefetch_desc(&map_q);
         tma_prefetch_desc(&map_k);
@@ -368,7 +356,6 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
     } else if (warp == 10) {
         // ------------------------------------------------------------ PV issuer
         if ((tid & 31) == 0 && n > 0) {
-            constexpr bool kPSplit = SBSA_ATTN_PSPLIT && BLK == 128;
             constexpr uint32_t idO = idesc_bf16_f32(128, D, true);
             const uint32_t v_addr = smem_u32(sV);
             const uint64_t pdesc0 = sdesc_sw128(smem_u32(sP), 16, 1024);
@@ -377,23 +364,17 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                 const int slot = j % NS;
                 const int b = j & 1;
                 if (!(ok = wait(&v_full[slot], (j / NS) & 1))) break;
-                if (!(ok = wait(kPSplit ? &p_half[b] : &p_full[b], (j >> 1) & 1))) break;
+                if (!(ok = wait(&p_full[b], (j >> 1) & 1))) break;
                 tc_fence_after();
                 const uint64_t vdesc0 = sdesc_sw128(v_addr + slot * C::kVTile, BLK * 128, 1024);
                 const uint64_t pdesc = pdesc0 + static_cast<uint64_t>((b * C::kPBytes) >> 4);
                 const uint32_t d_o = tmem + C::kColO0 + b * 128;
 #pragma unroll
                 for (int kk = 0; kk < BLK / 16; ++kk) {
-                    if (kPSplit && kk == BLK / 32) {
-                        // the second half of P_j
-                        if (!(ok = wait(&p_full[b], (j >> 1) & 1))) break;
-                        tc_fence_after();
-                    }
                     const uint64_t da = pdesc + static_cast<uint64_t>(((kk / 4) * (128 * 128) + (kk % 4) * 32) >> 4);
                     const uint64_t db = vdesc0 + static_cast<uint64_t>((kk * 16 * 128) >> 4);
                     umma_ss(d_o, da, db, idO, (j > 1 || kk > 0) ? 1u : 0u);
                 }
-                if (!ok) break;
                 umma_commit(&v_empty[slot]);
                 umma_commit(&pv_done[b]);
                 if constexpr (kQkAfterPv > 0) mbar_arrive(&pv_issued[j & 3]);
@@ -472,41 +453,16 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                 for (int e = 0; e < BLK; ++e)
                     if (e >= nvalid) s[e] = -INFINITY;
             }
-            float mx;
-#if SBSA_ATTN_MAXTREE
-            {
-                // block max as a tree of three-input maxima (depth 5)
-                float t1[(BLK + 2) / 3];
+            // block max: eight independent chains of three-input maxima, then a tree
+            float mx8[8];
 #pragma unroll
-                for (int c = 0; c < BLK / 3; ++c) t1[c] = fmax3(s[3 * c], s[3 * c + 1], s[3 * c + 2]);
-                if constexpr (BLK % 3 == 1) t1[BLK / 3] = s[BLK - 1];
-                if constexpr (BLK % 3 == 2) t1[BLK / 3] = fmaxf(s[BLK - 2], s[BLK - 1]);
-                constexpr int N1 = (BLK + 2) / 3;
-                float t2[(N1 + 2) / 3];
+            for (int c = 0; c < 8; ++c) mx8[c] = fmaxf(s[c], s[c + 8]);
 #pragma unroll
-                for (int c = 0; c < N1 / 3; ++c) t2[c] = fmax3(t1[3 * c], t1[3 * c + 1], t1[3 * c + 2]);
-                if constexpr (N1 % 3 == 1) t2[N1 / 3] = t1[N1 - 1];
-                if constexpr (N1 % 3 == 2) t2[N1 / 3] = fmaxf(t1[N1 - 2], t1[N1 - 1]);
-                constexpr int N2 = (N1 + 2) / 3;
-                float r = t2[0];
+            for (int e = 16; e < BLK; e += 16)
 #pragma unroll
-                for (int c = 1; c < N2; ++c) r = fmaxf(r, t2[c]);
-                mx = r * sl2;
-            }
-#else
-            {
-                // block max: eight independent chains of three-input maxima, then a tree
-                float mx8[8];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) mx8[c] = fmaxf(s[c], s[c + 8]);
-#pragma unroll
-                for (int e = 16; e < BLK; e += 16)
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) mx8[c] = fmax3(mx8[c], s[e + c], s[e + 8 + c]);
-                mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;
-            }
-#endif
+                for (int c = 0; c < 8; ++c) mx8[c] = fmax3(mx8[c], s[e + c], s[e + 8 + c]);
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;
             // Lazy rescaling: keep the old reference max unless the block's max exceeds
             // it by more than 8 (values up to 2^8 are safe in bf16 P and fp32 O / l).
             float alpha = 1.f;
@@ -579,35 +535,17 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                 }
             };
             using I0 = std::integral_constant<int, 0>;
-            using IH = std::integral_constant<int, BLK / 2>;
             using IB = std::integral_constant<int, BLK>;
             using C0 = std::integral_constant<int, 0>;
-            using CH = std::integral_constant<int, BLK / 16>;
             using CB = std::integral_constant<int, BLK / 8>;
-            if constexpr (SBSA_ATTN_PSPLIT && BLK == 128) {
-                exps(I0{}, IH{});
-                // PV_{j-2} must be done before P buffer g is overwritten or O_g rescaled
-                if (j >= 2) {
-                    ok = wait_warp(&pv_done[g], ((j - 2) >> 1) & 1);
-                    if (!ok) continue;
-                }
-                rescale_o();
-                store_p(C0{}, CH{});
-                fence_proxy_async_smem();
-                tc_fence_before();
-                mbar_arrive(&p_half[g]);
-                exps(IH{}, IB{});
-                store_p(CH{}, CB{});
-            } else {
-                exps(I0{}, IB{});
-                // PV_{j-2} must be done before P buffer g is overwritten or O_g rescaled
-                if (j >= 2) {
-                    ok = wait_warp(&pv_done[g], ((j - 2) >> 1) & 1);
-                    if (!ok) continue;
-                }
-                store_p(C0{}, CB{});
-                rescale_o();
+            exps(I0{}, IB{});
+            // PV_{j-2} must be done before P buffer g is overwritten or O_g rescaled
+            if (j >= 2) {
+                ok = wait_warp(&pv_done[g], ((j - 2) >> 1) & 1);
+                if (!ok) continue;
             }
+            store_p(C0{}, CB{});
+            rescale_o();
             const float2 s01 = __fadd2_rn(sum4[0], sum4[1]);
             const float2 s23 = __fadd2_rn(sum4[2], sum4[3]);
             const float2 sall = __fadd2_rn(s01, s23);
