@@ -55,6 +55,11 @@
 #ifndef SBSA_POLY_EXP2_EIGHTHS
 #define SBSA_POLY_EXP2_EIGHTHS 2
 #endif
+// The same for the FP8 form, measured fastest with one eighth (2% over two at the
+// long-sequence size; the bf16 form is fastest with two: 0 and 1 are slower).
+#ifndef SBSA_POLY_EXP2_EIGHTHS_FP8
+#define SBSA_POLY_EXP2_EIGHTHS_FP8 1
+#endif
 
 // Issue order of the two MMA threads: with m > 0 the thread that issues S_j = Q K_j^T
 // waits until O += P_{j-m} V_{j-m} has been issued, which holds the Q K^T thread back so
@@ -73,7 +78,10 @@
 namespace sbsa {
 
 // Pairs (e, e+1) with e = 2 * (pair index); pair index mod 8 below EIGHTHS use the polynomial.
-__host__ __device__ constexpr bool kPolyPair(int e) { return ((e >> 1) & 7) < SBSA_POLY_EXP2_EIGHTHS; }
+template <bool FP8>
+__host__ __device__ constexpr bool kPolyPair(int e) {
+    return ((e >> 1) & 7) < (FP8 ? SBSA_POLY_EXP2_EIGHTHS_FP8 : SBSA_POLY_EXP2_EIGHTHS);
+}
 
 // 2^x on the FMA pipe for a pair, x <= 8 (x >= -125 after the clamp; smaller x give
 // ~2^-125).  Cody-Waite style split x = n + f with n = rint(x) (the 1.5*2^23 rounding
@@ -483,7 +491,7 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                     for (int e = E0; e < E1; e += 2) {
                         const float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), sl2x2, nm2);
                         float2 pr;
-                        if (kPolyPair(e)) {
+                        if (kPolyPair<FP8>(e)) {
                             pr = exp2_poly2(x);
                         } else {
                             pr.x = ex2_approx(x.x);
