@@ -21,10 +21,18 @@
 #pragma once
 #include <type_traits>
 
+// 1: the tensor-core selection's top-k counts on the floating-point pipe
+// (select_row_topk_f); 0: on the integer pipe (select_row_topk).
+#ifndef SBSA_SELECT_FCOUNT
+#define SBSA_SELECT_FCOUNT 1
+#endif
+
 #include "common.cuh"
 #include "ptx.cuh"
 
 namespace sbsa {
+
+constexpr bool kSelFloatCount = SBSA_SELECT_FCOUNT != 0;
 
 // fp32 -> uint32 with the same order (larger float -> larger key).
 __device__ __forceinline__ uint32_t order_key(float s) {
@@ -185,6 +193,144 @@ __device__ __forceinline__ void select_row_topk(const uint32_t* __restrict__ key
             bits &= bits - 1u;
         }
         base += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+    if (lane == 0) row_ptr[row] = static_cast<int32_t>(row * k_keep);
+    __syncwarp();
+}
+
+// The float whose order key is k (k the key of a finite float).
+__device__ __forceinline__ float key_float(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// select_row_topk with the row's scores kept as floats (the shared-memory row holds their
+// bit patterns): the search is the same, over the same order keys, but each probe's count
+// of keys >= cand is taken on the floating-point pipe -- key(s) >= cand exactly when
+// s > f, f the float whose key is cand - 1, and s > f exactly when (s - f) * inf
+// saturates to 1 (it gives +inf there, -inf below and NaN at equality, which saturate to
+// 1, 0 and 0) -- where the integer form spends two integer instructions per key on the
+// integer pipe, which the top-k otherwise saturates.  Non-candidates are -inf.
+template <int KPL>
+__device__ __forceinline__ void select_row_topk_f(const uint32_t* __restrict__ row_bits, int nb, int i, int k_keep,
+                                                  long long row, int32_t* __restrict__ row_ptr,
+                                                  int32_t* __restrict__ col_idx, uint32_t& hint) {
+    static_assert(KPL <= 32, "one output word per lane");
+    const int lane = threadIdx.x % 32;
+    const uint32_t lt = lanemask_lt();
+    const int kk = k_keep - 1;  // off-diagonal blocks to keep
+    float sv[KPL];
+#pragma unroll
+    for (int s = 0; s < KPL; ++s) {
+        const int j = s * 32 + lane;
+        sv[s] = (j < nb && j != i) ? __uint_as_float(row_bits[j]) : -INFINITY;
+    }
+    // The search of select_row_topk over order keys: count(key >= lo) >= k-1 > count(key >= hi).
+    uint32_t T = 0u;
+    bool exact = kk == 0;
+    if (kk > 0) {
+        float fmin = INFINITY, fmax = -INFINITY;
+        int nc = 0;
+#pragma unroll
+        for (int s = 0; s < KPL; ++s) {
+            if (sv[s] != -INFINITY) {
+                fmin = fminf(fmin, sv[s]);
+                ++nc;
+            }
+            fmax = fmaxf(fmax, sv[s]);
+        }
+        uint32_t lo = __reduce_min_sync(0xFFFFFFFFu, order_key(fmin));
+        // keys of finite scores are at most 0xFF7FFFFF, so hi = top + 1 fits in 32 bits
+        uint32_t hi = min(__reduce_max_sync(0xFFFFFFFFu, order_key(fmax)), 0xFFFFFFFEu) + 1u;
+        int c_lo = __reduce_add_sync(0xFFFFFFFFu, nc);  // candidates: count(key >= lo)
+        int c_hi = 0;
+        bool halve = false;
+        bool use_hint = hint > lo && hint < hi;
+        T = lo;
+#pragma unroll 1
+        for (int it = 0; it < 73 && hi - lo > 1u; ++it) {
+            const uint32_t range = hi - lo;
+            uint32_t cand;
+            if (use_hint) {
+                cand = hint;
+                use_hint = false;
+            } else {
+                uint32_t off;
+                if (halve) {
+                    off = range >> 1;
+                } else {
+                    const float f = __fdividef(static_cast<float>(c_lo - kk), static_cast<float>(c_lo - c_hi));
+                    off = static_cast<uint32_t>(f * static_cast<float>(range));
+                }
+                off = min(max(off, 1u), range - 1u);
+                cand = lo + off;
+            }
+            // count(key >= cand) = count(s > f): lo < cand, so cand - 1 is a finite float's key
+            const float f = key_float(cand - 1u);
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int s = 0; s < KPL; ++s) a4[s & 3] += __saturatef(__fmul_rn(__fsub_rn(sv[s], f), INFINITY));
+            const int cnt = __reduce_add_sync(0xFFFFFFFFu, __float2int_rn((a4[0] + a4[1]) + (a4[2] + a4[3])));
+            if (cnt == kk) {  // {key >= cand} is exactly the top k-1
+                T = cand;
+                exact = true;
+                break;
+            }
+            if (cnt > kk) {
+                lo = cand;
+                c_lo = cnt;
+            } else {
+                hi = cand;
+                c_hi = cnt;
+            }
+            T = lo;
+            halve = !halve && 2ull * (hi - lo) > range;
+        }
+        hint = T;
+    }
+    // Ascending output: the ballot of slot s over the lanes is the 32-block word of blocks
+    // 32 s .. 32 s + 31; lane w keeps word w.  The diagonal is added to its word.
+    uint32_t word = 0u;
+    if (exact) {
+        // keep key(s) >= T, i.e. s > the float whose key is T - 1 (T > 0 whenever k > 1)
+        const float f = kk > 0 ? key_float(T - 1u) : INFINITY;
+#pragma unroll
+        for (int s = 0; s < KPL; ++s) {
+            const uint32_t b = __ballot_sync(0xFFFFFFFFu, sv[s] > f);
+            word = lane == s ? b : word;
+        }
+    } else {
+        // keys > T kept, and keys == T lowest j first until k-1 are kept
+        int g4[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int s = 0; s < KPL; ++s) g4[s & 3] += (sv[s] != -INFINITY && order_key(sv[s]) > T) ? 1 : 0;
+        const int need_eq = kk - __reduce_add_sync(0xFFFFFFFFu, (g4[0] + g4[1]) + (g4[2] + g4[3]));
+        int eq_seen = 0;
+#pragma unroll
+        for (int s = 0; s < KPL; ++s) {
+            const bool cand = sv[s] != -INFINITY;
+            const uint32_t key = cand ? order_key(sv[s]) : 0u;
+            const bool is_eq = cand && key == T;
+            const uint32_t eq_mask = __ballot_sync(0xFFFFFFFFu, is_eq);
+            const bool keep = (cand && key > T) || (is_eq && eq_seen + __popc(eq_mask & lt) < need_eq);
+            eq_seen += __popc(eq_mask);
+            const uint32_t b = __ballot_sync(0xFFFFFFFFu, keep);
+            word = lane == s ? b : word;
+        }
+    }
+    if (lane == i / 32) word |= 1u << (i % 32);  // the diagonal
+    const int cnt = __popc(word);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    int32_t* out = col_idx + row * k_keep;
+    int pos = incl - cnt;
+    while (word) {
+        const int b = __ffs(static_cast<int>(word)) - 1;
+        out[pos++] = 32 * lane + b;
+        word &= word - 1u;
     }
     if (lane == 0) row_ptr[row] = static_cast<int32_t>(row * k_keep);
     __syncwarp();
@@ -487,7 +633,7 @@ __global__ void __launch_bounds__(kSelTcThreads, 2) select_tc_kernel(const __gri
                     const int j = 128 * t + 32 * q4 + lane;
                     if (j < NBP) {
 #pragma unroll
-                        for (int c = 0; c < HALF; ++c) keys[c * NBP + j] = order_key(__uint_as_float(v[c]));
+                        for (int c = 0; c < HALF; ++c) keys[c * NBP + j] = kSelFloatCount ? v[c] : order_key(__uint_as_float(v[c]));
                     }
                 }
             }
@@ -496,9 +642,14 @@ __global__ void __launch_bounds__(kSelTcThreads, 2) select_tc_kernel(const __gri
 #pragma unroll 1
             for (int q = 0; q < HALF / 8; ++q) {
                 const int r = r0 + warp * (HALF / 8) + q;
-                if (r < nq)
-                    select_row_topk<KPL>(keys + (r - r0) * NBP, nb, i0 + r, p.k_keep, bh * nb + i0 + r, row_ptr,
-                                         col_idx, hint);
+                if (r < nq) {
+                    if constexpr (kSelFloatCount)
+                        select_row_topk_f<KPL>(keys + (r - r0) * NBP, nb, i0 + r, p.k_keep, bh * nb + i0 + r, row_ptr,
+                                               col_idx, hint);
+                    else
+                        select_row_topk<KPL>(keys + (r - r0) * NBP, nb, i0 + r, p.k_keep, bh * nb + i0 + r, row_ptr,
+                                             col_idx, hint);
+                }
             }
             asm volatile("bar.sync 1, 256;" ::: "memory");
         }
