@@ -228,20 +228,18 @@ __device__ __forceinline__ void select_row_topk_f(const uint32_t* __restrict__ r
     uint32_t T = 0u;
     bool exact = kk == 0;
     if (kk > 0) {
+        // -inf (the non-candidates) never wins a min over the candidates' +inf start;
+        // the max of the non-candidates is -inf, below every candidate
         float fmin = INFINITY, fmax = -INFINITY;
-        int nc = 0;
 #pragma unroll
         for (int s = 0; s < KPL; ++s) {
-            if (sv[s] != -INFINITY) {
-                fmin = fminf(fmin, sv[s]);
-                ++nc;
-            }
+            fmin = fminf(fmin, sv[s] == -INFINITY ? INFINITY : sv[s]);
             fmax = fmaxf(fmax, sv[s]);
         }
         uint32_t lo = __reduce_min_sync(0xFFFFFFFFu, order_key(fmin));
         // keys of finite scores are at most 0xFF7FFFFF, so hi = top + 1 fits in 32 bits
         uint32_t hi = min(__reduce_max_sync(0xFFFFFFFFu, order_key(fmax)), 0xFFFFFFFEu) + 1u;
-        int c_lo = __reduce_add_sync(0xFFFFFFFFu, nc);  // candidates: count(key >= lo)
+        int c_lo = nb - 1;  // candidates: every block but the diagonal, count(key >= lo)
         int c_hi = 0;
         bool halve = false;
         bool use_hint = hint > lo && hint < hi;
@@ -264,12 +262,20 @@ __device__ __forceinline__ void select_row_topk_f(const uint32_t* __restrict__ r
                 off = min(max(off, 1u), range - 1u);
                 cand = lo + off;
             }
-            // count(key >= cand) = count(s > f): lo < cand, so cand - 1 is a finite float's key
+            // count(key >= cand) = count(s > f): lo < cand, so cand - 1 is a finite float's key;
+            // the differences and the sums two keys at a time (packed fp32)
             const float f = key_float(cand - 1u);
-            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+            const float2 nf2 = make_float2(-f, -f);
+            float2 a2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int s = 0; s < KPL; ++s) a4[s & 3] += __saturatef(__fmul_rn(__fsub_rn(sv[s], f), INFINITY));
-            const int cnt = __reduce_add_sync(0xFFFFFFFFu, __float2int_rn((a4[0] + a4[1]) + (a4[2] + a4[3])));
+            for (int s = 0; s + 1 < KPL; s += 2) {
+                const float2 d = __fadd2_rn(make_float2(sv[s], sv[s + 1]), nf2);
+                a2[(s >> 1) & 3] = __fadd2_rn(a2[(s >> 1) & 3], make_float2(__saturatef(__fmul_rn(d.x, INFINITY)),
+                                                                            __saturatef(__fmul_rn(d.y, INFINITY))));
+            }
+            const float2 a01 = __fadd2_rn(a2[0], a2[1]), a23 = __fadd2_rn(a2[2], a2[3]);
+            const float2 aa = __fadd2_rn(a01, a23);
+            const int cnt = __reduce_add_sync(0xFFFFFFFFu, __float2int_rn(aa.x + aa.y));
             if (cnt == kk) {  // {key >= cand} is exactly the top k-1
                 T = cand;
                 exact = true;
