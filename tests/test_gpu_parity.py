@@ -77,6 +77,29 @@ def test_select_exact_ties_prefer_lower_index(d):
     np.testing.assert_array_equal(got, ref)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_select_threshold_among_zero_scores(d):
+    """Scores exactly 0 (from +0 and -0 key means) around the k-th place: every zero ties,
+    and the lowest indices win, as in the oracle (which compares in fp64, where -0 == +0)."""
+    nb, k = 48, 15
+    qm = torch.full((1, 1, nb, d), 0.25, device="cuda")
+    km = torch.zeros(1, 1, nb, d, device="cuda")
+    km[0, 0, :10] = torch.linspace(1.0, 2.0, 10, device="cuda")[:, None]   # positive scores
+    km[0, 0, 10:20] = -0.0                                                  # -0 scores
+    km[0, 0, 30:] = -torch.linspace(1.0, 2.0, nb - 30, device="cuda")[:, None]  # negative scores
+    s = sbsa.make_shape(1, 1, nb * 64, d, 64)
+    _, ci = pu.gpu_select(s, qm, km, k)
+    sbsa.sbsa_check()
+    got = ci.cpu().numpy().reshape(1, 1, nb, k)
+    qn, kn = qm.double().cpu().numpy(), km.double().cpu().numpy()
+    ref = oracle.select(qn, kn, k)
+    if d == 128:
+        # the tensor-core path compares scores as floats after adding +0: exact agreement
+        np.testing.assert_array_equal(got, ref)
+    else:
+        pu.assert_selection_ok(got, ref, qn, kn, k)
+
+
 @pytest.mark.parametrize("scale", [1e-3, 1e4])
 def test_select_scaled_means(scale):
     """The tf32 split of the scores is exact at any magnitude: scaled means select alike."""

@@ -203,10 +203,18 @@ __device__ __forceinline__ float key_float(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
+// f with key(s) >= c exactly when s > f, for scores s that are never -0 (the caller adds
+// +0 to each): the float whose key is c - 1, stepped one key further down where that
+// float is -0, which compares equal to the score +0 whose key is c.
+__device__ __forceinline__ float float_below_key(uint32_t c) {
+    const uint32_t k = c - 1u;
+    return key_float(k == 0x7FFFFFFFu ? k - 1u : k);
+}
+
 // select_row_topk with the row's scores kept as floats (the shared-memory row holds their
 // bit patterns): the search is the same, over the same order keys, but each probe's count
 // of keys >= cand is taken on the floating-point pipe -- key(s) >= cand exactly when
-// s > f, f the float whose key is cand - 1, and s > f exactly when (s - f) * inf
+// s > f, f = float_below_key(cand), and s > f exactly when (s - f) * inf
 // saturates to 1 (it gives +inf there, -inf below and NaN at equality, which saturate to
 // 1, 0 and 0) -- where the integer form spends two integer instructions per key on the
 // integer pipe, which the top-k otherwise saturates.  Non-candidates are -inf.
@@ -222,7 +230,8 @@ __device__ __forceinline__ void select_row_topk_f(const uint32_t* __restrict__ r
 #pragma unroll
     for (int s = 0; s < KPL; ++s) {
         const int j = s * 32 + lane;
-        sv[s] = (j < nb && j != i) ? __uint_as_float(row_bits[j]) : -INFINITY;
+        // + 0 turns a -0 score into +0, so that float order and key order agree
+        sv[s] = (j < nb && j != i) ? __fadd_rn(__uint_as_float(row_bits[j]), 0.f) : -INFINITY;
     }
     // The search of select_row_topk over order keys: count(key >= lo) >= k-1 > count(key >= hi).
     uint32_t T = 0u;
@@ -264,7 +273,7 @@ __device__ __forceinline__ void select_row_topk_f(const uint32_t* __restrict__ r
             }
             // count(key >= cand) = count(s > f): lo < cand, so cand - 1 is a finite float's key;
             // the differences and the sums two keys at a time (packed fp32)
-            const float f = key_float(cand - 1u);
+            const float f = float_below_key(cand);
             const float2 nf2 = make_float2(-f, -f);
             float2 a2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
@@ -298,7 +307,7 @@ __device__ __forceinline__ void select_row_topk_f(const uint32_t* __restrict__ r
     uint32_t word = 0u;
     if (exact) {
         // keep key(s) >= T, i.e. s > the float whose key is T - 1 (T > 0 whenever k > 1)
-        const float f = kk > 0 ? key_float(T - 1u) : INFINITY;
+        const float f = kk > 0 ? float_below_key(T) : INFINITY;
 #pragma unroll
         for (int s = 0; s < KPL; ++s) {
             const uint32_t b = __ballot_sync(0xFFFFFFFFu, sv[s] > f);
