@@ -162,6 +162,7 @@ struct AttnParams {
     unsigned int epoch;
     const float* q_scale;  // FP8 form: per (b, h, block) scales of the codes
     const float* k_scale;
+    int prefetch_dist;     // units ahead whose Q tile is prefetched into L2 (0: none; the SM count)
 };
 
 // e4m3 x e4m3 -> fp32 instruction descriptor (format 0 = E4M3 for both operands).
@@ -282,6 +283,15 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
 #pragma unroll
             for (int a = 0; a < C::kQKAtoms; ++a)
                 tma_load_2d(sQ + a * 128 * 128, &map_q, q_full, a * C::kQKElemsPerAtom, row0 + qb * BLK, pol_q);
+            // The unit that starts about one CTA lifetime from now (one CTA per SM, units
+            // dispatched in order) is unit + prefetch_dist: its Q tile is brought into L2
+            // now, so that its first load does not wait for HBM
+            const long long u2 = unit + p.prefetch_dist;
+            if (p.prefetch_dist > 0 && u2 < p.units) {
+                const int row2 = static_cast<int>((u2 / p.nb) * p.Lp + (u2 % p.nb) * BLK);
+#pragma unroll
+                for (int a = 0; a < C::kQKAtoms; ++a) tma_prefetch_l2_2d(&map_q, a * C::kQKElemsPerAtom, row2);
+            }
             int kseq = 0, vseq = 0;
             auto load = [&](int j, bool is_v) -> bool {
                 int& seq = is_v ? vseq : kseq;

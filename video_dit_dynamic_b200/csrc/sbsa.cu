@@ -358,6 +358,7 @@ sbsa_status launch_attn_t(const sbsa_shape* s, const void* q, const void* k, con
     p.epoch = g_epoch.fetch_add(1);
     p.q_scale = q_scale;
     p.k_scale = k_scale;
+    p.prefetch_dist = sm_count();
     auto kern = attn_kernel<D, BLK, FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "attention smem attribute");
