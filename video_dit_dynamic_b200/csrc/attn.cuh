@@ -33,8 +33,14 @@
 //   pv_done[b] PV_j done (commit)          -> P buffer b is free and O_b is stable
 //
 // TMEM columns: S buffers at 0 and 128 (BLK fp32 columns each), O_0 at 256 and O_1 at
-// 384 (D columns each).  For BLK = 64 the 128-row Q tile also holds the next block's
-// 64 rows; those rows are computed and discarded.
+// 384 (D columns each).
+//
+// BLK = 64 (bf16): a CTA takes two neighbouring query blocks, qa = 2i and qa + 1, as the
+// two halves of its 128-row tile.  When both kept lists are strictly ascending, in range
+// and short enough, the CTA walks their union once (a key block kept by both is
+// computed once for all 128 rows); otherwise it walks list a and then list b.  Each
+// entry carries which row halves it serves; the rows of the other half see it fully
+// masked.  (Unpaired, half of every 128-row product would be for rows discarded.)
 //
 // Every wait is bounded (the pipeline limit, 1 s unless a test lowered it); a wait that
 // runs out latches SBSA_ERR_TIMEOUT, makes every CTA of the launch give up, drains this
@@ -140,7 +146,13 @@ struct AttnCfg {
     // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2],
     // s_free[2], p_full[2], pv_done[2], drain[2], pv_issued[4]
     static constexpr int kNumBars = 1 + 4 * kStages + 2 * 5 + 4;
-    static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // + tmem slot, flag, alignment slack
+    // paired query blocks (BLK = 64, bf16): the kept lists copied to shared memory and
+    // their union, when each list holds at most kListCap entries
+    static constexpr bool kPaired = BLK == 64 && !FP8;
+    static constexpr int kListCap = kPaired ? 256 : 0;
+    static constexpr int kSeqOff = kBarOff + kNumBars * 8 + 16;  // after the tmem slot and flag
+    static constexpr int kSeqBytes = kPaired ? (4 * kListCap + 4) * 4 : 0;  // union, two lists, mode and length
+    static constexpr int kSmemBytes = kSeqOff + kSeqBytes + 1024;  // + alignment slack
     static constexpr int kThreads = 352;
     static constexpr uint32_t kColS0 = 0, kColO0 = 256;  // S_b at b*128, O_g at 256 + g*128
     static_assert(kStages >= 2, "need at least two slots per ring");
@@ -163,6 +175,7 @@ struct AttnParams {
     const float* q_scale;  // FP8 form: per (b, h, block) scales of the codes
     const float* k_scale;
     int prefetch_dist;     // units ahead whose Q tile is prefetched into L2 (0: none; the SM count)
+    int units_per_bh;      // units per (b, h): nb, or ceil(nb / 2) with paired query blocks
 };
 
 // e4m3 x e4m3 -> fp32 instruction descriptor (format 0 = E4M3 for both operands).
@@ -220,13 +233,28 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
     if (__syncthreads_or(launch_aborted(p.epoch) ? 1 : 0)) return;
 
     const long long unit = blockIdx.x;
-    const long long bh = unit / p.nb;
-    const int qb = static_cast<int>(unit % p.nb);
-    int rs = __ldg(p.row_ptr + unit);
-    int re = __ldg(p.row_ptr + unit + 1);
-    const bool bad_row = rs < 0 || re < rs;
-    if (bad_row) re = rs = 0;
-    const int n = re - rs;
+    const long long bh = unit / p.units_per_bh;
+    // first query block of the tile (paired: qb and qb + 1, when qb + 1 exists)
+    const int qb = static_cast<int>(unit % p.units_per_bh) * (C::kPaired ? 2 : 1);
+    const bool has_b = C::kPaired && qb + 1 < p.nb;
+    const long long row_a = bh * p.nb + qb;
+    int rs = __ldg(p.row_ptr + row_a);
+    int re = __ldg(p.row_ptr + row_a + 1);
+    bool bad_row = rs < 0 || re < rs;
+    if (rs < 0 || re < rs) re = rs = 0;
+    int rs2 = 0, re2 = 0;  // the second query block's list (paired)
+    if (has_b) {
+        rs2 = __ldg(p.row_ptr + row_a + 1);
+        re2 = __ldg(p.row_ptr + row_a + 2);
+        if (rs2 < 0 || re2 < rs2) {
+            bad_row = true;
+            re2 = rs2 = 0;
+        }
+    }
+    uint32_t* seq = reinterpret_cast<uint32_t*>(smem + C::kSeqOff);  // union: block | halves << 30
+    int* list_a = reinterpret_cast<int*>(seq + 2 * C::kListCap);
+    int* list_b = list_a + C::kListCap;
+    int* seq_info = list_b + C::kListCap;  // [0] 1 = walk the union, [1] entries
 
     if (tid == 256) {
         *abort_flag = 0;
@@ -255,10 +283,78 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
+    if constexpr (C::kPaired) {
+        if (warp == 8) {
+            // the union of the two kept lists, when both are strictly ascending, in range
+            // and at most kListCap long (uniform over the warp)
+            const int na = re - rs, nb2 = re2 - rs2;
+            bool use_union = na <= C::kListCap && nb2 <= C::kListCap;
+            if (use_union) {
+                bool good = true;
+                for (int i = (tid & 31); i < na; i += 32) {
+                    const int v = __ldg(p.col_idx + rs + i);
+                    list_a[i] = v;
+                    good = good && v >= 0 && v < p.nb && (i == 0 || __ldg(p.col_idx + rs + i - 1) < v);
+                }
+                for (int i = (tid & 31); i < nb2; i += 32) {
+                    const int v = __ldg(p.col_idx + rs2 + i);
+                    list_b[i] = v;
+                    good = good && v >= 0 && v < p.nb && (i == 0 || __ldg(p.col_idx + rs2 + i - 1) < v);
+                }
+                use_union = __all_sync(0xFFFFFFFFu, good);
+            }
+            __syncwarp();
+            if ((tid & 31) == 0) {
+                int o = na + nb2;
+                if (use_union) {
+                    // merge; every step takes one entry of a or of b or both
+                    int i = 0, k2 = 0;
+                    o = 0;
+                    while (i < na || k2 < nb2) {
+                        uint32_t v, halves;
+                        if (k2 >= nb2 || (i < na && list_a[i] < list_b[k2])) {
+                            v = static_cast<uint32_t>(list_a[i++]);
+                            halves = 1u;
+                        } else if (i >= na || list_b[k2] < list_a[i]) {
+                            v = static_cast<uint32_t>(list_b[k2++]);
+                            halves = 2u;
+                        } else {
+                            v = static_cast<uint32_t>(list_a[i]);
+                            ++i;
+                            ++k2;
+                            halves = 3u;
+                        }
+                        seq[o++] = v | (halves << 30);
+                    }
+                }
+                seq_info[0] = use_union ? 1 : 0;
+                seq_info[1] = o;
+            }
+        }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // kept entries of this CTA and, for entry j, its key block and the row halves it
+    // serves (bit h: rows 64 h .. 64 h + 63; both bits unpaired)
+    const bool walk_union = C::kPaired && seq_info[0] != 0;
+    const int n = C::kPaired ? seq_info[1] : re - rs;
+    auto entry = [&](int j, uint32_t& halves) -> int {
+        if constexpr (C::kPaired) {
+            if (walk_union) {
+                const uint32_t e = seq[j];
+                halves = e >> 30;
+                return static_cast<int>(e & 0x3FFFFFFFu);
+            }
+            const int na = re - rs;
+            halves = j < na ? 1u : 2u;
+            return j < na ? __ldg(p.col_idx + rs + j) : __ldg(p.col_idx + rs2 + (j - na));
+        } else {
+            halves = 3u;
+            return __ldg(p.col_idx + rs + j);
+        }
+    };
 
     auto give_up = [&]() {
         *abort_flag = 1;
@@ -288,7 +384,8 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
             // now, so that its first load does not wait for HBM
             const long long u2 = unit + p.prefetch_dist;
             if (p.prefetch_dist > 0 && u2 < p.units) {
-                const int row2 = static_cast<int>((u2 / p.nb) * p.Lp + (u2 % p.nb) * BLK);
+                const int qb2 = static_cast<int>(u2 % p.units_per_bh) * (C::kPaired ? 2 : 1);
+                const int row2 = static_cast<int>((u2 / p.units_per_bh) * p.Lp + qb2 * BLK);
 #pragma unroll
                 for (int a = 0; a < C::kQKAtoms; ++a) tma_prefetch_l2_2d(&map_q, a * C::kQKElemsPerAtom, row2);
             }
@@ -298,7 +395,8 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
                 const int slot = seq % NS;
                 const uint32_t ph = (seq / NS) & 1;
                 if (!wait(is_v ? &v_empty[slot] : &k_empty[slot], ph ^ 1)) return false;
-                int blk = __ldg(p.col_idx + rs + j);
+                uint32_t halves;
+                int blk = entry(j, halves);
                 if (blk < 0 || blk >= p.nb) blk = 0;  // masked by the softmax warps
                 uint8_t* dst = is_v ? sV + slot * C::kVTile : sK + slot * C::kKTile;
                 uint64_t* full = is_v ? &v_full[slot] : &k_full[slot];
@@ -409,7 +507,8 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
         const int r = tid & 127;     // row within the 128-row tile
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const int t = qb * BLK + r;
-        const bool row_in_block = r < BLK;
+        const bool row_in_block = r < BLK || has_b;  // paired: rows BLK.. are block qb + 1
+        const uint32_t my_half = static_cast<uint32_t>(r >= 64 ? 2 : 1);
         const bool row_valid = row_in_block && t < p.L;
         // logit scale |scale| * log2(e) > 0; the FP8 form also folds in this query
         // block's scale here and each key block's scale below
@@ -430,17 +529,19 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
             const bool w = wait(bar, parity);
             return __all_sync(0xFFFFFFFFu, w);
         };
-        int blk_next = g < n ? __ldg(p.col_idx + rs + g) : 0;
+        uint32_t halves_next = 3u;
+        int blk_next = g < n ? entry(g, halves_next) : 0;
         float ks_next = 1.f;
         if constexpr (FP8) {
             if (g < n && blk_next >= 0 && blk_next < p.nb) ks_next = __ldg(p.k_scale + bh * p.nb + blk_next);
         }
         for (int j = g; j < n; j += 2) {
             const int blk = blk_next;
+            const uint32_t halves = halves_next;
             const float sl2 = sl2_q * ks_next;
             const float2 sl2x2 = make_float2(sl2, sl2);
             if (j + 2 < n) {
-                blk_next = __ldg(p.col_idx + rs + j + 2);
+                blk_next = entry(j + 2, halves_next);
                 if constexpr (FP8) {
                     ks_next = (blk_next >= 0 && blk_next < p.nb) ? __ldg(p.k_scale + bh * p.nb + blk_next) : 1.f;
                 }
@@ -450,7 +551,9 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
             tc_fence_after();
             const bool bad = blk < 0 || blk >= p.nb;
             if (bad && r == 0) raise_error(kErrBadIndex);
-            const int nvalid = bad ? 0 : min(BLK, p.L - blk * BLK);  // valid keys of the block
+            // valid keys of the block for this row: none when the entry does not serve its
+            // half of the tile (uniform per warp: a warp's 32 rows lie in one half)
+            const int nvalid = (bad || (halves & my_half) == 0) ? 0 : min(BLK, p.L - blk * BLK);
             float s[BLK];
             {
                 uint32_t raw[BLK];
@@ -465,7 +568,7 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
 #pragma unroll
                 for (int e = 0; e < BLK; ++e) s[e] = -s[e];
             }
-            const bool masked = nvalid < BLK;  // padded tail block or skipped index (uniform)
+            const bool masked = nvalid < BLK;  // padded tail, skipped index or other half (warp-uniform)
             if (masked) {
 #pragma unroll
                 for (int e = 0; e < BLK; ++e)

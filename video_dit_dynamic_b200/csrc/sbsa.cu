@@ -349,7 +349,9 @@ sbsa_status launch_attn_t(const sbsa_shape* s, const void* q, const void* k, con
     p.row_ptr = rp;
     p.col_idx = ci;
     p.o = static_cast<__nv_bfloat16*>(o);
-    p.units = num_rows(s);
+    // paired query blocks (block 64): one unit per two neighbouring query blocks
+    p.units_per_bh = C::kPaired ? (num_blocks(s) + 1) / 2 : num_blocks(s);
+    p.units = static_cast<long long>(s->batch) * s->heads * p.units_per_bh;
     p.L = s->seq_len;
     p.Lp = s->seq_len_padded;
     p.nb = num_blocks(s);
