@@ -35,7 +35,7 @@
 // TMEM columns: S buffers at 0 and 128 (BLK fp32 columns each), O_0 at 256 and O_1 at
 // 384 (D columns each).
 //
-// BLK = 64 (bf16): a CTA takes two neighbouring query blocks, qa = 2i and qa + 1, as the
+// BLK = 64: a CTA takes two neighbouring query blocks, qa = 2i and qa + 1, as the
 // two halves of its 128-row tile.  When both kept lists are strictly ascending, in range
 // and short enough, the CTA walks their union once (a key block kept by both is
 // computed once for all 128 rows); otherwise it walks list a and then list b.  Each
@@ -146,9 +146,9 @@ struct AttnCfg {
     // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2],
     // s_free[2], p_full[2], pv_done[2], drain[2], pv_issued[4]
     static constexpr int kNumBars = 1 + 4 * kStages + 2 * 5 + 4;
-    // paired query blocks (BLK = 64, bf16): the kept lists copied to shared memory and
-    // their union, when each list holds at most kListCap entries
-    static constexpr bool kPaired = BLK == 64 && !FP8;
+    // paired query blocks (BLK = 64): the kept lists copied to shared memory and their
+    // union, when each list holds at most kListCap entries
+    static constexpr bool kPaired = BLK == 64;
     static constexpr int kListCap = kPaired ? 256 : 0;
     static constexpr int kSeqOff = kBarOff + kNumBars * 8 + 16;  // after the tmem slot and flag
     static constexpr int kSeqBytes = kPaired ? (4 * kListCap + 4) * 4 : 0;  // union, two lists, mode and length
@@ -512,7 +512,8 @@ __global__ void __launch_bounds__(352, 1) attn_kernel(const __grid_constant__ CU
         const bool row_valid = row_in_block && t < p.L;
         // logit scale |scale| * log2(e) > 0; the FP8 form also folds in this query
         // block's scale here and each key block's scale below
-        const float sl2_q = FP8 ? p.scale_log2 * __ldg(p.q_scale + unit) : p.scale_log2;
+        // (paired: rows BLK.. belong to query block qb + 1, whose scale is the next one)
+        const float sl2_q = FP8 ? p.scale_log2 * __ldg(p.q_scale + row_a + (r >= BLK && has_b ? 1 : 0)) : p.scale_log2;
         const uint32_t s_col = tmem + lane_base + C::kColS0 + g * 128;
         const uint32_t o_col = tmem + lane_base + C::kColO0 + g * 128;
         // this row of P_g: 128-byte rows, 16-byte chunks swizzled by (row mod 8), one
