@@ -34,6 +34,15 @@ def test_forward_full_size(name):
     _check_forward(inputs.WORKLOADS[name], n_units=64, full_head=name != "long122880")
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_forward_full_size_block64(d):
+    """Blocks of 64 on the 480p grid (512 blocks, keep 20%): the attention runs as paired
+    128-row tiles over the union of two query blocks' kept lists; every mean and selection,
+    a whole head and 64 sampled units against the oracle."""
+    wl = inputs.Workload("480p_b64_d%d" % d, 1, 40 if d == 128 else 24, (21, 30, 52), d, 64, 0.2)
+    _check_forward(wl, n_units=64, full_head=True)
+
+
 @pytest.mark.parametrize("keep", [1.0, 0.5, 0.3, 0.2, 0.1])
 def test_forward_keep_sweep(keep):
     """The keep-fraction sweep at L = 32,768 (keep = 1 is dense attention from the same kernel)."""
