@@ -48,8 +48,16 @@ def _sample_units(H, nb, n, seed):
 
 
 # ---------------------------------------------------------------------------- FP8 path
-def test_fp8_path_full_size(sbsa):
-    wl = inputs.WORKLOADS["long122880"]
+_FP8_WORKLOADS = {
+    "long122880": inputs.WORKLOADS["long122880"],
+    # blocks of 64 on the 480p grid: the attention runs as paired 128-row tiles
+    "480p_b64": inputs.Workload("480p_b64", 1, 40, (21, 30, 52), 128, 64, 0.2),
+}
+
+
+@pytest.mark.parametrize("name", list(_FP8_WORKLOADS))
+def test_fp8_path_full_size(sbsa, name):
+    wl = _FP8_WORKLOADS[name]
     B, H, d, blk = wl.batch, wl.heads, wl.head_dim, wl.block
     L, Lp, nb = wl.seq_len, wl.seq_len_padded, wl.num_blocks
     kk = sbsa.sbsa_keep_blocks(nb, wl.keep)
@@ -105,7 +113,7 @@ def test_fp8_path_full_size(sbsa):
         ref[idx] = oracle.attention_fp8(qc[:, h:h + 1], qsc[:, h:h + 1], kc[:, h:h + 1], ksc[:, h:h + 1],
                                         vb[:, h:h + 1], L, blk, oracle.uniform_row_ptr(1, 1, nb, kk),
                                         col[:, h:h + 1], units=loc)
-    pu.assert_attention_close(got, ref, "fp8 attention, long-sequence sampled units")
+    pu.assert_attention_close(got, ref, "fp8 attention, %s sampled units" % name)
 
 
 # ---------------------------------------------------------------------------- RoPE + pool
