@@ -192,6 +192,20 @@ def test_attention_explicit_scale():
     pu.assert_attention_close(o, ref, "scale=0.05")
 
 
+@pytest.mark.parametrize("d,blk", [(128, 128), (64, 64), (128, 64)])
+def test_attention_negative_scale(d, blk):
+    """A negative logit scale (the logits are -|scale|.S: the softmax favours the lowest
+    scores), through the unpaired and the paired (block 64) tiles."""
+    L = 9 * blk - 13
+    q, k, v = inputs.random_qkv(1, 2, 9 * blk, d, L=L, seed=36, device="cuda")
+    rp, col, _, _ = _oracle_mask(q, k, L, blk, 3)
+    s = pu.shape_of(q, L, blk)
+    o = pu.gpu_attention(s, q, k, v, torch.from_numpy(rp).cuda(), torch.from_numpy(col.reshape(-1)).cuda(),
+                         scale=-0.09)
+    ref = oracle.attention(pu.bits(q), pu.bits(k), pu.bits(v), L, blk, rp, col, scale=-0.09)
+    pu.assert_attention_close(o, ref, "scale=-0.09")
+
+
 @pytest.mark.parametrize("d,blk", [(128, 128), (64, 64)])
 def test_attention_variable_and_empty_rows(d, blk):
     H, nb = 2, 9
