@@ -334,6 +334,38 @@ def test_forward_from_host_chunked_pipeline(head_chunk):
         assert torch.equal(oh, ref)
 
 
+@pytest.mark.parametrize("d,blk", [(128, 128), (128, 64), (64, 64)])
+def test_forward_batch_two(d, blk):
+    """B = 2: sbsa_forward (pool, select, attention) over two batch entries of three heads
+    against the oracle on the whole output, and sbsa_forward_host chunked over the six
+    (batch, head) pairs bit-equal to it."""
+    B, H = 2, 3
+    L = 11 * blk - 9
+    s = sbsa.make_shape(B, H, L, d, blk)
+    q, k, v = inputs.random_qkv(B, H, s.seq_len_padded, d, L=L, seed=37)
+    kk = sbsa.sbsa_keep_blocks(s.num_blocks, 0.3)
+    o = torch.empty_like(q, device="cuda")
+    col = torch.empty(B * H * s.num_blocks * kk, dtype=torch.int32, device="cuda")
+    sbsa.sbsa_forward(s, q.cuda(), k.cuda(), v.cuda(), kk, 0.0, o, col, sbsa.alloc_workspace(s, kk))
+    sbsa.sbsa_check()
+    qb, kb, vb = pu.bits(q), pu.bits(k), pu.bits(v)
+    qm, km = oracle.pool(qb, L, blk), oracle.pool(kb, L, blk)
+    ref_col = oracle.select(qm, km, kk)
+    pu.assert_selection_ok(col.cpu().numpy().reshape(ref_col.shape), ref_col, qm, km, kk)
+    rp = oracle.uniform_row_ptr(B, H, s.num_blocks, kk)
+    ref = oracle.attention(qb, kb, vb, L, blk, rp, col.cpu().numpy())
+    pu.assert_attention_close(o, ref, "B = 2")
+    oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    dq, dk, dv, do = (torch.empty_like(o) for _ in range(4))
+    st = torch.cuda.current_stream()
+    sbsa.sbsa_forward_host(s, q.pin_memory(), k.pin_memory(), v.pin_memory(), kk, 0.0, oh, dq, dk, dv, do,
+                           sbsa.alloc_workspace(s, kk), pairs_per_chunk=2, stream=st,
+                           h2d_stream=torch.cuda.Stream(), d2h_stream=torch.cuda.Stream())
+    st.synchronize()
+    sbsa.sbsa_check()
+    assert torch.equal(oh, o.cpu())
+
+
 @pytest.mark.parametrize("pinned,copy_streams", [(True, True), (False, False)])
 def test_forward_host_entry_point(pinned, copy_streams):
     """sbsa_forward_host through the C ABI: pinned host memory with separate copy streams,
