@@ -231,6 +231,24 @@ def test_attention_variable_and_empty_rows(d, blk):
     sbsa.sbsa_check()
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_attention_unsorted_and_repeated_lists(d):
+    """Lists in any order, with repeats (a block listed twice counts twice, as in the
+    oracle), at blocks of 128."""
+    blk, H, nb = 128, 2, 7
+    L = nb * blk - 3
+    q, k, v = inputs.random_qkv(1, H, nb * blk, d, L=L, seed=38, device="cuda")
+    rng = np.random.default_rng(39)
+    rows = [rng.integers(0, nb, size=int(rng.integers(1, 9))).tolist() for _ in range(H * nb)]
+    rp = np.cumsum([0] + [len(x) for x in rows]).astype(np.int32)
+    ci = np.array([j for x in rows for j in x], dtype=np.int32)
+    s = pu.shape_of(q, L, blk)
+    o = pu.gpu_attention(s, q, k, v, torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda())
+    sbsa.sbsa_check()
+    ref = oracle.attention(pu.bits(q), pu.bits(k), pu.bits(v), L, blk, rp, ci)
+    pu.assert_attention_close(o, ref, "unsorted, repeated")
+
+
 def test_attention_out_of_range_index_is_skipped_and_reported():
     d, blk, nb = 64, 64, 6
     L = nb * blk
