@@ -142,8 +142,9 @@ sbsa_status sbsa_select_blocks(const sbsa_shape *shape, const float *q_mean, con
  * key, are written as 0.
  *   q, k, v : bf16 [B][H][Lp][d] (device).
  *   row_ptr : int32 [B*H*nb + 1], non-decreasing, row_ptr[0] == 0; any list length.
- *   col_idx : int32 key-block indices in [0, nb).  An index outside that range is
- *             skipped (contributes nothing) and latches SBSA_ERR_BAD_INDEX.
+ *   col_idx : int32 key-block indices in [0, nb), in any order; a block listed twice
+ *             contributes its keys twice.  An index outside that range is skipped
+ *             (contributes nothing) and latches SBSA_ERR_BAD_INDEX.
  *   scale   : logit scale; 0 means 1/sqrt(head_dim).
  *   o       : bf16 [B][H][Lp][d] (device, written).
  * Arithmetic: bf16 tensor-core products (tcgen05) with fp32 accumulation, fp32 online
